@@ -1,0 +1,445 @@
+"""CPU oracle for SageSLA attention (INT8 block-quantised, top-k block-sparse
+softmax attention plus a linear-attention branch for the blocks not picked).
+
+TEST INFRASTRUCTURE ONLY.  This module is the slow, plain statement of what
+the CUDA path computes.  Only the tests, the package's smoke check and the
+benchmark's CPU-baseline leg may import it; the library itself never does,
+and it shares no code with the CUDA sources.
+
+Sources.  The pages describe the method only in prose:
+
+[P1] "Turbo Diffusion：秒级生成与高清保真的视频扩散技术突破" (lanhy.cn),
+     section 三(一) SageAttention2++ items 1-3 (outlier smoothing, per-sub-block
+     quantisation parameters, 128x128 tensor-core tiles with a parallel
+     softmax) and section 三(二) SLA items 1-3 (top-K 10% selection of the
+     important regions, an O(N) linear branch with a linear projection, and
+     SageSLA = SLA selection followed by INT8 computation on the kept part).
+[P3] "TurboDiffusion技术指南：突破视频生成效率瓶颈的实践方案" (blog.gitcode.com),
+     section "SageSLA：注意力机制的'瘦身'专家" and the T2V parameter list
+     (``--sla_topk 0.1`` keeps 10%).
+[P4] "TurboDiffusion: 即時AI影片生成的重大突破" (bonega.ai), section
+     "SLA: 稀疏線性注意力" (sparse where full attention is not needed, near
+     linear cost elsewhere).
+
+The pages fix no formula, precision, layout or tie rule.  The precise
+semantics below are the readings this project adopts (each stated where it is
+used); every function says which passage it follows.
+
+Notation: inputs are bf16 bit patterns, uint16 arrays Q, K, V [B, H, N, d] and
+W_proj [d, d]; ``block`` tokens per block; nblk = ceil(N / block); block r
+covers rows [r*block, min(N, (r+1)*block)).
+
+Parity status: every function here is pinned by a test in
+tests/test_oracle_pins.py against a closed form, a library routine, a brute
+force or a hand-derived case, except the choice of raw K (rather than
+smoothed K) inside phi(K) for the linear branch, which no passage decides
+("parity unpinned" for that choice; see the linear_states docstring).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+NEAR_TIE_REL = 1e-9
+
+
+# ---------------------------------------------------------------------------
+# number formats
+# ---------------------------------------------------------------------------
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> exact float64 values."""
+    u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> exact float32 values."""
+    u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32)
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value, ties to even.
+
+    bf16 keeps 8 significant bits.  With x = m * 2**e, 0.5 <= |m| < 1
+    (frexp), the spacing of bf16 values near x is 2**(e-8); below the
+    smallest normal (2**-126) the spacing stays 2**-133.  Scaling by a power
+    of two is exact, so rint (half to even) does the only rounding.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    e = np.maximum(e, -125)
+    y = np.ldexp(np.rint(np.ldexp(x, 8 - e)), e - 8)
+    big = np.abs(y) > 3.3895313892515355e38  # beyond the largest finite bf16
+    return np.where(big, np.copysign(np.inf, x), y)
+
+
+def round_rational_to_f32(num: int, den: int) -> float:
+    """The float32 nearest to num/den (exact integers, den > 0), ties to even."""
+    if den <= 0:
+        raise ValueError("den must be positive")
+    if num == 0:
+        return 0.0
+    sign = -1.0 if num < 0 else 1.0
+    a = abs(num)
+
+    def split(e):
+        if e >= 0:
+            q, r = divmod(a, den << e)
+            return q, r, den << e
+        q, r = divmod(a << (-e), den)
+        return q, r, den
+
+    e = a.bit_length() - den.bit_length() - 24
+    while True:
+        q, r, dd = split(e)
+        if q >= (1 << 24):
+            e += 1
+        elif q < (1 << 23) and e > -149:
+            e -= 1
+        else:
+            break
+    if e < -149:                        # subnormal float32: fixed spacing 2**-149
+        e = -149
+        q, r, dd = split(e)
+    if 2 * r > dd or (2 * r == dd and (q & 1)):
+        q += 1
+    return sign * math.ldexp(q, e)
+
+
+def topk_count(nblk: int, topk_frac: float) -> int:
+    """Number of key blocks kept per query block: ceil(topk_frac * nblk) in [1, nblk].
+
+    [P1] section 三(二) item 1 keeps the top K = 10% and [P3] reads
+    ``--sla_topk 0.1`` as 10%.  Reading: the fraction is taken as the float32
+    value the C interface receives, multiplied by nblk exactly (in float64),
+    rounded up, and clamped to [1, nblk].
+    """
+    f = float(np.float32(topk_frac))
+    if not (f > 0.0 and f <= 1.0):
+        raise ValueError("topk_frac must be in (0, 1]")
+    kc = math.ceil(f * nblk)
+    return min(nblk, max(1, kc))
+
+
+# ---------------------------------------------------------------------------
+# smoothing and quantisation  ([P1] section 三(一) items 1 and 2)
+# ---------------------------------------------------------------------------
+
+def channel_mean(k_bits: np.ndarray) -> np.ndarray:
+    """mu[b, h, c] = float32 nearest to the exact mean of K[b, h, :, c] over all N tokens.
+
+    [P1] section 三(一) item 1 smooths outliers before quantising while keeping
+    the overall distribution; the reading adopted is subtraction of the
+    per-channel mean over tokens.  Reading: the mean is exact (the sum is
+    formed without any rounding) and rounded once to float32, ties to even.
+
+    A bf16 value is sig * 2**(E - 134) with an integer significand sig
+    (|sig| < 256) and E = max(exponent field, 1).  Integer significands are
+    accumulated per exponent (np.bincount; each partial sum is an integer of
+    magnitude below 2**53, so its float64 accumulation is exact) and then
+    combined as a Python integer multiple of 2**-133.
+    """
+    k = np.asarray(k_bits, dtype=np.uint16)
+    B, H, N, d = k.shape
+    mu = np.empty((B, H, d), dtype=np.float32)
+    for b in range(B):
+        for h in range(H):
+            bits = k[b, h].astype(np.int64)
+            expo = (bits >> 7) & 0xFF
+            if np.any(expo == 0xFF):
+                raise ValueError("K holds Inf/NaN")
+            frac = bits & 0x7F
+            sig = np.where(expo > 0, frac + 128, frac)
+            sig = np.where((bits >> 15) & 1, -sig, sig)
+            e = np.maximum(expo, 1)
+            key = np.arange(d, dtype=np.int64)[None, :] * 256 + e
+            counts = np.bincount(key.ravel(), weights=sig.ravel().astype(np.float64),
+                                 minlength=d * 256).reshape(d, 256)
+            for c in range(d):
+                total = 0
+                for ee in np.nonzero(counts[c])[0]:
+                    total += int(counts[c, ee]) << (int(ee) - 1)   # units of 2**-133
+                mu[b, h, c] = round_rational_to_f32(total, N << 133)
+    return mu
+
+
+def smooth_k(k_bits: np.ndarray, mu: np.ndarray) -> np.ndarray:
+    """K_s = float32(K) - mu, one float32 rounding per element ([P1] 三(一) item 1).
+
+    Q is not smoothed.  Reading: smoothing serves the quantisation only; the
+    pooled mask and the linear branch use the raw K.
+    """
+    return bf16_to_f32(k_bits) - mu[:, :, None, :].astype(np.float32)
+
+
+def quantize_blocks(x32: np.ndarray, block: int) -> tuple[np.ndarray, np.ndarray]:
+    """Symmetric INT8 quantisation with one float32 scale per block of tokens.
+
+    [P1] section 三(一) item 2: each sub-block gets its own quantisation
+    parameters.  Readings: a block is ``block`` consecutive tokens by all d
+    channels (the same blocks as the sparse mask); m = max |x| over the
+    block's valid rows; scale s = float32(m / 127) (IEEE division);
+    x_i8 = clamp(round_half_even(float32(x / s)), -127, 127); a block with
+    m = 0 has s = 0 and all-zero codes.  Output rows past N (up to
+    nblk * block) are zero.
+
+    Returns (codes int8 [B, H, nblk*block, d], scales float32 [B, H, nblk]).
+    """
+    x32 = np.asarray(x32, dtype=np.float32)
+    B, H, N, d = x32.shape
+    nblk = (N + block - 1) // block
+    codes = np.zeros((B, H, nblk * block, d), dtype=np.int8)
+    scales = np.zeros((B, H, nblk), dtype=np.float32)
+    for r in range(nblk):
+        lo, hi = r * block, min(N, (r + 1) * block)
+        xb = x32[:, :, lo:hi, :]
+        m = np.max(np.abs(xb), axis=(2, 3))                      # float32, exact
+        s = (m / np.float32(127.0)).astype(np.float32)           # IEEE float32 division
+        scales[:, :, r] = s
+        safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+        qf = (xb / safe[:, :, None, None]).astype(np.float32)    # float32 quotient
+        qi = np.clip(np.rint(qf), -127, 127)                     # half to even
+        qi = np.where(s[:, :, None, None] > 0, qi, 0)
+        codes[:, :, lo:hi, :] = qi.astype(np.int8)
+    return codes, scales
+
+
+def quantize(q_bits: np.ndarray, k_bits: np.ndarray, block: int) -> dict:
+    """Everything the quantisation entry point produces: mu, smoothed-K codes, Q codes, scales."""
+    mu = channel_mean(k_bits)
+    qi8, sq = quantize_blocks(bf16_to_f32(q_bits), block)
+    ki8, sk = quantize_blocks(smooth_k(k_bits, mu), block)
+    return {"mu": mu, "q_i8": qi8, "q_scale": sq, "k_i8": ki8, "k_scale": sk}
+
+
+# ---------------------------------------------------------------------------
+# block mask  ([P1] section 三(二) item 1; [P3] --sla_topk)
+# ---------------------------------------------------------------------------
+
+def block_means(x_bits: np.ndarray, block: int) -> np.ndarray:
+    """Mean of each block's valid rows, per channel, in float64: [B, H, nblk, d].
+
+    Reading: the block importance of [P1] 三(二) item 1 (a learnt predictor on
+    the pages, which needs trained weights) is replaced by mean-pooled Q and
+    K blocks; pooling uses the raw (unsmoothed) values; a partial last block
+    is averaged over its valid rows only.
+    """
+    x = bf16_to_f64(x_bits)
+    B, H, N, d = x.shape
+    nblk = (N + block - 1) // block
+    out = np.empty((B, H, nblk, d), dtype=np.float64)
+    for r in range(nblk):
+        lo, hi = r * block, min(N, (r + 1) * block)
+        out[:, :, r, :] = x[:, :, lo:hi, :].sum(axis=2) / float(hi - lo)
+    return out
+
+
+def block_probs(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """Row-wise softmax over key blocks of qbar_i . kbar_j / sqrt(d), float64: [..., nblk, nblk]."""
+    d = qbar.shape[-1]
+    s = np.matmul(qbar, np.swapaxes(kbar, -1, -2)) / math.sqrt(d)
+    e = np.exp(s - s.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def select_topk(p: np.ndarray, kc: int) -> tuple[np.ndarray, np.ndarray]:
+    """Keep the kc largest entries of each row of p; equal values go to the lower index.
+
+    Returns (indices int32 [..., kc] in ascending order, near_tie bool [...]).
+    A row is a near tie when its kc-th and (kc+1)-th largest values differ by
+    at most 1e-9 of the kc-th (then a different but equally valid choice is
+    possible under any other rounding of the scores).
+    """
+    shp = p.shape[:-1]
+    n = p.shape[-1]
+    flat = p.reshape(-1, n)
+    idx = np.empty((flat.shape[0], kc), dtype=np.int32)
+    tie = np.zeros(flat.shape[0], dtype=bool)
+    order_key = np.arange(n)
+    for r in range(flat.shape[0]):
+        row = flat[r]
+        order = np.lexsort((order_key, -row))      # by value desc, then index asc
+        idx[r] = np.sort(order[:kc])
+        if kc < n:
+            a, b = row[order[kc - 1]], row[order[kc]]
+            tie[r] = (a - b) <= NEAR_TIE_REL * a
+    return idx.reshape(shp + (kc,)), tie.reshape(shp)
+
+
+def block_mask(q_bits: np.ndarray, k_bits: np.ndarray, block: int, topk_frac: float) -> dict:
+    """The critical key blocks of every query block: {"idx", "near_tie", "probs", "kc"}."""
+    qbar = block_means(q_bits, block)
+    kbar = block_means(k_bits, block)
+    p = block_probs(qbar, kbar)
+    kc = topk_count(p.shape[-1], topk_frac)
+    idx, tie = select_topk(p, kc)
+    return {"idx": idx, "near_tie": tie, "probs": p, "kc": kc}
+
+
+def bitmap_of(idx: np.ndarray, nblk: int) -> np.ndarray:
+    """uint8 [..., nblk, nblk] with 1 at the kept (query block, key block) pairs."""
+    out = np.zeros(idx.shape[:-1] + (nblk,), dtype=np.uint8)
+    np.put_along_axis(out, idx.astype(np.int64), 1, axis=-1)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# critical blocks: INT8 QK^T, softmax, bf16 P, PV  ([P1] 三(一) item 3, 三(二) item 3)
+# ---------------------------------------------------------------------------
+
+def critical_rows(qi8_blk, sq_i, ki8, sk, v64, crit, N, block, *, pcast=True,
+                  q64_blk=None, ks64=None):
+    """O_sparse for the rows of one query block over its critical key blocks (float64).
+
+    Quantised mode (q64_blk is None), readings of [P1] 三(一) item 3 and
+    三(二) item 3: S = float32(int32(Qi8 . Ki8^T)) * float32(sq_i * sk_j) *
+    float32(1/sqrt(d)) in float32; keys at or past N are masked; softmax with
+    the row maximum over all critical keys; P = exp(S - max) (float64 here);
+    the normaliser l sums the unrounded P; P is rounded to bf16 when
+    ``pcast``; O = (P . V) / l.
+
+    The integer products are formed with a float64 matmul: every entry is an
+    integer of magnitude at most d * 127**2 < 2**53, so it is exact.
+
+    Unquantised mode (q64_blk, ks64 given): S = Q . K_s^T / sqrt(d) in float64.
+    """
+    d = v64.shape[-1]
+    keys = np.concatenate([np.arange(j * block, (j + 1) * block) for j in crit])
+    valid = keys < N
+    if q64_blk is None:
+        acc = np.matmul(qi8_blk.astype(np.float64), ki8[keys].astype(np.float64).T)
+        c = (np.float32(sq_i) * np.repeat(sk[crit], block).astype(np.float32)).astype(np.float32)
+        S = (acc.astype(np.float32) * c[None, :]).astype(np.float32)
+        S = (S * np.float32(1.0 / math.sqrt(d))).astype(np.float32).astype(np.float64)
+    else:
+        kk = np.zeros((len(keys), d))
+        kk[valid] = ks64[keys[valid]]
+        S = np.matmul(q64_blk, kk.T) / math.sqrt(d)
+    S[:, ~valid] = -np.inf
+    M = S.max(axis=1, keepdims=True)
+    P = np.exp(S - M)
+    ell = P.sum(axis=1, keepdims=True)
+    Pb = round_bf16(P) if pcast else P
+    vv = np.zeros((len(keys), d))
+    vv[valid] = v64[keys[valid]]
+    return np.matmul(Pb, vv) / ell
+
+
+# ---------------------------------------------------------------------------
+# linear branch  ([P1] 三(二) item 2; [P4] "SLA: 稀疏線性注意力")
+# ---------------------------------------------------------------------------
+
+def phi(x: np.ndarray) -> np.ndarray:
+    """Feature map elu(x) + 1: x + 1 for x > 0, exp(x) otherwise (always positive)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def linear_states(k64: np.ndarray, v64: np.ndarray, block: int) -> tuple[np.ndarray, np.ndarray]:
+    """Per key block j of one head: h_j = sum_n phi(k_n) v_n^T [d, d], z_j = sum_n phi(k_n) [d].
+
+    [P1] 三(二) item 2 gives the non-selected part an O(N) linear form; the
+    reading adopted is phi = elu + 1 kernelised linear attention with
+    per-block states.  Reading (parity unpinned: no passage decides it):
+    phi is applied to the raw K, not the smoothed K.  Rows past N are left
+    out of the sums.
+    """
+    N, d = k64.shape
+    nblk = (N + block - 1) // block
+    pk = np.zeros((nblk * block, d))
+    pk[:N] = phi(k64)
+    vv = np.zeros((nblk * block, d))
+    vv[:N] = v64
+    pk = pk.reshape(nblk, block, d)
+    vv = vv.reshape(nblk, block, d)
+    h = np.matmul(np.swapaxes(pk, 1, 2), vv)
+    z = pk.sum(axis=1)
+    return h, z
+
+
+def linear_rows(q64_blk: np.ndarray, h: np.ndarray, z: np.ndarray, crit) -> np.ndarray:
+    """O_lin for the rows of one query block: phi(q) h_rest / (phi(q) . z_rest).
+
+    h_rest and z_rest are summed directly over the key blocks NOT in ``crit``
+    (the plain definition: every non-critical block goes through the linear
+    branch).  When every block is critical there is no linear part and
+    O_lin = 0.
+    """
+    nblk, d, _ = h.shape
+    keep = np.ones(nblk, dtype=bool)
+    keep[np.asarray(crit, dtype=np.int64)] = False
+    if not keep.any():
+        return np.zeros((q64_blk.shape[0], d))
+    h_rest = h[keep].sum(axis=0)
+    z_rest = z[keep].sum(axis=0)
+    pq = phi(q64_blk)
+    return np.matmul(pq, h_rest) / np.matmul(pq, z_rest)[:, None]
+
+
+# ---------------------------------------------------------------------------
+# the whole operator
+# ---------------------------------------------------------------------------
+
+def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, *,
+                  items=None, quant=True, pcast=True, smooth=True, idx_override=None):
+    """SageSLA attention: out = O_sparse + O_lin . W_proj.
+
+    [P1] 三(二) item 3 (SLA selection, then INT8 computation on the selected
+    blocks) and item 2 (the rest through the linear branch and a linear
+    projection); [P3] "SageSLA" section.  Reading: W_proj multiplies O_lin on
+    the right (row vectors); the output is rounded to bf16 at the very end.
+
+    items: iterable of (b, h, i) query blocks to evaluate (default: all).
+    quant/pcast/smooth: False switches off INT8 quantisation (float64 scores),
+    the bf16 cast of P, or the K smoothing; all True is the operator itself.
+    idx_override: optional {(b, h, i): key-block list} replacing the mask's
+    choice for those rows (used where the mask is a near tie).
+
+    Returns {"out": {(b,h,i): float64 [rows, d]}, "out_bf16": same rounded,
+    "o_sparse", "o_lin", "mask": block_mask(...), "quant": quantize(...)}.
+    """
+    q_bits = np.asarray(q_bits, dtype=np.uint16)
+    B, H, N, d = q_bits.shape
+    nblk = (N + block - 1) // block
+    mask = block_mask(q_bits, k_bits, block, topk_frac)
+    qz = quantize(q_bits, k_bits, block) if quant else None
+    mu = qz["mu"] if quant else channel_mean(k_bits)
+    w64 = bf16_to_f64(w_bits)
+    if items is None:
+        items = [(b, h, i) for b in range(B) for h in range(H) for i in range(nblk)]
+    by_head = {}
+    for (b, h, i) in items:
+        by_head.setdefault((b, h), []).append(i)
+    res = {"out": {}, "out_bf16": {}, "o_sparse": {}, "o_lin": {}, "mask": mask, "quant": qz}
+    for (b, h), rows in by_head.items():
+        q64 = bf16_to_f64(q_bits[b, h])
+        k64 = bf16_to_f64(k_bits[b, h])
+        v64 = bf16_to_f64(v_bits[b, h])
+        hst, zst = linear_states(k64, v64, block)
+        ks64 = k64 - mu[b, h].astype(np.float64)[None, :] if smooth else k64
+        for i in rows:
+            crit = mask["idx"][b, h, i]
+            if idx_override is not None and (b, h, i) in idx_override:
+                crit = np.asarray(idx_override[(b, h, i)], dtype=np.int32)
+            lo, hi = i * block, min(N, (i + 1) * block)
+            if quant:
+                qi8_blk = qz["q_i8"][b, h, i * block:(i + 1) * block]
+                os_ = critical_rows(qi8_blk, qz["q_scale"][b, h, i], qz["k_i8"][b, h],
+                                    qz["k_scale"][b, h], v64, crit, N, block, pcast=pcast)
+            else:
+                qb = np.zeros((block, d))
+                qb[:hi - lo] = q64[lo:hi]
+                os_ = critical_rows(None, None, None, None, v64, crit, N, block, pcast=pcast,
+                                    q64_blk=qb, ks64=ks64)
+            os_ = os_[:hi - lo]
+            ol = linear_rows(q64[lo:hi], hst, zst, crit)
+            out = os_ + np.matmul(ol, w64)
+            res["o_sparse"][(b, h, i)] = os_
+            res["o_lin"][(b, h, i)] = ol
+            res["out"][(b, h, i)] = out
+            res["out_bf16"][(b, h, i)] = round_bf16(out)
+    return res

@@ -1,0 +1,362 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks one oracle function against a closed form, a library
+routine, a brute force or a hand-derived case (tests/golden/), chosen so that
+a dropped term, a wrong sign or index, or a transposed operand fails one of
+them.  No GPU needed.
+"""
+
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as O
+from synth import make_inputs
+from synth.workloads import f32_to_bf16_bits
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def bits(x):
+    """float values that bf16 holds exactly -> bf16 bits (asserts exactness)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    b = f32_to_bf16_bits(x32)
+    assert np.array_equal(O.bf16_to_f32(b), x32), "test value not representable in bf16"
+    return b
+
+
+# --- number formats --------------------------------------------------------
+
+def test_round_bf16_special_values():
+    e = 2.0 ** -8
+    cases = {
+        1.0: 1.0,
+        1.0 + e: 1.0,                     # tie, even neighbour is 1.0
+        1.0 + 3 * e: 1.0 + 4 * e,         # tie, even neighbour is 1 + 2**-6
+        -(1.0 + e): -1.0,
+        1.0 + 1.5 * e: 1.0 + 2 * e,       # above the tie
+        2.0 ** -130: 2.0 ** -130,         # bf16 subnormal, exact
+        3 * 2.0 ** -135: 2.0 ** -133,     # 0.75 of the subnormal spacing
+        0.0: 0.0,
+    }
+    for x, y in cases.items():
+        assert O.round_bf16(np.array([x]))[0] == y, x
+
+
+def test_round_bf16_matches_torch_on_float32_inputs():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(200000) * np.exp(rng.uniform(-20, 20, 200000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(O.round_bf16(x.astype(np.float64)), ref)
+
+
+def _nearest_f32_bruteforce(fr: Fraction) -> float:
+    f = np.float32(float(fr))
+    best = None
+    for c in (np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))):
+        err = abs(Fraction(float(c)) - fr)
+        key = (err, int(np.array(c, dtype=np.float32).view(np.uint32)) & 1)
+        if best is None or key < best[0]:
+            best = (key, float(c))
+    return best[1]
+
+
+def test_round_rational_to_f32_bruteforce():
+    rng = np.random.default_rng(7)
+    for _ in range(3000):
+        num = int(rng.integers(-2**62, 2**62)) * (1 << int(rng.integers(0, 40)))
+        den = int(rng.integers(1, 2**40))
+        assert O.round_rational_to_f32(num, den) == _nearest_f32_bruteforce(Fraction(num, den))
+    # exact ties between two float32 values: (1 + 2**-24) is halfway between 1 and 1 + 2**-23
+    assert O.round_rational_to_f32((1 << 24) + 1, 1 << 24) == 1.0
+    assert O.round_rational_to_f32((1 << 24) + 3, 1 << 24) == 1.0 + 2.0 ** -22
+
+
+# --- smoothing -------------------------------------------------------------
+
+def test_channel_mean_is_exact_where_float64_summation_is_not():
+    # per channel: 2**100, 1, -2**100  -> exact sum 1; a float64 running sum gives 0
+    k = np.zeros((1, 1, 3, 2), dtype=np.float32)
+    k[0, 0, :, 0] = [2.0 ** 100, 1.0, -(2.0 ** 100)]
+    k[0, 0, :, 1] = [3.0, -1.0, 2.0 ** -60]
+    mu = O.channel_mean(bits(k))
+    assert mu[0, 0, 0] == np.float32(1.0 / 3.0)
+    assert mu[0, 0, 1] == _nearest_f32_bruteforce((Fraction(2) + Fraction(2) ** -60) / 3)
+
+
+def test_channel_mean_matches_exact_rationals():
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((2, 1, 37, 3)) * np.exp(rng.uniform(-30, 30, (2, 1, 37, 3)))).astype(np.float32)
+    b = f32_to_bf16_bits(x)
+    vals = O.bf16_to_f64(b)
+    mu = O.channel_mean(b)
+    for i in range(2):
+        for c in range(3):
+            ex = sum(Fraction(float(t)) for t in vals[i, 0, :, c]) / 37
+            assert mu[i, 0, c] == _nearest_f32_bruteforce(ex)
+
+
+# --- quantisation ----------------------------------------------------------
+
+def test_quant_ties_golden():
+    g = golden("quant_ties.json")
+    x = np.array(g["x"], dtype=np.float32).reshape(1, 1, -1, 1)
+    codes, scales = O.quantize_blocks(x, g["block"])
+    assert scales[0, 0, 0] == g["scale"]
+    assert codes[0, 0, :, 0].tolist() == g["codes"]
+
+
+def test_quant_round_trip_of_representable_blocks():
+    rng = np.random.default_rng(3)
+    block, d, nblk = 16, 8, 5
+    m = rng.integers(-127, 128, size=(1, 1, nblk * block, d))
+    for r in range(nblk):           # force max |m| = 127 in every block
+        m[0, 0, r * block, 0] = 127 if r % 2 else -127
+    s = 2.0 ** -np.arange(3, 3 + nblk)
+    x = (m * np.repeat(s, block)[None, None, :, None]).astype(np.float32)
+    codes, scales = O.quantize_blocks(x, block)
+    assert np.array_equal(codes.astype(np.int64), m)
+    assert np.array_equal(scales[0, 0], s.astype(np.float32))
+
+
+def test_quant_zero_block_partial_block_and_padding():
+    x = np.zeros((1, 1, 10, 4), dtype=np.float32)
+    x[0, 0, 8:10] = [[1, -2, 3, 0.5], [0, 0, -3, 1]]
+    codes, scales = O.quantize_blocks(x, 4)            # blocks [0,4) [4,8) zero, [8,10) partial
+    assert codes.shape == (1, 1, 12, 4)
+    assert scales[0, 0].tolist() == [0.0, 0.0, np.float32(3.0) / np.float32(127.0)]
+    assert not codes[0, 0, :8].any() and not codes[0, 0, 10:].any()
+    assert codes[0, 0, 8].tolist() == [42, -85, 127, 21]     # x/s = 42.33, -84.67, 127, 21.17
+
+
+# --- mask ------------------------------------------------------------------
+
+def test_topk_counts_golden():
+    for c in golden("topk_counts.json")["cases"]:
+        assert O.topk_count(c["nblk"], c["frac"]) == c["kc"], c
+    with pytest.raises(ValueError):
+        O.topk_count(10, 0.0)
+    with pytest.raises(ValueError):
+        O.topk_count(10, 1.5)
+
+
+def test_select_topk_bruteforce_over_all_subsets():
+    rng = np.random.default_rng(2)
+    for trial in range(300):
+        n = int(rng.integers(1, 9))
+        kc = int(rng.integers(1, n + 1))
+        p = rng.integers(0, 4, size=n).astype(np.float64)   # many exact ties
+        idx, _ = O.select_topk(p[None, :], kc)
+        winners = []
+        for sub in itertools.combinations(range(n), kc):
+            rest = [j for j in range(n) if j not in sub]
+            if all(p[a] > p[b] or (p[a] == p[b] and a < b) for a in sub for b in rest):
+                winners.append(list(sub))
+        assert len(winners) == 1
+        assert idx[0].tolist() == winners[0]
+
+
+def test_near_tie_flag():
+    p = np.array([[0.5, 0.3, 0.3 * (1 - 1e-12), 0.1], [0.5, 0.3, 0.29, 0.1]])
+    _, tie = O.select_topk(p, 2)
+    assert tie.tolist() == [True, False]
+
+
+def test_block_means_closed_form_with_partial_block():
+    N, block, d = 10, 4, 3
+    x = np.zeros((1, 1, N, d), dtype=np.float32)
+    for n in range(N):
+        x[0, 0, n] = [n, -2 * n, 1.0]
+    means = O.block_means(bits(x), block)
+    assert means[0, 0].tolist() == [[1.5, -3.0, 1.0], [5.5, -11.0, 1.0], [8.5, -17.0, 1.0]]
+
+
+def test_block_probs_matches_scipy_softmax():
+    rng = np.random.default_rng(4)
+    qb, kb = rng.standard_normal((2, 3, 7, 16)), rng.standard_normal((2, 3, 7, 16))
+    ref = scipy.special.softmax(np.einsum("bhic,bhjc->bhij", qb, kb) / 4.0, axis=-1)
+    assert np.allclose(O.block_probs(qb, kb), ref, rtol=0, atol=1e-15)
+
+
+def test_mask_hand_case():
+    g = golden("linear_hand_case.json")
+    q, k = bits(np.array(g["q"])[None, None]), bits(np.array(g["k"])[None, None])
+    m = O.block_mask(q, k, g["block"], g["topk_frac"])
+    assert m["idx"][0, 0].tolist() == g["idx"]
+
+
+# --- linear branch -----------------------------------------------------------
+
+def test_phi_values():
+    x = np.array([-2.0, -1.0, -1e-300, 0.0, 1e-300, 0.5, 3.0])
+    assert np.allclose(O.phi(x), [math.exp(-2), math.exp(-1), 1.0, 1.0, 1.0, 1.5, 4.0], rtol=1e-15)
+
+
+def test_linear_hand_case():
+    g = golden("linear_hand_case.json")
+    q = np.array(g["q"], dtype=np.float64)
+    k = np.array(g["k"], dtype=np.float64)
+    v = np.array(g["v"], dtype=np.float64)
+    h, z = O.linear_states(k, v, g["block"])
+    assert h.tolist() == g["h"] and z.tolist() == g["z"]
+    e = math.e
+    expect = np.array([[eval(s, {"e": e}) for s in row] for row in g["o_lin_expr"]])
+    got = np.concatenate([O.linear_rows(q[0:2], h, z, g["idx"][0]),
+                          O.linear_rows(q[2:4], h, z, g["idx"][1])])
+    assert np.allclose(got, expect, rtol=1e-14, atol=0)
+
+
+def test_linear_states_skip_rows_past_n():
+    k = np.ones((5, 2))
+    v = np.arange(10, dtype=np.float64).reshape(5, 2)
+    h, z = O.linear_states(k, v, 4)           # second block has one valid row
+    assert z.tolist() == [[8.0, 8.0], [2.0, 2.0]]
+    assert h[1].tolist() == [[16.0, 18.0], [16.0, 18.0]]
+
+
+def test_whole_operator_closed_form_q_k_zero():
+    """Q = K = 0: every score ties, so the lowest kc key blocks are kept; all
+    codes are 0, so P = 1 on every kept key and phi = 1 elsewhere:
+    out = mean(V over kept keys) + mean(V over the other keys) . W."""
+    rng = np.random.default_rng(9)
+    B, H, N, d, block, frac = 1, 2, 200, 8, 32, 0.3          # nblk 7 (last block 8 rows), kc 3
+    v = rng.standard_normal((B, H, N, d)).astype(np.float32)
+    w = rng.standard_normal((d, d)).astype(np.float32) / 4
+    vb, wb = f32_to_bf16_bits(v), f32_to_bf16_bits(w)
+    z = np.zeros((B, H, N, d), dtype=np.uint16)
+    res = O.sla_attention(z, z, vb, wb, block, frac)
+    kc = O.topk_count(7, frac)
+    V, W = O.bf16_to_f64(vb), O.bf16_to_f64(wb)
+    for h in range(H):
+        assert (res["mask"]["idx"][0, h] == np.arange(kc)).all()
+        expect = V[0, h, :kc * block].mean(0) + V[0, h, kc * block:].mean(0) @ W
+        for i in range(7):
+            rows = res["out"][(0, h, i)]
+            assert np.allclose(rows, np.broadcast_to(expect, rows.shape), rtol=0, atol=1e-12)
+
+
+def test_all_blocks_critical_means_no_linear_part():
+    x = make_inputs(1, 1, 96, 16, seed=1)
+    res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 32, 1.0)
+    for key, ol in res["o_lin"].items():
+        assert not ol.any()
+        assert np.array_equal(res["out"][key], res["o_sparse"][key])
+
+
+# --- critical-block attention ----------------------------------------------------
+
+def _sdpa64(q, k, v):
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None], torch.from_numpy(k)[None, None],
+        torch.from_numpy(v)[None, None]).numpy()[0, 0]
+
+
+@pytest.mark.parametrize("N,block", [(256, 64), (200, 64), (130, 32)])
+def test_dense_unquantised_equals_library_attention(N, block):
+    x = make_inputs(1, 2, N, 32, seed=N)
+    res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, 1.0,
+                          quant=False, pcast=False)
+    Q, K, V = (O.bf16_to_f64(x[t]) for t in ("q", "k", "v"))
+    for h in range(2):
+        ref = _sdpa64(Q[0, h], K[0, h], V[0, h])
+        got = np.concatenate([res["out"][(0, h, i)] for i in range((N + block - 1) // block)])
+        assert np.max(np.abs(got - ref)) <= 1e-10
+
+
+def test_smoothing_does_not_change_unquantised_output():
+    x = make_inputs(1, 2, 320, 32, seed=5)
+    a = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.4, quant=False, pcast=False)
+    b = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.4, quant=False, pcast=False,
+                        smooth=False)
+    assert np.array_equal(a["mask"]["idx"], b["mask"]["idx"])
+    for key in a["out"]:
+        assert np.max(np.abs(a["out"][key] - b["out"][key])) <= 1e-12
+
+
+def test_quantised_path_on_losslessly_quantisable_inputs():
+    """Blocks of integers times 2**-6 with max |int| = 127 quantise without loss,
+    and K rows in +- pairs have channel mean 0, so smoothing is the identity:
+    the INT8 path then equals float64 attention up to float32 rounding of S."""
+    rng = np.random.default_rng(12)
+    N, d, block = 256, 32, 64
+    qi = rng.integers(-127, 128, size=(1, 1, N, d))
+    kh = rng.integers(-127, 128, size=(N // 2, d))
+    for r in range(N // block):
+        qi[0, 0, r * block, 0] = 127
+    for r in range(N // 2 // block):
+        kh[r * block, 1] = 127
+    ki = np.concatenate([kh, -kh])[None, None]
+    for r in range(N // block):
+        assert np.abs(ki[0, 0, r * block:(r + 1) * block]).max() == 127
+    qv = (qi * 2.0 ** -6).astype(np.float32)
+    kv = (ki * 2.0 ** -6).astype(np.float32)
+    v = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    qb, kb, vb = bits(qv), bits(kv), f32_to_bf16_bits(v)
+    wb = f32_to_bf16_bits(np.eye(d, dtype=np.float32))
+    qz = O.quantize(qb, kb, block)
+    assert not qz["mu"].any()
+    assert np.array_equal(qz["q_i8"].astype(np.int64), qi)
+    assert np.array_equal(qz["k_i8"].astype(np.int64), ki)
+    a = O.sla_attention(qb, kb, vb, wb, block, 0.5, pcast=False)
+    b = O.sla_attention(qb, kb, vb, wb, block, 0.5, pcast=False, quant=False)
+    for key in a["out"]:
+        assert np.max(np.abs(a["o_sparse"][key] - b["o_sparse"][key])) <= 1e-5
+
+
+def test_bf16_cast_of_p_error_bound():
+    """Rounding P to bf16 changes each P by at most 2**-9 of itself, so O moves by
+    at most 2**-9 * max |V|."""
+    x = make_inputs(1, 1, 512, 32, seed=8)
+    a = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.25)
+    b = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.25, pcast=False)
+    vmax = np.abs(O.bf16_to_f64(x["v"])).max()
+    worst = max(np.abs(a["o_sparse"][k] - b["o_sparse"][k]).max() for k in a["o_sparse"])
+    assert 0 < worst <= 2.0 ** -9 * vmax
+
+
+def test_projection_multiplies_on_the_right():
+    """W_proj = identity gives out = O_sparse + O_lin; W_proj = 0 gives O_sparse; a
+    permutation matrix permutes the columns of O_lin."""
+    x = make_inputs(1, 1, 256, 16, seed=21)
+    d = 16
+    eye = f32_to_bf16_bits(np.eye(d, dtype=np.float32))
+    zero = np.zeros((d, d), dtype=np.uint16)
+    perm = np.roll(np.eye(d, dtype=np.float32), 1, axis=1)          # e_a -> e_{a+1}
+    a = O.sla_attention(x["q"], x["k"], x["v"], eye, 32, 0.25)
+    b = O.sla_attention(x["q"], x["k"], x["v"], zero, 32, 0.25)
+    c = O.sla_attention(x["q"], x["k"], x["v"], f32_to_bf16_bits(perm), 32, 0.25)
+    for key in a["out"]:
+        assert np.array_equal(a["out"][key], a["o_sparse"][key] + a["o_lin"][key])
+        assert np.array_equal(b["out"][key], b["o_sparse"][key])
+        assert np.allclose(c["out"][key] - c["o_sparse"][key], np.roll(c["o_lin"][key], 1, axis=1),
+                           rtol=0, atol=1e-15)
+
+
+def test_quant_codes_match_exact_rational_division():
+    """Each code is the float32 nearest to x / s (exact rational arithmetic),
+    rounded half to even; s is the float32 nearest to max|x| / 127."""
+    rng = np.random.default_rng(17)
+    x = (rng.standard_normal((1, 1, 64, 32)) * 3).astype(np.float32)
+    x = O.bf16_to_f32(f32_to_bf16_bits(x))
+    codes, scales = O.quantize_blocks(x[:, :, :, :], 16)
+    for r in range(4):
+        blk = x[0, 0, r * 16:(r + 1) * 16]
+        m = Fraction(float(np.abs(blk).max()))
+        s = _nearest_f32_bruteforce(m / 127)
+        assert scales[0, 0, r] == s
+        for (n, c), val in np.ndenumerate(blk):
+            qf = _nearest_f32_bruteforce(Fraction(float(val)) / Fraction(s))
+            want = max(-127, min(127, int(np.rint(qf))))
+            assert codes[0, 0, r * 16 + n, c] == want
