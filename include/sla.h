@@ -1,0 +1,132 @@
+/*
+ * sla.h -- C interface of the SageSLA attention library for NVIDIA B200
+ * (sm_100a): INT8 block-quantised, top-k block-sparse softmax attention plus
+ * a linear-attention branch for the key blocks that were not selected.
+ *
+ * The operation is the SageSLA attention module of the pages
+ *   [P1] "Turbo Diffusion：秒级生成与高清保真的视频扩散技术突破" (lanhy.cn),
+ *        section 三(一) SageAttention2++ items 1-3 and section 三(二) SLA
+ *        items 1-3;
+ *   [P3] "TurboDiffusion技术指南：突破视频生成效率瓶颈的实践方案"
+ *        (blog.gitcode.com), section "SageSLA" and the T2V parameter list
+ *        (--attention_type sagesla, --sla_topk 0.1 = keep 10%).
+ * The pages give no formulas; the exact semantics implemented here are:
+ *   1. mu = per-channel mean of K over the N tokens (exact sum, rounded once to
+ *      float32); K_s = float32(K) - mu.  ([P1] 三(一) item 1, "outlier smoothing")
+ *   2. Q and K_s are quantised to INT8 per block of `block` tokens x d channels:
+ *      s = max|x| / 127 (float32), code = clamp(round_half_even(x / s), +-127).
+ *      ([P1] 三(一) item 2)
+ *   3. Block mask: qbar_i, kbar_j = means of the raw Q, K rows of each block
+ *      (float64); score = qbar_i . kbar_j / sqrt(d); each query block keeps the
+ *      kc = ceil(topk_frac * nblk) key blocks with the largest scores (equal
+ *      scores: lower block index first), listed in ascending order.
+ *      ([P1] 三(二) item 1; [P3] --sla_topk)
+ *   4. For the kept blocks: S = int32(Qi8 . Ki8^T) * sq * sk / sqrt(d),
+ *      float32 online softmax, P rounded to bf16, O_sparse = (P . V) / l with
+ *      float32 accumulation.  ([P1] 三(一) item 3, 三(二) item 3)
+ *   5. For the other blocks: phi = elu + 1 linear attention,
+ *      O_lin = phi(q) (sum h_j) / (phi(q) . sum z_j) with per-key-block states
+ *      h_j = sum phi(k) v^T, z_j = sum phi(k) of the raw K; none when every
+ *      block is kept.  ([P1] 三(二) item 2)
+ *   6. out = O_sparse + O_lin . W_proj in float32 (the accumulation
+ *      precision; the pages name no output rounding).  ([P1] 三(二) item 2,
+ *      "linear projection")
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major.  q, k, v: bf16 [B, H, N, d] (d innermost); out:
+ *     float32 [B, H, N, d].
+ *     proj (W_proj): bf16 [d, d], used as O_lin . proj (row vectors).
+ *   - All tensor pointers are DEVICE pointers except where an entry point says
+ *     HOST.  They must be 16-byte aligned.  The caller owns all memory; the
+ *     library never frees or retains caller pointers.
+ *   - nblk = ceil(N / block); kc = sla_topk_count(N, block, topk_frac).
+ *   - Supported: d in {64, 128}; block in {64, 128}; B, H, N >= 1;
+ *     0 < topk_frac <= 1; nblk <= 16384; B*H <= 65535; B*H*nblk*block < 2^31.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Device
+ *     entry points only enqueue work on `stream` and return; they may draw
+ *     temporary device memory from a library-owned stream-ordered pool.
+ *   - Arguments are checked before anything is enqueued; an invalid call
+ *     returns an error code and touches no memory.  Faults inside the kernels
+ *     surface at the caller's next synchronisation or through
+ *     sla_get_error().
+ *   - Thread safety: calls are re-entrant; concurrent calls on different
+ *     streams are independent.
+ */
+#ifndef SLA_H_
+#define SLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLA_OK = 0,
+  SLA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, value out of range     */
+  SLA_ERR_UNSUPPORTED = 2,  /* well-formed but outside the supported shapes        */
+  SLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                   */
+  SLA_ERR_OOM = 4,          /* temporary device memory could not be obtained       */
+  SLA_ERR_TIMEOUT = 5,      /* a kernel's bounded wait gave up (sla_get_error)     */
+  SLA_ERR_INEXACT_MEAN = 6  /* the K channel mean could not be proven exact: some
+                               channel's values span more exponents than a float64
+                               sum holds exactly (sla_get_error; results are still
+                               written)                                            */
+} sla_status;
+
+/* Number of key blocks each query block keeps:
+ * clamp(ceil(float(topk_frac) * nblk), 1, nblk), computed exactly in double.
+ * Returns -SLA_ERR_INVALID_ARG if N < 1, block < 1 or topk_frac not in (0, 1].
+ * Host only; touches no device. */
+int sla_topk_count(int N, int block, float topk_frac);
+
+/* Steps 1-2 only (SageAttention2++ smoothing + quantisation, [P1] 三(一) 1-2).
+ *   q, k     : in,  bf16 [B,H,N,d]
+ *   q_i8     : out, int8 [B,H,nblk*block,d]   codes of Q; rows >= N are 0
+ *   k_i8     : out, int8 [B,H,nblk*block,d]   codes of K - mu; rows >= N are 0
+ *   q_scale  : out, float [B,H,nblk]
+ *   k_scale  : out, float [B,H,nblk]
+ *   k_mean   : out, float [B,H,d] (mu), or NULL */
+int sla_quant(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q_scale, float* k_scale,
+              float* k_mean, int B, int H, int N, int d, int block, void* stream);
+
+/* Step 3 only (SLA block selection, [P1] 三(二) 1).
+ *   blk_idx : out, int32 [B,H,nblk,kc], kept key blocks of each query block, ascending
+ *   bitmap  : out, uint8 [B,H,nblk,nblk], 1 where kept, or NULL */
+int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, int B, int H, int N, int d,
+             int block, float topk_frac, void* stream);
+
+/* The whole operator, steps 1-6 ([P1] 三(二) 3, SageSLA).
+ *   q, k, v : in,  bf16 [B,H,N,d]
+ *   proj    : in,  bf16 [d,d]
+ *   out     : out, float [B,H,N,d], fully overwritten */
+int sla_attn(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N,
+             int d, int block, float topk_frac, void* stream);
+
+/* sla_attn that also returns the critical-block part before the projection
+ * and the sum (for inspection and tests):
+ *   o_sparse : out, float [B,H,N,d] = O_sparse of step 4, or NULL. */
+int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, void* out, float* o_sparse,
+                int B, int H, int N, int d, int block, float topk_frac, void* stream);
+
+/* sla_attn on HOST buffers (pageable or pinned): copies q, k, v, proj to the
+ * device, runs the operator on an internal stream of the current device,
+ * copies out back and returns when it is in host memory. */
+int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
+                  int N, int d, int block, float topk_frac);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: SLA_ERR_TIMEOUT if a kernel's bounded wait gave up,
+ * SLA_ERR_INEXACT_MEAN if a channel mean could not be proven exact,
+ * SLA_ERR_CUDA if the synchronisation itself failed, else SLA_OK. */
+int sla_get_error(void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* sla_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H_ */

@@ -1,0 +1,154 @@
+"""SageSLA attention for NVIDIA B200 (sm_100a) -- Python binding.
+
+This module only marshals arguments: every step of the operator runs in the
+CUDA kernels of ``libsla.so`` (built from ``csrc/`` by ``build.py``), called
+through its C interface (``include/sla.h``).  PyTorch supplies device memory
+and streams.  There is no CPU fallback: if the library is missing, importing
+the binding's functions raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsla.so")
+
+SLA_OK = 0
+STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "SLA_ERR_CUDA",
+                4: "SLA_ERR_OOM", 5: "SLA_ERR_TIMEOUT", 6: "SLA_ERR_INEXACT_MEAN"}
+
+EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
+           "sla_get_error", "sla_status_string")
+
+
+class SlaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsla.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with `python -m int8_block_sparse_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.sla_topk_count.argtypes = [i, i, f]
+        L.sla_quant.argtypes = [vp] * 7 + [i] * 5 + [vp]
+        L.sla_mask.argtypes = [vp] * 4 + [i] * 5 + [f, vp]
+        L.sla_attn.argtypes = [vp] * 5 + [i] * 5 + [f, vp]
+        L.sla_attn_ex.argtypes = [vp] * 6 + [i] * 5 + [f, vp]
+        L.sla_attn_host.argtypes = [vp] * 5 + [i] * 5 + [f]
+        L.sla_get_error.argtypes = [vp]
+        L.sla_status_string.argtypes = [i]
+        L.sla_status_string.restype = ctypes.c_char_p
+        for name in EXPORTS:
+            if name != "sla_status_string":
+                getattr(L, name).restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().sla_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != SLA_OK:
+        raise SlaError(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    return tuple(int(x) for x in q.shape)
+
+
+def topk_count(N: int, block: int, topk_frac: float) -> int:
+    kc = lib().sla_topk_count(int(N), int(block), float(topk_frac))
+    if kc < 0:
+        raise SlaError(-kc, "sla_topk_count")
+    return kc
+
+
+def nblk(N: int, block: int) -> int:
+    return (N + block - 1) // block
+
+
+def sla_quant(q, k, block: int, stream=None):
+    """Smoothing + INT8 quantisation.  Returns (q_i8, k_i8, q_scale, k_scale, k_mean)."""
+    import torch
+
+    B, H, N, d = _shape(q)
+    nb = nblk(N, block)
+    dev = q.device
+    qi8 = torch.empty((B, H, nb * block, d), dtype=torch.int8, device=dev)
+    ki8 = torch.empty_like(qi8)
+    sq = torch.empty((B, H, nb), dtype=torch.float32, device=dev)
+    sk = torch.empty_like(sq)
+    mu = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    _check(lib().sla_quant(_ptr(q), _ptr(k), _ptr(qi8), _ptr(ki8), _ptr(sq), _ptr(sk), _ptr(mu),
+                           B, H, N, d, block, _stream(stream)), "sla_quant")
+    return qi8, ki8, sq, sk, mu
+
+
+def sla_mask(q, k, block: int, topk_frac: float, bitmap: bool = False, stream=None):
+    """Pooled top-k block mask.  Returns idx [B,H,nblk,kc] int32 (and the uint8 bitmap)."""
+    import torch
+
+    B, H, N, d = _shape(q)
+    nb = nblk(N, block)
+    kc = topk_count(N, block, topk_frac)
+    idx = torch.empty((B, H, nb, kc), dtype=torch.int32, device=q.device)
+    bm = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=q.device) if bitmap else None
+    _check(lib().sla_mask(_ptr(q), _ptr(k), _ptr(idx), _ptr(bm), B, H, N, d, block, float(topk_frac),
+                          _stream(stream)), "sla_mask")
+    return (idx, bm) if bitmap else idx
+
+
+def sla_attn(q, k, v, proj, block: int = 128, topk_frac: float = 0.1, out=None, o_sparse=None,
+             stream=None):
+    """SageSLA attention; q, k, v bf16 [B,H,N,d], proj bf16 [d,d] on the GPU.  Returns out (float32)."""
+    import torch
+
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
+    if o_sparse is None:
+        rc = lib().sla_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
+                            float(topk_frac), _stream(stream))
+    else:
+        rc = lib().sla_attn_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), _ptr(o_sparse), B, H, N, d,
+                               block, float(topk_frac), _stream(stream))
+    _check(rc, "sla_attn")
+    return out
+
+
+def sla_attn_host(q, k, v, proj, out, block: int = 128, topk_frac: float = 0.1) -> None:
+    """SageSLA attention on host (CPU) tensors (out: float32); copies in and out inside the call."""
+    B, H, N, d = _shape(q)
+    _check(lib().sla_attn_host(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
+                               float(topk_frac)), "sla_attn_host")
+
+
+def get_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error status."""
+    return lib().sla_get_error(_stream(stream))

@@ -1,0 +1,102 @@
+// K2: fused smooth + quantise, one CTA per (tensor, head, block of tokens).
+//
+// "Turbo Diffusion：秒级生成与高清保真的视频扩散技术突破", section 三(一)
+// SageAttention2++: item 1 (smooth outliers before quantising -- here K minus
+// its per-channel mean over tokens) and item 2 (every sub-block has its own
+// quantisation parameters -- here one float32 scale per block of BLK tokens x
+// D channels).  Per block: m = max|x|, s = m / 127 (IEEE float32 division),
+// code = clamp(round_half_even(x / s), -127, 127) with an IEEE division per
+// element; a block with m = 0 has s = 0 and zero codes.  Rows past N (up to
+// NB*BLK) get zero codes.  For Q the kernel also writes the float64 sums of
+// each block (the pooled block means of the mask).
+#pragma once
+#include <cuda_bf16.h>
+#include "sm100.cuh"
+
+namespace sla {
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(256) k_quant(const __nv_bfloat16* __restrict__ Q,
+                                              const __nv_bfloat16* __restrict__ K, const float* __restrict__ mu,
+                                              int8_t* __restrict__ qi8, int8_t* __restrict__ ki8,
+                                              float* __restrict__ sq, float* __restrict__ sk,
+                                              double* __restrict__ qsum, int N, int NB) {
+  constexpr int VEC = 8;
+  constexpr int GROUPS = D / VEC;
+  constexpr int NV = BLK * GROUPS / 256;   // 16-byte vectors per thread
+  static_assert(NV >= 1 && (BLK * GROUPS) % 256 == 0, "tile shape");
+  constexpr int RSTEP = 256 / GROUPS;
+  __shared__ float wmax[8];
+  __shared__ double red[RSTEP * D];
+
+  const int j = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const bool isk = blockIdx.z == 1;
+  const int tid = threadIdx.x;
+  const int row0 = j * BLK;
+  const int rows = min(BLK, N - row0);
+  const __nv_bfloat16* src = (isk ? K : Q) + (bh * N + row0) * (long long)D;
+  const int g = tid % GROUPS;
+
+  float x[NV][VEC];
+  float mloc = 0.f;
+#pragma unroll
+  for (int t = 0; t < NV; ++t) {
+    const int r = tid / GROUPS + t * RSTEP;
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (r < rows) raw = *reinterpret_cast<const uint4*>(src + (long long)r * D + g * VEC);
+    const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      float f = __uint_as_float(uint32_t(hv[e]) << 16);
+      if (isk && r < rows) f = __fsub_rn(f, mu[bh * D + g * VEC + e]);
+      x[t][e] = f;
+      mloc = fmaxf(mloc, fabsf(f));
+    }
+  }
+  if (!isk && qsum != nullptr) {
+    double part[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) part[e] = 0.0;
+#pragma unroll
+    for (int t = 0; t < NV; ++t)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) part[e] += (double)x[t][e];   // padding rows hold 0
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) red[(tid / GROUPS) * D + g * VEC + e] = part[e];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+  if ((tid & 31) == 0) wmax[tid >> 5] = mloc;
+  __syncthreads();
+  float m = wmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+  const float s = __fdiv_rn(m, 127.0f);
+  float* sdst = isk ? sk : sq;
+  if (tid == 0 && sdst != nullptr) sdst[bh * NB + j] = s;
+  if (!isk && qsum != nullptr && tid < D) {
+    double acc = 0.0;
+    for (int q = 0; q < RSTEP; ++q) acc += red[q * D + tid];
+    qsum[(bh * NB + j) * (long long)D + tid] = acc;
+  }
+  int8_t* dbase = isk ? ki8 : qi8;
+  if (dbase == nullptr) return;
+  int8_t* dst = dbase + (bh * (long long)NB * BLK + row0) * (long long)D;
+#pragma unroll
+  for (int t = 0; t < NV; ++t) {
+    const int r = tid / GROUPS + t * RSTEP;
+    uint32_t packed[2] = {0u, 0u};
+    if (s > 0.f) {
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        int qv = __float2int_rn(__fdiv_rn(x[t][e], s));
+        qv = max(-127, min(127, qv));
+        packed[e >> 2] |= (uint32_t(qv) & 0xFFu) << (8 * (e & 3));
+      }
+    }
+    *reinterpret_cast<uint2*>(dst + (long long)r * D + g * VEC) = make_uint2(packed[0], packed[1]);
+  }
+}
+
+}  // namespace sla

@@ -1,0 +1,484 @@
+// C interface of the SageSLA attention library: argument checks, temporary
+// device memory, TMA descriptors and the launch sequence of the kernels
+//   K1 k_kstats        K block sums + linear states          (k_stats.cuh)
+//      k_channel_mean  mu                                   (k_stats.cuh)
+//   K2 k_quant         smoothing + INT8 codes + Q block sums (k_quant.cuh)
+//   K3 k_mask          pooled scores + top-k                 (k_mask.cuh)
+//   K5a k_lingemm      sums of the non-selected states       (k_linear.cuh)
+//   K4 k_attn          critical-block attention              (k_attn.cuh)
+//   K5b k_linout       linear branch, projection, add        (k_linear.cuh)
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sla.h"
+#include "k_attn.cuh"
+#include "k_linear.cuh"
+#include "k_mask.cuh"
+#include "k_quant.cuh"
+#include "k_stats.cuh"
+
+using namespace sla;
+
+namespace {
+
+// ------------------------------------------------------------------ helpers
+struct Shape {
+  int B, H, N, d, block;
+  long long BH, NB, NP, kc;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int N, int d, int block, Shape* s) {
+  if (B < 1 || H < 1 || N < 1 || d < 1 || block < 1) return SLA_ERR_INVALID_ARG;
+  if (!(d == 64 || d == 128) || !(block == 64 || block == 128)) return SLA_ERR_UNSUPPORTED;
+  s->B = B; s->H = H; s->N = N; s->d = d; s->block = block;
+  s->BH = (long long)B * H;
+  s->NB = (N + block - 1) / block;
+  s->NP = s->NB * block;
+  if (s->BH > 65535 || s->NB > 16384) return SLA_ERR_UNSUPPORTED;
+  if (s->BH * s->NP >= (1LL << 31)) return SLA_ERR_UNSUPPORTED;
+  return SLA_OK;
+}
+
+long long topk_count_ll(long long nblk, float frac) {
+  const double kc = std::ceil((double)frac * (double)nblk);
+  if (kc < 1.0) return 1;
+  if (kc > (double)nblk) return nblk;
+  return (long long)kc;
+}
+
+bool frac_ok(float f) { return f > 0.f && f <= 1.f; }
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ptr, const cuuint64_t* dims,
+              const cuuint64_t* strides_bytes, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, (cuuint32_t)rank, const_cast<void*>(ptr), dims, strides_bytes, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ temporary memory
+// One stream-ordered pool per device that keeps its memory between calls.
+cudaMemPool_t pool_for_current_device() {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (pools[dev] == nullptr) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return nullptr;
+    uint64_t thr = UINT64_MAX;
+    cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &thr);
+    pools[dev] = p;
+  }
+  return pools[dev];
+}
+
+struct Arena {
+  char* base = nullptr;
+  size_t off = 0, cap = 0;
+  template <class T>
+  T* take(size_t count) {
+    const size_t bytes = (count * sizeof(T) + 255) & ~size_t(255);
+    T* p = reinterpret_cast<T*>(base + off);
+    off += bytes;
+    return p;
+  }
+};
+
+template <class T>
+size_t rounded(size_t count) { return (count * sizeof(T) + 255) & ~size_t(255); }
+
+struct Workspace {
+  double* ksum; uint8_t* kexp; float* mu; double* qsum;
+  int8_t* qi8; int8_t* ki8; float* sq; float* sk; int32_t* idx;
+  __nv_bfloat16* notcrit; __nv_bfloat16* hstate; __nv_bfloat16* grest; float* zrest;
+  long long ncpitch, hpitch;
+};
+
+// what: bit 0 quant outputs, bit 1 mask, bit 2 attention, bit 3 linear branch
+size_t workspace_bytes(const Shape& s, int what) {
+  const size_t BH = s.BH, NB = s.NB, NP = s.NP, d = s.d, kc = s.kc;
+  const size_t ncpitch = (NB + 63) / 64 * 64, hpitch = d * d + d;
+  size_t b = rounded<double>(BH * NB * d) * 2 + rounded<uint8_t>(BH * NB * d * 2) + rounded<float>(BH * d);
+  if (what & 1) b += rounded<int8_t>(BH * NP * d) * 2 + rounded<float>(BH * NB) * 2;
+  if (what & 2) b += rounded<int32_t>(BH * NB * kc);
+  if (what & 8)
+    b += rounded<__nv_bfloat16>(BH * NB * ncpitch) + rounded<__nv_bfloat16>(BH * NB * hpitch) +
+         rounded<__nv_bfloat16>(BH * NB * d * d) + rounded<float>(BH * NB * d);
+  return b;
+}
+
+Workspace carve(const Shape& s, int what, char* base) {
+  Arena a;
+  a.base = base;
+  Workspace w{};
+  const size_t BH = s.BH, NB = s.NB, NP = s.NP, d = s.d, kc = s.kc;
+  w.ncpitch = (NB + 63) / 64 * 64;
+  w.hpitch = d * d + d;
+  w.ksum = a.take<double>(BH * NB * d);
+  w.qsum = a.take<double>(BH * NB * d);
+  w.kexp = a.take<uint8_t>(BH * NB * d * 2);
+  w.mu = a.take<float>(BH * d);
+  if (what & 1) {
+    w.qi8 = a.take<int8_t>(BH * NP * d);
+    w.ki8 = a.take<int8_t>(BH * NP * d);
+    w.sq = a.take<float>(BH * NB);
+    w.sk = a.take<float>(BH * NB);
+  }
+  if (what & 2) w.idx = a.take<int32_t>(BH * NB * kc);
+  if (what & 8) {
+    w.notcrit = a.take<__nv_bfloat16>(BH * NB * w.ncpitch);
+    w.hstate = a.take<__nv_bfloat16>(BH * NB * w.hpitch);
+    w.grest = a.take<__nv_bfloat16>(BH * NB * d * d);
+    w.zrest = a.take<float>(BH * NB * d);
+  }
+  return w;
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SLA_OK;
+  if (e == cudaErrorMemoryAllocation) return SLA_ERR_OOM;
+  return SLA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ launch helpers
+template <int D, int BLK>
+int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                       Workspace& w, bool states, bool kcodes, int8_t* qi8, int8_t* ki8, float* sq, float* sk,
+                       cudaStream_t st) {
+  const size_t sm1 = kstats_smem<D, BLK>();
+  cudaFuncSetAttribute(k_kstats<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+  dim3 g1((unsigned)s.NB, (unsigned)s.BH);
+  k_kstats<D, BLK><<<g1, 256, sm1, st>>>(k, v, w.ksum, w.kexp, states ? w.hstate : nullptr, s.N, (int)s.NB,
+                                         w.hpitch);
+  const long long tot = s.BH * D;
+  k_channel_mean<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, D, s.N, tot);
+  dim3 g2((unsigned)s.NB, (unsigned)s.BH, kcodes ? 2u : 1u);
+  k_quant<D, BLK><<<g2, 256, 0, st>>>(q, k, w.mu, qi8, ki8, sq, sk, w.qsum, s.N, (int)s.NB);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+int launch_mask(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __nv_bfloat16* notcrit,
+                cudaStream_t st) {
+  int rows = 16;
+  while (rows > 1 && mask_smem<D>(rows, (int)s.NB) > 200 * 1024) rows /= 2;
+  const size_t sm = mask_smem<D>(rows, (int)s.NB);
+  cudaFuncSetAttribute(k_mask<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  dim3 g((unsigned)((s.NB + rows - 1) / rows), (unsigned)s.BH);
+  k_mask<D><<<g, 256, sm, st>>>(w.qsum, w.ksum, s.N, (int)s.NB, s.block, (int)s.kc, rows, idx, bitmap, notcrit,
+                                (int)w.ncpitch);
+  return cuda_status(cudaGetLastError());
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D, int BLK>
+int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* v, float* o, cudaStream_t st) {
+  using C = AttnCfg<D, BLK>;
+  CUtensorMap mq, mk, mv;
+  const CUtensorMapSwizzle ksw = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(s.BH * s.NP)};
+    cuuint64_t str[1] = {(cuuint64_t)D};
+    cuuint32_t boxq[2] = {(cuuint32_t)D, 128u};
+    cuuint32_t boxk[2] = {(cuuint32_t)D, (cuuint32_t)BLK};
+    if (!make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w.qi8, dims, str, boxq, ksw)) return SLA_ERR_CUDA;
+    if (!make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w.ki8, dims, str, boxk, ksw)) return SLA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
+    cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)s.N * D * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)BLK, 1u};
+    if (!make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  AttnParams p;
+  p.idx = w.idx; p.sq = w.sq; p.sk = w.sk; p.o = o;
+  p.N = s.N; p.NB = (int)s.NB; p.NP = (int)s.NP; p.kc = (int)s.kc; p.items = (int)(s.BH * s.NB);
+  p.qk_scale = (float)(1.4426950408889634 / std::sqrt((double)D));
+  cudaFuncSetAttribute(k_attn<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const int ctas = (int)std::min<long long>(num_sms(), (p.items + 1) / 2);
+  k_attn<D, BLK><<<ctas, 384, C::SMEM, st>>>(mq, mk, mv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __nv_bfloat16* proj,
+                  const float* osparse, float* out, cudaStream_t st) {
+  CUtensorMap ma, mb, mg, mw;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)w.ncpitch, (cuuint64_t)s.NB, (cuuint64_t)s.BH};
+    cuuint64_t str[2] = {(cuuint64_t)w.ncpitch * 2, (cuuint64_t)(w.ncpitch * s.NB * 2)};
+    cuuint32_t box[3] = {64u, 128u, 1u};
+    if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.notcrit, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)w.hpitch, (cuuint64_t)s.NB, (cuuint64_t)s.BH};
+    cuuint64_t str[2] = {(cuuint64_t)w.hpitch * 2, (cuuint64_t)(w.hpitch * s.NB * 2)};
+    cuuint32_t box[3] = {64u, 64u, 1u};
+    if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.hstate, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(s.BH * s.NB * D)};
+    cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)D};
+    if (!make_map(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.grest, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)D};
+    cuuint64_t str[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)D};
+    if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, proj, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  LinGemmParams gp;
+  gp.grest = w.grest; gp.zrest = w.zrest; gp.NB = (int)s.NB; gp.D = D; gp.E = D * D + D;
+  gp.nkt = (int)((s.NB + 63) / 64);
+  cudaFuncSetAttribute(k_lingemm, cudaFuncAttributeMaxDynamicSharedMemorySize, LG_SMEM);
+  dim3 g1((unsigned)((gp.E + 255) / 256), (unsigned)((s.NB + 127) / 128), (unsigned)s.BH);
+  k_lingemm<<<g1, 128, LG_SMEM, st>>>(ma, mb, gp);
+  LinOutParams op;
+  op.q = q; op.zrest = w.zrest; op.osparse = osparse; op.out = out;
+  op.N = s.N; op.NB = (int)s.NB; op.BLK = s.block;
+  cudaFuncSetAttribute(k_linout<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinOutCfg<D>::SMEM);
+  dim3 g2((unsigned)s.NB, (unsigned)s.BH);
+  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, mw, op);
+  return cuda_status(cudaGetLastError());
+}
+
+// ------------------------------------------------------------------ dispatch
+template <int D, int BLK>
+int run_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+             const __nv_bfloat16* proj, float* out, float* o_sparse, Workspace& w, cudaStream_t st) {
+  const bool linear = s.kc < s.NB;
+  int rc = launch_stats_quant<D, BLK>(s, q, k, v, w, linear, true, w.qi8, w.ki8, w.sq, w.sk, st);
+  if (rc) return rc;
+  rc = launch_mask<D>(s, w, w.idx, nullptr, linear ? w.notcrit : nullptr, st);
+  if (rc) return rc;
+  // O_sparse goes to o_sparse when the caller wants it, else straight into
+  // out, which the linear branch then updates in place.
+  float* osp = (linear && o_sparse != nullptr) ? o_sparse : out;
+  rc = launch_attn<D, BLK>(s, w, v, osp, st);
+  if (rc) return rc;
+  if (linear) return launch_linear<D>(s, w, q, proj, osp, out, st);
+  if (o_sparse != nullptr)
+    return cuda_status(cudaMemcpyAsync(o_sparse, out, (size_t)s.BH * s.N * D * sizeof(float),
+                                       cudaMemcpyDeviceToDevice, st));
+  return SLA_OK;
+}
+
+template <class F>
+int with_dims(int d, int block, F&& f) {
+  if (d == 128 && block == 128) return f(std::integral_constant<int, 128>(), std::integral_constant<int, 128>());
+  if (d == 128 && block == 64) return f(std::integral_constant<int, 128>(), std::integral_constant<int, 64>());
+  if (d == 64 && block == 128) return f(std::integral_constant<int, 64>(), std::integral_constant<int, 128>());
+  if (d == 64 && block == 64) return f(std::integral_constant<int, 64>(), std::integral_constant<int, 64>());
+  return SLA_ERR_UNSUPPORTED;
+}
+
+struct Scratch {
+  void* ptr = nullptr;
+  cudaStream_t st = nullptr;
+  int get(size_t bytes, cudaStream_t s) {
+    st = s;
+    cudaMemPool_t pool = pool_for_current_device();
+    if (pool == nullptr) return SLA_ERR_CUDA;
+    const cudaError_t e = cudaMallocFromPoolAsync(&ptr, bytes, pool, s);
+    if (e != cudaSuccess) { ptr = nullptr; return cuda_status(e); }
+    return SLA_OK;
+  }
+  ~Scratch() {
+    if (ptr != nullptr) cudaFreeAsync(ptr, st);
+  }
+};
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int sla_topk_count(int N, int block, float topk_frac) {
+  if (N < 1 || block < 1 || !frac_ok(topk_frac)) return -SLA_ERR_INVALID_ARG;
+  const long long nb = ((long long)N + block - 1) / block;
+  return (int)topk_count_ll(nb, topk_frac);
+}
+
+const char* sla_status_string(int status) {
+  switch (status) {
+    case SLA_OK: return "ok";
+    case SLA_ERR_INVALID_ARG: return "invalid argument";
+    case SLA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case SLA_ERR_CUDA: return "CUDA error";
+    case SLA_ERR_OOM: return "out of device memory";
+    case SLA_ERR_TIMEOUT: return "a kernel wait timed out";
+    case SLA_ERR_INEXACT_MEAN: return "K channel mean not proven exact";
+    default: return "unknown status";
+  }
+}
+
+int sla_quant(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q_scale, float* k_scale,
+              float* k_mean, int B, int H, int N, int d, int block, void* stream) {
+  if (!q || !k || !q_i8 || !k_i8 || !q_scale || !k_scale) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  s.kc = 1;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch sc;
+  if ((rc = sc.get(workspace_bytes(s, 0), st))) return rc;
+  Workspace w = carve(s, 0, static_cast<char*>(sc.ptr));
+  if (k_mean != nullptr) w.mu = k_mean;
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    return launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                      static_cast<const __nv_bfloat16*>(k), w, false, true, q_i8, k_i8, q_scale,
+                                      k_scale, st);
+  });
+}
+
+int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, int B, int H, int N, int d,
+             int block, float topk_frac, void* stream) {
+  if (!q || !k || !blk_idx) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return SLA_ERR_INVALID_ARG;
+  if (!frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  s.kc = topk_count_ll(s.NB, topk_frac);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch sc;
+  if ((rc = sc.get(workspace_bytes(s, 0), st))) return rc;
+  Workspace w = carve(s, 0, static_cast<char*>(sc.ptr));
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                       static_cast<const __nv_bfloat16*>(k), w, false, false, nullptr, nullptr,
+                                       nullptr, nullptr, st);
+    if (r) return r;
+    return launch_mask<D>(s, w, blk_idx, bitmap, nullptr, st);
+  });
+}
+
+int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, void* out, float* o_sparse,
+                int B, int H, int N, int d, int block, float topk_frac, void* stream) {
+  if (!q || !k || !v || !proj || !out) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj) || !aligned16(out) ||
+      !aligned16(o_sparse))
+    return SLA_ERR_INVALID_ARG;
+  if (!frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  s.kc = topk_count_ll(s.NB, topk_frac);
+  const bool linear = s.kc < s.NB;
+  const int what = 1 | 2 | 4 | (linear ? 8 : 0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch sc;
+  if ((rc = sc.get(workspace_bytes(s, what), st))) return rc;
+  Workspace w = carve(s, what, static_cast<char*>(sc.ptr));
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    return run_attn<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                            static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(proj),
+                            static_cast<float*>(out), o_sparse, w, st);
+  });
+}
+
+int sla_attn(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N, int d,
+             int block, float topk_frac, void* stream) {
+  return sla_attn_ex(q, k, v, proj, out, nullptr, B, H, N, d, block, topk_frac, stream);
+}
+
+int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N,
+                  int d, int block, float topk_frac) {
+  if (!q || !k || !v || !proj || !out) return SLA_ERR_INVALID_ARG;
+  if (!frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  const size_t tb = (size_t)s.BH * N * d * 2, ob = (size_t)s.BH * N * d * 4, pb = (size_t)d * d * 2;
+  cudaStream_t st = nullptr;
+  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return SLA_ERR_CUDA;
+  char* buf = nullptr;
+  const size_t off = (tb + 255) & ~size_t(255), ooff = (ob + 255) & ~size_t(255), poff = (pb + 255) & ~size_t(255);
+  cudaMemPool_t pool = pool_for_current_device();
+  cudaError_t e = pool ? cudaMallocFromPoolAsync(reinterpret_cast<void**>(&buf), 3 * off + ooff + poff, pool, st)
+                       : cudaErrorInitializationError;
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(st);
+    return cuda_status(e);
+  }
+  char *dq = buf, *dk = buf + off, *dv = buf + 2 * off, *dout = buf + 3 * off, *dp = buf + 3 * off + ooff;
+  rc = SLA_OK;
+  if (cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(dp, proj, pb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    rc = SLA_ERR_CUDA;
+  if (rc == SLA_OK) rc = sla_attn(dq, dk, dv, dp, dout, B, H, N, d, block, topk_frac, st);
+  if (rc == SLA_OK && cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess) rc = SLA_ERR_CUDA;
+  cudaFreeAsync(buf, st);
+  const cudaError_t se = cudaStreamSynchronize(st);
+  if (rc == SLA_OK && se != cudaSuccess) rc = SLA_ERR_CUDA;
+  cudaStreamDestroy(st);
+  return rc;
+}
+
+int sla_get_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SLA_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return SLA_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SLA_ERR_CUDA;
+  if (word & DEV_ERR_TIMEOUT) return SLA_ERR_TIMEOUT;
+  if (word & DEV_ERR_INEXACT) return SLA_ERR_INEXACT_MEAN;
+  return SLA_OK;
+}
+
+}  // extern "C"

@@ -390,8 +390,9 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
 
     [P1] 三(二) item 3 (SLA selection, then INT8 computation on the selected
     blocks) and item 2 (the rest through the linear branch and a linear
-    projection); [P3] "SageSLA" section.  Reading: W_proj multiplies O_lin on
-    the right (row vectors); the output is rounded to bf16 at the very end.
+    projection); [P3] "SageSLA" section.  Readings: W_proj multiplies O_lin on
+    the right (row vectors); no output rounding is named, so the result keeps
+    the accumulation precision (float64 here; the CUDA path returns float32).
 
     items: iterable of (b, h, i) query blocks to evaluate (default: all).
     quant/pcast/smooth: False switches off INT8 quantisation (float64 scores),
@@ -399,8 +400,8 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
     idx_override: optional {(b, h, i): key-block list} replacing the mask's
     choice for those rows (used where the mask is a near tie).
 
-    Returns {"out": {(b,h,i): float64 [rows, d]}, "out_bf16": same rounded,
-    "o_sparse", "o_lin", "mask": block_mask(...), "quant": quantize(...)}.
+    Returns {"out": {(b,h,i): float64 [rows, d]}, "o_sparse", "o_lin",
+    "mask": block_mask(...), "quant": quantize(...)}.
     """
     q_bits = np.asarray(q_bits, dtype=np.uint16)
     B, H, N, d = q_bits.shape
@@ -414,7 +415,7 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
     by_head = {}
     for (b, h, i) in items:
         by_head.setdefault((b, h), []).append(i)
-    res = {"out": {}, "out_bf16": {}, "o_sparse": {}, "o_lin": {}, "mask": mask, "quant": qz}
+    res = {"out": {}, "o_sparse": {}, "o_lin": {}, "mask": mask, "quant": qz}
     for (b, h), rows in by_head.items():
         q64 = bf16_to_f64(q_bits[b, h])
         k64 = bf16_to_f64(k_bits[b, h])
@@ -441,5 +442,4 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
             res["o_sparse"][(b, h, i)] = os_
             res["o_lin"][(b, h, i)] = ol
             res["out"][(b, h, i)] = out
-            res["out_bf16"][(b, h, i)] = round_bf16(out)
     return res

@@ -1,0 +1,177 @@
+"""CUDA path vs the CPU oracle, element by element, through the C interface.
+
+Integer work (INT8 codes, scales, the channel mean, the block lists) must be
+bit-exact; a block list may differ only on a row the oracle marks as a near
+tie, and then the oracle is re-run with the GPU's list for that row.  The
+float32 output must be within max-abs 2e-2, mean-abs 2e-3 and cosine 0.9999
+of the oracle's float64 output.
+"""
+
+import numpy as np
+import pytest
+
+import oracle as O
+from synth import CONFIGS, make_inputs, make_workload
+from tests.parity import (assert_out_ok, compare_out, mask_mismatch, sample_items,
+                          to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def S():
+    import torch
+
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import int8_block_sparse_b200 as S
+    from int8_block_sparse_b200.build import build
+
+    build()
+    S.lib()
+    return S
+
+
+def run_quant(S, x, block):
+    q, k = to_dev(x["q"]), to_dev(x["k"])
+    qi8, ki8, sq, sk, mu = S.sla_quant(q, k, block)
+    assert S.get_error() == 0
+    return {"q_i8": qi8.cpu().numpy(), "k_i8": ki8.cpu().numpy(), "q_scale": sq.cpu().numpy(),
+            "k_scale": sk.cpu().numpy(), "mu": mu.cpu().numpy()}
+
+
+def check_quant(got, ref):
+    for key in ("mu", "q_scale", "k_scale"):
+        assert np.array_equal(got[key].view(np.uint32), ref[key].view(np.uint32)), key
+    for key in ("q_i8", "k_i8"):
+        assert np.array_equal(got[key], ref[key]), (key, int(np.sum(got[key] != ref[key])))
+
+
+def run_attn(S, x, block, frac):
+    import torch
+
+    q, k, v, w = (to_dev(x[t]) for t in ("q", "k", "v", "proj"))
+    B, H, N, d = x["q"].shape
+    osp = torch.empty((B, H, N, d), dtype=torch.float32, device="cuda")
+    out = S.sla_attn(q, k, v, w, block=block, topk_frac=frac, o_sparse=osp)
+    idx = S.sla_mask(q, k, block, frac)
+    assert S.get_error() == 0
+    return out.cpu().numpy().astype(np.float64), osp.cpu().numpy().astype(np.float64), idx.cpu().numpy()
+
+
+def check_attn(x, block, frac, items=None):
+    """Full comparison (items None) or on sampled query blocks."""
+    import int8_block_sparse_b200 as S
+
+    out, osp, gidx = run_attn(S, x, block, frac)
+    B, H, N, d = x["q"].shape
+    ref_mask = O.block_mask(x["q"], x["k"], block, frac)
+    diff, bad = mask_mismatch(gidx, ref_mask["idx"], ref_mask["near_tie"])
+    assert not bad.any(), f"{int(bad.sum())} block lists differ off near ties"
+    override = {tuple(int(t) for t in ix): gidx[tuple(ix)] for ix in np.argwhere(diff)}
+    res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, frac, items=items,
+                          idx_override=override or None)
+    got, ref, gs, rs = [], [], [], []
+    for (b, h, i), o in res["out"].items():
+        lo, hi = i * block, min(N, (i + 1) * block)
+        got.append(out[b, h, lo:hi])
+        ref.append(o)
+        gs.append(osp[b, h, lo:hi])
+        rs.append(res["o_sparse"][(b, h, i)])
+    st = compare_out(np.concatenate(got), np.concatenate(ref))
+    st_sp = compare_out(np.concatenate(gs), np.concatenate(rs))
+    assert_out_ok(st_sp, "o_sparse")
+    assert_out_ok(st, "out")
+    return st, st_sp, int(diff.sum())
+
+
+# ---------------------------------------------------------------- small cases
+
+SMALL = [
+    # (B, H, N, d, block, frac, dist, seed)
+    (1, 2, 1024, 64, 64, 0.25, "iid", 0),        # the tiny configuration
+    (1, 1, 1000, 128, 128, 0.25, "iid", 11),     # ragged tail (1000 = 7*128 + 104)
+    (2, 3, 640, 128, 128, 0.4, "iid", 12),       # several heads, B > 1
+    (1, 2, 129, 128, 128, 0.5, "iid", 13),       # last block has one row
+    (1, 1, 1, 128, 128, 0.1, "iid", 14),         # a single token
+    (1, 2, 777, 64, 128, 0.3, "iid", 15),        # d = 64 with 128-token blocks
+    (1, 2, 700, 128, 64, 0.2, "iid", 16),        # 64-token blocks with d = 128
+    (1, 2, 2048, 128, 128, 1.0, "iid", 17),      # every block kept: no linear branch
+    (1, 2, 4096, 128, 128, 0.1, "field", 18),    # field inputs, many blocks
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,block,frac,dist,seed", SMALL)
+def test_quant_bitexact_small(S, B, H, N, d, block, frac, dist, seed):
+    grid = (4, 32, 32) if dist == "field" else None
+    x = make_inputs(B, H, N, d, seed, dist, grid)
+    check_quant(run_quant(S, x, block), O.quantize(x["q"], x["k"], block))
+
+
+@pytest.mark.parametrize("B,H,N,d,block,frac,dist,seed", SMALL)
+def test_attention_small(S, B, H, N, d, block, frac, dist, seed):
+    grid = (4, 32, 32) if dist == "field" else None
+    x = make_inputs(B, H, N, d, seed, dist, grid)
+    check_attn(x, block, frac)
+
+
+def test_mask_bitmap_and_list_agree(S):
+    x = make_inputs(1, 2, 1500, 128, 3)
+    q, k = to_dev(x["q"]), to_dev(x["k"])
+    idx, bm = S.sla_mask(q, k, 128, 0.3, bitmap=True)
+    idx, bm = idx.cpu().numpy(), bm.cpu().numpy()
+    assert np.array_equal(bm, O.bitmap_of(idx, bm.shape[-1]))
+    assert np.all(np.diff(idx, axis=-1) > 0)
+
+
+def test_host_buffers_match_device_path(S):
+    import torch
+
+    x = make_inputs(1, 2, 900, 128, 4)
+    dev = [to_dev(x[t]) for t in ("q", "k", "v", "proj")]
+    out_dev = S.sla_attn(*dev, block=128, topk_frac=0.25)
+    host = [t.cpu().pin_memory() for t in dev]
+    out_host = torch.empty(host[0].shape, dtype=torch.float32).pin_memory()
+    S.sla_attn_host(*host, out_host, block=128, topk_frac=0.25)
+    assert torch.equal(out_host, out_dev.cpu())
+
+
+def test_repeated_calls_are_deterministic(S):
+    import torch
+
+    x = make_inputs(1, 3, 2000, 128, 5, "field", (2, 25, 40))
+    dev = [to_dev(x[t]) for t in ("q", "k", "v", "proj")]
+    a = S.sla_attn(*dev, block=128, topk_frac=0.2)
+    b = S.sla_attn(*dev, block=128, topk_frac=0.2)
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- full-size configurations
+
+def _full_case(S, name, per_head):
+    w = CONFIGS[name]
+    x = make_workload(w)
+    check_quant(run_quant(S, x, w.block), O.quantize(x["q"], x["k"], w.block))
+    items = sample_items(w.B, w.H, w.nblk, per_head=per_head, seed=w.seed)
+    st, st_sp, ndiff = check_attn(x, w.block, w.topk_frac, items=items)
+    print(f"{name}: out {st} o_sparse {st_sp} near-tie rows with other lists: {ndiff}")
+
+
+def test_full_tiny(S):
+    _full_case(S, "tiny", per_head=16)
+
+
+def test_full_480p(S):
+    _full_case(S, "480p", per_head=4)
+
+
+def test_full_dense(S):
+    _full_case(S, "dense", per_head=2)
+
+
+@pytest.mark.parametrize("name", ["sweep0.05", "sweep0.10", "sweep0.20", "sweep0.40"])
+def test_full_sweep(S, name):
+    _full_case(S, name, per_head=2)
+
+
+def test_full_720p(S):
+    _full_case(S, "720p", per_head=2)
