@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Throughput of SageSLA attention on B200: effective (dense-equivalent) TOPS
+and ms per call at the 480P video-DiT shape (B=1, H=12, N=32768, d=128,
+block=128, top-10%), one call of the whole operator per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Every (batch, head) problem is
+independent, so each rank runs its own full-size problem with no collective
+on the data path ("scaling": "weak"); ranks only meet at the timing barriers
+and the max-over-ranks of the elapsed time.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (oracle/, the plain statement of the
+method, run as it stands on the host cores) on a bounded sample of the same
+workload: one query block of a head per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "480p"
+METRIC = "effective sparse-attn TOPS & ms/call, N=32768 H=12 d=128 top-10%, 1 B200"
+UNIT = "TOPS"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "k_attn_480p.md")
+ATTN_SOURCE = os.path.join(ROOT, "int8_block_sparse_b200", "csrc", "k_attn.cuh")
+
+
+# ---------------------------------------------------------------- work accounting
+
+def dense_equivalent_ops(B, H, N, d):
+    """4 * B * H * N^2 * d: QK^T and PV of dense attention, 2 ops per MAC each."""
+    return 4.0 * B * H * N * N * d
+
+
+def critical_ops(B, H, N, d, block, kc):
+    """Ops of the critical-block work: int8 QK^T and bf16 PV, 2*rows*keys*d each.
+
+    With a full last block (N a multiple of block) every selected pair is
+    block x block; otherwise the count is an upper bound by at most one
+    partial block per row (the 480P workload has no partial block)."""
+    nblk = (N + block - 1) // block
+    pairs = B * H * nblk * kc
+    per = 2.0 * block * block * d
+    return pairs * per, pairs * per
+
+
+def attn_roofline(qk_ops, pv_flops, peaks):
+    """Peak for the mixed kernel: ops / (QK at the int8 peak + PV at the bf16 peak)."""
+    if peaks is not None:
+        bf16 = float(peaks["bf16_tflops"])
+        src = "measured (MEASURED_PEAKS.json bf16_tflops burst; int8 = 2 x bf16, nominal ratio)"
+    else:
+        bf16 = FALLBACK_BF16_TFLOPS
+        src = "fallback 1.59 PFLOP/s bf16 (int8 = 2 x bf16, nominal ratio)"
+    i8 = 2.0 * bf16
+    t_roof = qk_ops / (i8 * 1e12) + pv_flops / (bf16 * 1e12)
+    return (qk_ops + pv_flops) / t_roof / 1e12, src
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return None
+
+
+def profiled_traffic():
+    """DRAM bytes per k_attn launch from the committed ncu summary, if it was
+    taken on the kernel source as it is now (else None)."""
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            text = f.read()
+        with open(ATTN_SOURCE, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("k_attn.cuh sha256") != sha:
+        return None
+    try:
+        return float(vals["dram bytes per launch (480p)"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+class Dist:
+    def __init__(self, n_gpus):
+        import torch
+
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world != n_gpus:
+            raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE {self.world}")
+        self.pg = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        return reduce_max(x, self.pg)
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+def reduce_max(x: float, dist_mod=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist_mod is None:
+        return float(x)
+    import torch
+
+    dev = "cuda" if dist_mod.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist_mod.all_reduce(t, op=dist_mod.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(ops_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput in TOPS: all ranks' work over the slowest rank's time."""
+    return ops_per_rank * world / max_seconds / 1e12
+
+
+# ---------------------------------------------------------------- clocks
+
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of this rank's GPU during the timed region."""
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            sel = str(device_index)
+        self.sel = sel
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(w, nq: int):
+    """Time the CPU oracle on head 0 of the workload: its quantisation, mask and
+    states plus the outputs of nq query blocks.  Returns (seconds, ops, sample)."""
+    import numpy as np
+
+    import oracle as O
+    from synth import make_workload
+
+    x = make_workload(w, heads=[0])
+    items = [(0, 0, i) for i in np.linspace(0, w.nblk - 1, nq).astype(int)]
+    t0 = time.perf_counter()
+    O.sla_attention(x["q"], x["k"], x["v"], x["proj"], w.block, w.topk_frac, items=items)
+    dt = time.perf_counter() - t0
+    ops = nq * 4.0 * w.block * w.N * w.d   # dense-equivalent ops of nq query blocks
+    return dt, ops, (f"CPU oracle on head 0 of {w.name}: per-head quantisation, mask and linear "
+                     f"states, then {nq} query blocks of {w.block} rows; value = dense-equivalent "
+                     f"ops of those rows / wall time")
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------- arms
+
+def run_ours(args, dist):
+    import numpy as np
+    import torch
+
+    import int8_block_sparse_b200 as S
+    from int8_block_sparse_b200.build import build
+    from synth import CONFIGS, make_workload
+
+    build()
+    S.lib()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    w = CONFIGS[WORKLOAD]
+    if args.heads:
+        import dataclasses
+
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}-first{args.heads}heads")
+        x = make_workload(CONFIGS[WORKLOAD], heads=list(range(args.heads)))
+    else:
+        x = make_workload(w)
+    t = {k: torch.from_numpy(x[k].view(np.int16)).view(torch.bfloat16).to(dev) for k in ("q", "k", "v", "proj")}
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        S.sla_attn(t["q"], t["k"], t["v"], t["proj"], block=w.block, topk_frac=w.topk_frac, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc = S.get_error()
+    if rc != 0:
+        raise SystemExit(f"device error after warm-up: {S.status_string(rc)}")
+
+    sampler = ClockSampler(dist.local)
+    sampler.start()
+    S.profile_read()
+    S.profile_enable(True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    S.profile_enable(False)
+    clocks = sampler.stop()
+    prof = S.profile_read()
+    rc = S.get_error()
+    if rc != 0:
+        raise SystemExit(f"device error in the timed region: {S.status_string(rc)}")
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = dist.max(ms_local)
+
+    ops = dense_equivalent_ops(w.B, w.H, w.N, w.d)
+    value = weak_scaling_value(ops, dist.world, ms / 1e3)
+    kc = S.topk_count(w.N, w.block, w.topk_frac)
+    qk, pv = critical_ops(w.B, w.H, w.N, w.d, w.block, kc)
+    peaks = load_peaks()
+    peak, peak_src = attn_roofline(qk, pv, peaks)
+    attn_ms, attn_n = prof["attn"]
+    attn_avg = attn_ms / max(attn_n, 1)
+    achieved = (qk + pv) / (attn_avg / 1e3) / 1e12
+    roof = {"bound": "tensor", "kernel": "k_attn<128,128> (critical-block attention)",
+            "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+            "peak_source": peak_src, "ops_per_launch": qk + pv,
+            "kernel_ms": round(attn_avg, 4)}
+    launches = int(sum(n for _, n in prof.values()))
+    kernels = {k: {"ms_per_call": round(v[0] / max(v[1], 1), 4), "launches": int(v[1])} for k, v in prof.items()}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(S, t, w, args, dist)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8,bf16 (f32 accumulate)",
+        "data": "synthetic (seeded field-plus-noise, see synth/workloads.py)",
+        "config": {"workload": w.describe(), "kc": kc,
+                   "parallelism": f"replicas x{dist.world} (independent problems per rank)",
+                   "l2": "inputs larger than L2 (q, k, v: 302 MB; ~1 GB moved per call), no flush"},
+        "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "e2e": e2e,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
+        dt, cops, sample = oracle_sample(w, args.cpu_query_blocks)
+        line["cpu_baseline"] = {"value": round(cops / dt / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+    return line
+
+
+def run_e2e(S, t, w, args, dist):
+    """Same metric through the host-buffer entry point: H2D of q, k, v, proj,
+    the operator, D2H of out, every step (host wall clock around the
+    synchronous call)."""
+    import torch
+
+    host = {k: v.cpu().pin_memory() for k, v in t.items()}
+    hout = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32).pin_memory()
+    S.sla_attn_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block, topk_frac=w.topk_frac)
+    n = max(1, min(args.steps, args.e2e_steps))
+    dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        S.sla_attn_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block,
+                        topk_frac=w.topk_frac)
+    dt = dist.max((time.perf_counter() - t0) / n)
+    ops = dense_equivalent_ops(w.B, w.H, w.N, w.d)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = hout.numel() * hout.element_size()
+    return {"value": round(weak_scaling_value(ops, dist.world, dt), 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(dt * 1e3, 3),
+            "steps": n, "timer": "host wall clock around sla_attn_host (synchronous)"}
+
+
+def run_reference(args, dist):
+    """The CPU oracle as the reference arm: one query block per step."""
+    import numpy as np
+
+    import oracle as O
+    from synth import CONFIGS, make_workload
+
+    w = CONFIGS[WORKLOAD]
+    if dist.rank != 0:
+        return None
+    x = make_workload(w, heads=[0])
+    # per-head preparation (quantisation, mask, linear states) is timed once
+    # and amortised over the workload's query blocks in the reported value
+    t0 = time.perf_counter()
+    res0 = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], w.block, w.topk_frac, items=[(0, 0, 0)])
+    prep = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    blocks = rng.integers(0, w.nblk, size=args.warmup + args.steps)
+    q64 = O.bf16_to_f64(x["q"][0, 0])
+    k64 = O.bf16_to_f64(x["k"][0, 0])
+    v64 = O.bf16_to_f64(x["v"][0, 0])
+    w64 = O.bf16_to_f64(x["proj"])
+    hst, zst = O.linear_states(k64, v64, w.block)
+    qz, mask = res0["quant"], res0["mask"]
+
+    def step(i):
+        crit = mask["idx"][0, 0, i]
+        lo, hi = i * w.block, min(w.N, (i + 1) * w.block)
+        os_ = O.critical_rows(qz["q_i8"][0, 0, lo:lo + w.block], qz["q_scale"][0, 0, i], qz["k_i8"][0, 0],
+                              qz["k_scale"][0, 0], v64, crit, w.N, w.block)[:hi - lo]
+        return os_ + np.matmul(O.linear_rows(q64[lo:hi], hst, zst, crit), w64)
+
+    for i in blocks[:args.warmup]:
+        step(int(i))
+    t0 = time.perf_counter()
+    for i in blocks[args.warmup:]:
+        step(int(i))
+    per = (time.perf_counter() - t0) / max(args.steps, 1)
+    per_block = per + prep / w.nblk
+    ops = 4.0 * w.block * w.N * w.d
+    value = ops / per_block / 1e12
+    ms_call = per_block * w.nblk * w.B * w.H * 1e3
+    sample = (f"CPU oracle, {args.steps} steps of one query block ({w.block} rows) of head 0 of {w.name}; "
+              f"per-head preparation {prep:.2f} s amortised over its {w.nblk} query blocks")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_call, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (int8 codes)",
+            "data": "synthetic (seeded field-plus-noise, see synth/workloads.py)",
+            "config": {"workload": w.describe(), "note": "ms_per_step = projected time of one full call"},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-query-blocks", type=int, default=64)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="keep only the first H heads (a smaller case for profiling; not the headline)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+
+        class _D:
+            pass
+
+        d = _D()
+        d.rank, d.world = 0, world
+        line = run_reference(args, d)
+        print(json.dumps(line), flush=True)
+        return 0
+    dist = Dist(args.gpus)
+    try:
+        line = run_ours(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -122,6 +122,27 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
  * SLA_ERR_CUDA if the synchronisation itself failed, else SLA_OK. */
 int sla_get_error(void* stream);
 
+/* Kernel kinds, in the order sla_profile_read() reports them. */
+typedef enum {
+  SLA_K_STATS = 0,   /* K block sums and linear states              */
+  SLA_K_MEAN = 1,    /* per-channel mean of K                        */
+  SLA_K_QUANT = 2,   /* smoothing + INT8 quantisation (+ Q block sums) */
+  SLA_K_MASK = 3,    /* pooled scores + top-k                        */
+  SLA_K_ATTN = 4,    /* critical-block attention                     */
+  SLA_K_LINGEMM = 5, /* sums of the non-selected states              */
+  SLA_K_LINOUT = 6,  /* linear branch, projection, add               */
+  SLA_K_COUNT = 7
+} sla_kernel_kind;
+
+/* Measurement support (no counterpart on the pages).  While enabled, every
+ * kernel the library launches is bracketed by two CUDA events recorded on the
+ * stream it runs on.  sla_profile_read() waits for those events, writes per
+ * kernel kind the summed device milliseconds (ms[k]) and the number of
+ * launches (launches[k]) for k < n (n <= SLA_K_COUNT), and clears them.
+ * Either array may be NULL.  Returns SLA_OK or SLA_ERR_CUDA. */
+int sla_profile_enable(int on);
+int sla_profile_read(double* ms, long long* launches, int n);
+
 /* Static description of a status code (never NULL). */
 const char* sla_status_string(int status);
 

@@ -20,7 +20,9 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
                 4: "SLA_ERR_OOM", 5: "SLA_ERR_TIMEOUT", 6: "SLA_ERR_INEXACT_MEAN"}
 
 EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
-           "sla_get_error", "sla_status_string")
+           "sla_get_error", "sla_status_string", "sla_profile_enable", "sla_profile_read")
+
+KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm", "linout")
 
 
 class SlaError(RuntimeError):
@@ -49,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.sla_get_error.argtypes = [vp]
         L.sla_status_string.argtypes = [i]
         L.sla_status_string.restype = ctypes.c_char_p
+        L.sla_profile_enable.argtypes = [i]
+        L.sla_profile_read.argtypes = [vp, vp, i]
         for name in EXPORTS:
             if name != "sla_status_string":
                 getattr(L, name).restype = i
@@ -147,6 +151,21 @@ def sla_attn_host(q, k, v, proj, out, block: int = 128, topk_frac: float = 0.1) 
     B, H, N, d = _shape(q)
     _check(lib().sla_attn_host(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
                                float(topk_frac)), "sla_attn_host")
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events (see sla_profile_read)."""
+    lib().sla_profile_enable(1 if on else 0)
+
+
+def profile_read() -> dict:
+    """{kernel kind: (summed device ms, launches)} since the last read; clears them."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    _check(lib().sla_profile_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p), n),
+           "sla_profile_read")
+    return {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}
 
 
 def get_error(stream=None) -> int:

@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "sla.h"
 #include "k_attn.cuh"
@@ -174,6 +175,33 @@ int cuda_status(cudaError_t e) {
   return SLA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ optional per-kernel timing
+struct ProfRecord {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof;
+
+// Records an event before the launch that follows and one after it (at scope exit).
+struct ProfScope {
+  int kind;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr, b = nullptr;
+  ProfScope(int k, cudaStream_t s) : kind(k), st(s) {
+    if (!g_prof_on) return;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return;
+    cudaEventRecord(a, st);
+  }
+  ~ProfScope() {
+    if (a == nullptr || b == nullptr) return;
+    cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back({kind, a, b});
+  }
+};
+
 // ------------------------------------------------------------------ launch helpers
 template <int D, int BLK>
 int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
@@ -182,12 +210,15 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
   const size_t sm1 = kstats_smem<D, BLK>();
   cudaFuncSetAttribute(k_kstats<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
   dim3 g1((unsigned)s.NB, (unsigned)s.BH);
+  { ProfScope ps(SLA_K_STATS, st);
   k_kstats<D, BLK><<<g1, 256, sm1, st>>>(k, v, w.ksum, w.kexp, states ? w.hstate : nullptr, s.N, (int)s.NB,
-                                         w.hpitch);
+                                         w.hpitch); }
   const long long tot = s.BH * D;
-  k_channel_mean<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, D, s.N, tot);
+  { ProfScope ps(SLA_K_MEAN, st);
+  k_channel_mean<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, D, s.N, tot); }
   dim3 g2((unsigned)s.NB, (unsigned)s.BH, kcodes ? 2u : 1u);
-  k_quant<D, BLK><<<g2, 256, 0, st>>>(q, k, w.mu, qi8, ki8, sq, sk, w.qsum, s.N, (int)s.NB);
+  { ProfScope ps(SLA_K_QUANT, st);
+  k_quant<D, BLK><<<g2, 256, 0, st>>>(q, k, w.mu, qi8, ki8, sq, sk, w.qsum, s.N, (int)s.NB); }
   return cuda_status(cudaGetLastError());
 }
 
@@ -199,6 +230,7 @@ int launch_mask(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __n
   const size_t sm = mask_smem<D>(rows, (int)s.NB);
   cudaFuncSetAttribute(k_mask<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   dim3 g((unsigned)((s.NB + rows - 1) / rows), (unsigned)s.BH);
+  ProfScope ps(SLA_K_MASK, st);
   k_mask<D><<<g, 256, sm, st>>>(w.qsum, w.ksum, s.N, (int)s.NB, s.block, (int)s.kc, rows, idx, bitmap, notcrit,
                                 (int)w.ncpitch);
   return cuda_status(cudaGetLastError());
@@ -241,6 +273,7 @@ int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* v, float* o, 
   p.qk_scale = (float)(1.4426950408889634 / std::sqrt((double)D));
   cudaFuncSetAttribute(k_attn<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int ctas = (int)std::min<long long>(num_sms(), (p.items + 1) / 2);
+  ProfScope ps(SLA_K_ATTN, st);
   k_attn<D, BLK><<<ctas, 384, C::SMEM, st>>>(mq, mk, mv, p);
   return cuda_status(cudaGetLastError());
 }
@@ -282,13 +315,15 @@ int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __
   gp.nkt = (int)((s.NB + 63) / 64);
   cudaFuncSetAttribute(k_lingemm, cudaFuncAttributeMaxDynamicSharedMemorySize, LG_SMEM);
   dim3 g1((unsigned)((gp.E + 255) / 256), (unsigned)((s.NB + 127) / 128), (unsigned)s.BH);
-  k_lingemm<<<g1, 128, LG_SMEM, st>>>(ma, mb, gp);
+  { ProfScope ps(SLA_K_LINGEMM, st);
+  k_lingemm<<<g1, 128, LG_SMEM, st>>>(ma, mb, gp); }
   LinOutParams op;
   op.q = q; op.zrest = w.zrest; op.osparse = osparse; op.out = out;
   op.N = s.N; op.NB = (int)s.NB; op.BLK = s.block;
   cudaFuncSetAttribute(k_linout<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinOutCfg<D>::SMEM);
   dim3 g2((unsigned)s.NB, (unsigned)s.BH);
-  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, mw, op);
+  { ProfScope ps(SLA_K_LINOUT, st);
+  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, mw, op); }
   return cuda_status(cudaGetLastError());
 }
 
@@ -468,6 +503,38 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
   const cudaError_t se = cudaStreamSynchronize(st);
   if (rc == SLA_OK && se != cudaSuccess) rc = SLA_ERR_CUDA;
   cudaStreamDestroy(st);
+  return rc;
+}
+
+int sla_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return SLA_OK;
+}
+
+int sla_profile_read(double* ms, long long* launches, int n) {
+  std::vector<ProfRecord> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    recs.swap(g_prof);
+  }
+  if (n > SLA_K_COUNT) n = SLA_K_COUNT;
+  for (int k = 0; k < n; ++k) {
+    if (ms) ms[k] = 0.0;
+    if (launches) launches[k] = 0;
+  }
+  int rc = SLA_OK;
+  for (const ProfRecord& r : recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      rc = SLA_ERR_CUDA;
+    if (r.kind < n) {
+      if (ms) ms[r.kind] += t;
+      if (launches) launches[r.kind] += 1;
+    }
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
   return rc;
 }
 
