@@ -69,10 +69,12 @@ typedef enum {
   SLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                   */
   SLA_ERR_OOM = 4,          /* temporary device memory could not be obtained       */
   SLA_ERR_TIMEOUT = 5,      /* a kernel's bounded wait gave up (sla_get_error)     */
-  SLA_ERR_INEXACT_MEAN = 6  /* the K channel mean could not be proven exact: some
+  SLA_ERR_INEXACT_MEAN = 6, /* the K channel mean could not be proven exact: some
                                channel's values span more exponents than a float64
                                sum holds exactly (sla_get_error; results are still
                                written)                                            */
+  SLA_ERR_SCRATCH_LIMIT = 7 /* sla_mask_noalloc: the problem needs more scratch than
+                               its fixed device buffer holds                       */
 } sla_status;
 
 /* Number of key blocks each query block keeps:
@@ -96,6 +98,35 @@ int sla_quant(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q
  *   bitmap  : out, uint8 [B,H,nblk,nblk], 1 where kept, or NULL */
 int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, int B, int H, int N, int d,
              int block, float topk_frac, void* stream);
+
+/* Size of the fixed device scratch buffer behind sla_mask_noalloc. */
+#define SLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* sla_mask without any device memory allocation.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot call
+ * cudaMalloc or any allocator while they run, for example an inference server
+ * that plans every byte of device memory at start-up and forbids allocation
+ * afterwards (so that memory use stays predictable and cannot fail with
+ * out-of-memory mid-request), or a host that owns the device allocator
+ * through another framework.
+ *   Arguments, outputs and errors are those of sla_mask.  The block sums the
+ * mask needs live in one file-scope device buffer of
+ * SLA_NOALLOC_SCRATCH_BYTES (16 MiB) in this library, which every GPU that
+ * loads the library holds until the process exits.  A problem must fit in
+ * it: 18 * B*H*nblk*d + 4 * B*H*d bytes, each part rounded up to 256 bytes
+ * (for example B*H = 12, nblk = 256, d = 128 fits; B*H = 40, nblk = 591
+ * does not); larger ones return SLA_ERR_SCRATCH_LIMIT before any work is
+ * enqueued.
+ *   The first call on a device looks up the buffer's device address (once
+ * per device, with that device current); make that first call before any
+ * stream capture.  No allocation happens on that or any later call (keep
+ * sla_profile_enable off, its default: profiling creates CUDA events).
+ *   All calls on a device share the one buffer and it keeps the last call's
+ * contents; every scratch element is written before it is read, so nothing
+ * needs clearing.  Calls whose work overlaps on the GPU (for example on two
+ * streams without ordering between them) race on the buffer: order them. */
+int sla_mask_noalloc(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, int B, int H, int N, int d,
+                     int block, float topk_frac, void* stream);
 
 /* The whole operator, steps 1-6 ([P1] 三(二) 3, SageSLA).
  *   q, k, v : in,  bf16 [B,H,N,d]

@@ -373,6 +373,28 @@ struct Scratch {
   }
 };
 
+// ------------------------------------------------------------------ fixed scratch for sla_mask_noalloc
+// For callers that cannot allocate device memory while they run: the block
+// sums of sla_mask_noalloc live here instead of in the stream-ordered pool.
+// Host code must not use this name as an address; see noalloc_scratch().
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SLA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (cudaGetSymbolAddress, checked); nullptr if the lookup failed.
+void* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -393,6 +415,7 @@ const char* sla_status_string(int status) {
     case SLA_ERR_OOM: return "out of device memory";
     case SLA_ERR_TIMEOUT: return "a kernel wait timed out";
     case SLA_ERR_INEXACT_MEAN: return "K channel mean not proven exact";
+    case SLA_ERR_SCRATCH_LIMIT: return "problem larger than the fixed no-allocation scratch buffer";
     default: return "unknown status";
   }
 }
@@ -431,6 +454,30 @@ int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, in
   Scratch sc;
   if ((rc = sc.get(workspace_bytes(s, 0), st))) return rc;
   Workspace w = carve(s, 0, static_cast<char*>(sc.ptr));
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                       static_cast<const __nv_bfloat16*>(k), w, false, false, nullptr, nullptr,
+                                       nullptr, nullptr, st);
+    if (r) return r;
+    return launch_mask<D>(s, w, blk_idx, bitmap, nullptr, st);
+  });
+}
+
+int sla_mask_noalloc(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, int B, int H, int N, int d,
+                     int block, float topk_frac, void* stream) {
+  if (!q || !k || !blk_idx) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return SLA_ERR_INVALID_ARG;
+  if (!frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  s.kc = topk_count_ll(s.NB, topk_frac);
+  if (workspace_bytes(s, 0) > SLA_NOALLOC_SCRATCH_BYTES) return SLA_ERR_SCRATCH_LIMIT;
+  void* scratch = noalloc_scratch();
+  if (scratch == nullptr) return SLA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Workspace w = carve(s, 0, static_cast<char*>(scratch));
   return with_dims(d, block, [&](auto D_, auto B_) {
     constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
     int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
