@@ -16,8 +16,13 @@
 //   warp 1 / 3   tcgen05.mma issuer of tile 0 / 1
 //   warps 4-7    softmax + epilogue of tile 0 (thread = query row = TMEM lane)
 //   warps 8-11   softmax + epilogue of tile 1
-// TMEM (512 columns): tile u uses columns [256u, 256u+128) for S (P, bf16,
-// is written over the first half of S) and [256u+128, 256u+128+D) for O.
+// A tile walks its key blocks in halves of 64 keys.  TMEM (512 columns): tile
+// u owns columns [256u, 256u+256): two S buffers of 64 columns (S for half h
+// goes to buffer h % 2; P, bf16, is written over the first 32 columns of its
+// S) and O in [256u+128, 256u+128+D).  With two S buffers the QK^T of the next
+// half is already queued on the tensor core while the softmax of this half
+// runs.  The tensor core executes one CTA's MMAs in issue order, so a QK^T
+// issued after a PV may overwrite the S buffer that PV reads P from.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -36,6 +41,8 @@ struct AttnParams {
 template <int D, int BLK>
 struct AttnCfg {
   static constexpr int BQ = 128;                 // query rows per tile (MMA M)
+  static constexpr int HB = 64;                  // keys per half block (MMA N of QK^T)
+  static constexpr int NH = BLK / HB;            // halves per key block
   static constexpr int Q_BYTES = BQ * D;         // int8
   static constexpr int K_BYTES = BLK * D;        // int8
   static constexpr int V_BYTES = BLK * D * 2;    // bf16
@@ -46,10 +53,13 @@ struct AttnCfg {
   static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
   static constexpr uint32_t KSW = (D == 128) ? 2u : 4u;     // Q/K swizzle: 128B or 64B rows
   static constexpr uint32_t KSBO = (D == 128) ? 1024u : 512u;
+  static constexpr uint32_t K_HALF_BYTES = HB * D;          // 64 rows of K (int8)
+  static constexpr uint32_t V_HALF_BYTES = HB * 128;        // 64 rows of one 64-channel V atom
 };
 
 struct TileBars {
-  uint64_t q_full, q_empty, s_full, p_full, o_full, o_free;
+  uint64_t q_full, q_empty, pv_done, o_full, o_free;
+  uint64_t s_full[2], p_full[2];
   uint64_t kv_full[2], kv_empty[2];
 };
 
@@ -64,6 +74,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
                                                  const __grid_constant__ CUtensorMap tm_k,
                                                  const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D, BLK>;
+  constexpr int NH = C::NH;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -78,11 +89,12 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
       TileBars& b = bars[u];
       mbar_init(&b.q_full, 1);
       mbar_init(&b.q_empty, 1);
-      mbar_init(&b.s_full, 1);
-      mbar_init(&b.p_full, 128);
+      mbar_init(&b.pv_done, 1);
       mbar_init(&b.o_full, 1);
       mbar_init(&b.o_free, 128);
       for (int s = 0; s < 2; ++s) {
+        mbar_init(&b.s_full[s], 1);
+        mbar_init(&b.p_full[s], 128);
         mbar_init(&b.kv_full[s], 1);
         mbar_init(&b.kv_empty[s], 1);
       }
@@ -107,66 +119,102 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
     const int u = warp >> 1;
     TileBars& b = bars[u];
     unsigned char* tq = base + u * C::TILE_BYTES;
-    unsigned char* tk[2] = {tq + C::Q_BYTES, tq + C::Q_BYTES + C::K_BYTES + C::V_BYTES};
-    unsigned char* tv[2] = {tk[0] + C::K_BYTES, tk[1] + C::K_BYTES};
     if ((warp & 1) == 0) {
       // ------------------------------------------------------------ producer
+      // The whole warp walks the block list (32 entries per load); lane 0
+      // issues the waits and the TMA copies.
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        uint32_t kv_it = 0, item_it = 0;
-        bool ok = true;
-        for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
-          const int bh = item / NB, i = item % NB;
-          if (!(ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag))) break;
-          mbar_expect_tx(&b.q_full, C::Q_BYTES);
-          tma_load_2d(tq, &tm_q, &b.q_full, 0, bh * p.NP + i * BLK);
-          const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
-          for (int t = 0; t < kc; ++t, ++kv_it) {
-            const int j = __ldg(lst + t);
-            const int s = kv_it & 1;
-            if (!(ok = mbar_wait(&b.kv_empty[s], ((kv_it >> 1) & 1) ^ 1, abort_flag))) break;
-            mbar_expect_tx(&b.kv_full[s], C::K_BYTES + C::V_BYTES);
-            tma_load_2d(tk[s], &tm_k, &b.kv_full[s], 0, bh * p.NP + j * BLK);
-#pragma unroll
-            for (int hh = 0; hh < D / 64; ++hh)
-              tma_load_3d(tv[s] + hh * BLK * 128, &tm_v, &b.kv_full[s], hh * 64, j * BLK, bh);
+      }
+      uint32_t kv_it = 0, item_it = 0;
+      int ok = 1;
+      for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
+        const int bh = item / NB, i = item % NB;
+        if (lane == 0) {
+          ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag);
+          if (ok) {
+            mbar_expect_tx(&b.q_full, C::Q_BYTES);
+            tma_load_2d(tq, &tm_q, &b.q_full, 0, bh * p.NP + i * BLK);
           }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
+        int jl = 0;
+        for (int t = 0; t < kc && ok; ++t, ++kv_it) {
+          if ((t & 31) == 0) jl = (t + lane < kc) ? __ldg(lst + t + lane) : 0;
+          const int j = __shfl_sync(0xffffffffu, jl, t & 31);
+          if (lane == 0) {
+            const int s = kv_it & 1;
+            unsigned char* tk = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES);
+            unsigned char* tv = tk + C::K_BYTES;
+            ok = mbar_wait(&b.kv_empty[s], ((kv_it >> 1) & 1) ^ 1, abort_flag);
+            if (ok) {
+              mbar_expect_tx(&b.kv_full[s], C::K_BYTES + C::V_BYTES);
+              tma_load_2d(tk, &tm_k, &b.kv_full[s], 0, bh * p.NP + j * BLK);
+#pragma unroll
+              for (int hh = 0; hh < D / 64; ++hh)
+                tma_load_3d(tv + hh * BLK * 128, &tm_v, &b.kv_full[s], hh * 64, j * BLK, bh);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
         }
       }
     } else {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
-        const uint32_t tS = tmem_base + u * 256;
+        const uint32_t tS = tmem_base + u * 256;   // S buffers at tS and tS + 64
         const uint32_t tO = tS + 128;
-        const uint32_t id_qk = idesc_i8(BLK);
+        const uint32_t id_qk = idesc_i8(C::HB);
         const uint32_t id_pv = idesc_bf16(D, false, true);
         const uint64_t dq = smem_desc(smem_u32(tq), 16, C::KSBO, C::KSW);
-        uint32_t kv_it = 0, item_it = 0, it = 0;
+        uint32_t kv_it = 0, item_it = 0, hg = 0;   // hg: halves of the items before this one
         bool ok = true;
         for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
+          const int H = kc * NH;
           if (!(ok = mbar_wait(&b.q_full, item_it & 1, abort_flag))) break;
-          for (int t = 0; t < kc; ++t, ++kv_it, ++it) {
-            const int s = kv_it & 1;
-            if (!(ok = mbar_wait(&b.kv_full[s], (kv_it >> 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            const uint64_t dk = smem_desc(smem_u32(tk[s]), 16, C::KSBO, C::KSW);
+          // S(y) = Q K_half(y)^T into buffer (hg + y) % 2; at the first half of a
+          // key block it first waits for that block's K/V stage
+          auto issue_qk = [&](int y) -> bool {
+            const uint32_t g = hg + y;
+            const uint32_t blk_it = kv_it + y / NH;
+            const int s = blk_it & 1;
+            if (y % NH == 0) {
+              if (!mbar_wait(&b.kv_full[s], (blk_it >> 1) & 1, abort_flag)) return false;
+              tc_fence_after();
+            }
+            unsigned char* tk = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES);
+            const uint64_t dk = smem_desc(smem_u32(tk) + (y % NH) * C::K_HALF_BYTES, 16, C::KSBO, C::KSW);
+            const uint32_t dS = tS + (g & 1) * 64;
 #pragma unroll
             for (int kk = 0; kk < D / 32; ++kk)
-              mma_i8_ss(tS, dq + uint64_t(kk * 2), dk + uint64_t(kk * 2), id_qk, kk > 0 ? 1u : 0u);
-            tc_commit(&b.s_full);
-            if (t == kc - 1) tc_commit(&b.q_empty);
-            if (!(ok = mbar_wait(&b.p_full, it & 1, abort_flag))) break;
-            if (t == 0 && !(ok = mbar_wait(&b.o_free, (item_it & 1) ^ 1, abort_flag))) break;
+              mma_i8_ss(dS, dq + uint64_t(kk * 2), dk + uint64_t(kk * 2), id_qk, kk > 0 ? 1u : 0u);
+            tc_commit(&b.s_full[g & 1]);
+            if (y == H - 1) tc_commit(&b.q_empty);
+            return true;
+          };
+          ok = issue_qk(0);
+          if (ok && H > 1) ok = issue_qk(1);
+          for (int x = 0; x < H && ok; ++x) {
+            const uint32_t g = hg + x;
+            if (!(ok = mbar_wait(&b.p_full[g & 1], (g >> 1) & 1, abort_flag))) break;
+            if (x == 0 && !(ok = mbar_wait(&b.o_free, (item_it & 1) ^ 1, abort_flag))) break;
             tc_fence_after();
-            const uint64_t dv = smem_desc(smem_u32(tv[s]), BLK * 128, 1024, 2);
+            const int s = (kv_it + x / NH) & 1;
+            unsigned char* tv = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES) + C::K_BYTES;
+            const uint64_t dv = smem_desc(smem_u32(tv) + (x % NH) * C::V_HALF_BYTES, BLK * 128, 1024, 2);
+            const uint32_t aP = tS + (g & 1) * 64;
 #pragma unroll
-            for (int kk = 0; kk < BLK / 16; ++kk)
-              mma_bf16_ts(tO, tS + kk * 8, dv + uint64_t(kk * (2048 >> 4)), id_pv, (t > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&b.kv_empty[s]);
-            if (t == kc - 1) tc_commit(&b.o_full);
+            for (int kk = 0; kk < C::HB / 16; ++kk)
+              mma_bf16_ts(tO, aP + kk * 8, dv + uint64_t(kk * (2048 >> 4)), id_pv, (x > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&b.pv_done);
+            if (x % NH == NH - 1) tc_commit(&b.kv_empty[s]);
+            if (x == H - 1) tc_commit(&b.o_full);
+            if (x + 2 < H) ok = issue_qk(x + 2);
           }
+          hg += H;
+          kv_it += kc;
         }
       }
     }
@@ -178,87 +226,122 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem_base + u * 256 + lane_off;
     const uint32_t tO = tS + 128;
-    uint32_t item_it = 0, it = 0;
+    uint32_t item_it = 0, hg = 0;
     bool ok = true;
+    const int part_rows = p.N % BLK;                // rows of a partial last block (0: none)
     for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
       const int bh = item / NB, i = item % NB;
-      const float sq_i = __ldg(p.sq + (long long)bh * NB + i);
+      const float sq_i = __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale;
       const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
+      const int H = kc * NH;
+      // running maximum m (log2 domain) and normaliser l of this row
       float m = -INFINITY, l = 0.f;
-      for (int t = 0; t < kc; ++t, ++it) {
-        const int j = __ldg(lst + t);
-        const float c = sq_i * __ldg(p.sk + (long long)bh * NB + j) * p.qk_scale;
-        const int nvalid = p.N - j * BLK;
-        if (!(ok = mbar_wait(&b.s_full, it & 1, abort_flag))) break;
-        tc_fence_after();
-        float mx = -INFINITY;
-#pragma unroll
-        for (int ch = 0; ch < BLK / 16; ++ch) {
-          uint32_t v[16];
-          SLA_TMEM_LD16(tS + ch * 16, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float x = (float)(int)v[e] * c;
-            if (ch * 16 + e >= nvalid) x = -INFINITY;
-            mx = fmaxf(mx, x);
-          }
+      float cl = 0.f;
+      int jl = 0;
+      for (int x = 0; x < H; ++x) {
+        const int t = x / NH;
+        const uint32_t g = hg + x;
+        if ((t & 31) == 0 && x % NH == 0) {   // block list and scales, 32 blocks at a time
+          jl = (t + lane < kc) ? __ldg(lst + t + lane) : 0;
+          cl = sq_i * __ldg(p.sk + (long long)bh * NB + jl);
         }
-        const float m_new = fmaxf(m, mx);
-        // tcgen05.ld/st are warp-collective: the whole warp rescales when any
-        // of its rows has a new maximum (alpha is exactly 1 for the others).
-        if (t > 0 && __any_sync(0xffffffffu, m_new > m)) {
-          const float alpha = (m_new > m) ? ex2_approx(m - m_new) : 1.f;
-          l *= alpha;
+        const int j = __shfl_sync(0xffffffffu, jl, t & 31);
+        const float c = __shfl_sync(0xffffffffu, cl, t & 31);   // sq_i * sk_j * log2(e) / sqrt(D) >= 0
+        // valid keys of this half (fewer only in a partial last block)
+        const int nvalid = (part_rows != 0 && j == NB - 1)
+                               ? min(max(part_rows - (x % NH) * C::HB, 0), C::HB)
+                               : C::HB;
+        const bool partial = nvalid < C::HB;       // uniform across the CTA
+        if (!(ok = mbar_wait(&b.s_full[g & 1], (g >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t sbuf = tS + (g & 1) * 64;
+        uint32_t v[64];
+        SLA_TMEM_LD32(sbuf, v);
+        SLA_TMEM_LD32(sbuf + 32, (v + 32));
+        tmem_ld_wait();
+        // row maximum of the int32 scores (c >= 0 keeps the order)
+        int amax = INT_MIN;
+        if (!partial) {
 #pragma unroll
-          for (int ch = 0; ch < D / 16; ++ch) {
-            uint32_t v[16];
-            SLA_TMEM_LD16(tO + ch * 16, v);
+          for (int e = 0; e < 64; ++e) amax = max(amax, (int)v[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (e < nvalid) amax = max(amax, (int)v[e]);
+        }
+        const float mx = (nvalid > 0) ? (float)amax * c : -INFINITY;
+        bool pv_waited = false;
+        if (x == 0) {
+          m = mx;
+        } else if (__any_sync(0xffffffffu, mx > m + 8.f)) {
+          // Some row's maximum grew by more than 2^8: once the previous PV has
+          // finished, the warp rescales O (tcgen05.ld/st are warp-collective);
+          // rows whose maximum did not grow keep alpha = 1.  Otherwise the
+          // stale maximum stays (P <= 2^8).
+          if (!(ok = mbar_wait(&b.pv_done, (g - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          pv_waited = true;
+          const float m_new = fmaxf(m, mx);
+          const float alpha = ex2_approx(m - m_new);
+          l *= alpha;
+          m = m_new;
+#pragma unroll
+          for (int ch = 0; ch < D / 16; ++ch) {   // 16 columns at a time: v[] is still live
+            uint32_t w[16];
+            SLA_TMEM_LD16(tO + ch * 16, w);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            SLA_TMEM_ST16(tO + ch * 16, v);
+            for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * alpha);
+            SLA_TMEM_ST16(tO + ch * 16, w);
           }
         }
-        m = m_new;
+        // P = 2^(acc * c - m), exact int -> float through the 1.5*2^23 magic
+        // number (|acc| <= D * 127^2 < 2^22), rounded to bf16 into TMEM
+        // (the packed pair e/2 goes to v[e/2], a slot already consumed)
+        const float nm = -m;
 #pragma unroll
-        for (int ch = 0; ch < BLK / 16; ++ch) {
-          uint32_t v[16];
-          SLA_TMEM_LD16(tS + ch * 16, v);
-          tmem_ld_wait();
-          uint32_t pk[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float x0 = (float)(int)v[e] * c, x1 = (float)(int)v[e + 1] * c;
-            float p0 = (ch * 16 + e < nvalid) ? ex2_approx(x0 - m) : 0.f;
-            float p1 = (ch * 16 + e + 1 < nvalid) ? ex2_approx(x1 - m) : 0.f;
-            l += p0 + p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < 64; e += 2) {
+          const float f0 = __int_as_float((int)v[e] + 0x4B400000) - 12582912.f;
+          const float f1 = __int_as_float((int)v[e + 1] + 0x4B400000) - 12582912.f;
+          float p0 = ex2_approx(fmaf(f0, c, nm));
+          float p1 = ex2_approx(fmaf(f1, c, nm));
+          if (partial) {
+            p0 = (e < nvalid) ? p0 : 0.f;
+            p1 = (e + 1 < nvalid) ? p1 : 0.f;
           }
-          SLA_TMEM_ST8(tS + ch * 8, pk);
+          l += p0 + p1;
+          v[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        SLA_TMEM_ST16(sbuf, v);
+        SLA_TMEM_ST16(sbuf + 16, (v + 16));
+        // every PV completion is consumed in order, before the next PV can start
+        if (x > 0 && !pv_waited) {
+          if (!(ok = mbar_wait(&b.pv_done, (g - 1) & 1, abort_flag))) break;
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&b.p_full);
+        mbar_arrive(&b.p_full[g & 1]);
       }
       if (!ok) break;
+      hg += H;
       if (!(ok = mbar_wait(&b.o_full, item_it & 1, abort_flag))) break;
+      if (!(ok = mbar_wait(&b.pv_done, (hg - 1) & 1, abort_flag))) break;   // the item's last PV
       tc_fence_after();
       const float inv_l = 1.f / l;
       const long long n = (long long)i * BLK + r;
       const bool valid = r < BLK && n < p.N;
       const long long obase = ((long long)bh * p.N + n) * D;
 #pragma unroll
-      for (int ch = 0; ch < D / 16; ++ch) {
-        uint32_t v[16];
-        SLA_TMEM_LD16(tO + ch * 16, v);
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t w[32];
+        SLA_TMEM_LD32(tO + ch * 32, w);
         tmem_ld_wait();
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.o + obase + ch * 16);
+          float4* dst = reinterpret_cast<float4*>(p.o + obase + ch * 32);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_float4(__uint_as_float(v[4 * q]) * inv_l, __uint_as_float(v[4 * q + 1]) * inv_l,
-                                 __uint_as_float(v[4 * q + 2]) * inv_l, __uint_as_float(v[4 * q + 3]) * inv_l);
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(w[4 * q]) * inv_l, __uint_as_float(w[4 * q + 1]) * inv_l,
+                                 __uint_as_float(w[4 * q + 2]) * inv_l, __uint_as_float(w[4 * q + 3]) * inv_l);
         }
       }
       tc_fence_before();
