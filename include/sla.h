@@ -113,7 +113,7 @@ int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, in
  * mask needs live in one file-scope device buffer of
  * SLA_NOALLOC_SCRATCH_BYTES (16 MiB) in this library, which every GPU that
  * loads the library holds until the process exits.  A problem must fit in
- * it: 18 * B*H*nblk*d + 4 * B*H*d bytes, each part rounded up to 256 bytes
+ * it: 26 * B*H*nblk*d + 4 * B*H*d bytes, each part rounded up to 256 bytes
  * (for example B*H = 12, nblk = 256, d = 128 fits; B*H = 40, nblk = 591
  * does not); larger ones return SLA_ERR_SCRATCH_LIMIT before any work is
  * enqueued.
@@ -173,6 +173,14 @@ typedef enum {
  * Either array may be NULL.  Returns SLA_OK or SLA_ERR_CUDA. */
 int sla_profile_enable(int on);
 int sla_profile_read(double* ms, long long* launches, int n);
+
+/* Failure-path self test (no counterpart on the pages): launches one tiny
+ * kernel whose bounded wait on a barrier that nothing completes gives up after
+ * its limit (about one second) exactly as a stalled pipeline would: it records
+ * SLA_ERR_TIMEOUT in the device error word and returns, leaving the context
+ * usable.  Returns SLA_OK once the kernel is enqueued; a following
+ * sla_get_error(stream) then reports SLA_ERR_TIMEOUT. */
+int sla_selftest_wait_timeout(void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* sla_status_string(int status);

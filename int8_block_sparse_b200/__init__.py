@@ -21,7 +21,7 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
 
 EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
            "sla_get_error", "sla_status_string", "sla_profile_enable", "sla_profile_read",
-           "sla_mask_noalloc")
+           "sla_mask_noalloc", "sla_selftest_wait_timeout")
 
 KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm", "linout")
 
@@ -47,6 +47,7 @@ def lib() -> ctypes.CDLL:
         L.sla_quant.argtypes = [vp] * 7 + [i] * 5 + [vp]
         L.sla_mask.argtypes = [vp] * 4 + [i] * 5 + [f, vp]
         L.sla_mask_noalloc.argtypes = [vp] * 4 + [i] * 5 + [f, vp]
+        L.sla_selftest_wait_timeout.argtypes = [vp]
         L.sla_attn.argtypes = [vp] * 5 + [i] * 5 + [f, vp]
         L.sla_attn_ex.argtypes = [vp] * 6 + [i] * 5 + [f, vp]
         L.sla_attn_host.argtypes = [vp] * 5 + [i] * 5 + [f]

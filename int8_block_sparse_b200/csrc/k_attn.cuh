@@ -58,8 +58,8 @@ struct AttnCfg {
 };
 
 struct TileBars {
-  uint64_t q_full, q_empty, pv_done, o_full, o_free;
-  uint64_t s_full[2], p_full[2];
+  uint64_t q_full, q_empty, o_full, o_free;
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t kv_full[2], kv_empty[2];
 };
 
@@ -89,12 +89,12 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
       TileBars& b = bars[u];
       mbar_init(&b.q_full, 1);
       mbar_init(&b.q_empty, 1);
-      mbar_init(&b.pv_done, 1);
       mbar_init(&b.o_full, 1);
       mbar_init(&b.o_free, 128);
       for (int s = 0; s < 2; ++s) {
         mbar_init(&b.s_full[s], 1);
         mbar_init(&b.p_full[s], 128);
+        mbar_init(&b.pv_done[s], 1);
         mbar_init(&b.kv_full[s], 1);
         mbar_init(&b.kv_empty[s], 1);
       }
@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
 #pragma unroll
             for (int kk = 0; kk < C::HB / 16; ++kk)
               mma_bf16_ts(tO, aP + kk * 8, dv + uint64_t(kk * (2048 >> 4)), id_pv, (x > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&b.pv_done);
+            tc_commit(&b.pv_done[g & 1]);
             if (x % NH == NH - 1) tc_commit(&b.kv_empty[s]);
             if (x == H - 1) tc_commit(&b.o_full);
             if (x + 2 < H) ok = issue_qk(x + 2);
@@ -270,7 +270,6 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             if (e < nvalid) amax = max(amax, (int)v[e]);
         }
         const float mx = (nvalid > 0) ? (float)amax * c : -INFINITY;
-        bool pv_waited = false;
         if (x == 0) {
           m = mx;
         } else if (__any_sync(0xffffffffu, mx > m + 8.f)) {
@@ -278,9 +277,11 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
           // finished, the warp rescales O (tcgen05.ld/st are warp-collective);
           // rows whose maximum did not grow keep alpha = 1.  Otherwise the
           // stale maximum stays (P <= 2^8).
-          if (!(ok = mbar_wait(&b.pv_done, (g - 1) & 1, abort_flag))) break;
+          // PV(g-2) and older are complete (QK(g) was issued after PV(g-2) and
+          // its S is ready); PV(g-1) uses buffer (g-1)&1, whose uses before it
+          // are complete, so this parity names PV(g-1) without ambiguity.
+          if (!(ok = mbar_wait(&b.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag))) break;
           tc_fence_after();
-          pv_waited = true;
           const float m_new = fmaxf(m, mx);
           const float alpha = ex2_approx(m - m_new);
           l *= alpha;
@@ -295,29 +296,36 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             SLA_TMEM_ST16(tO + ch * 16, w);
           }
         }
-        // P = 2^(acc * c - m), exact int -> float through the 1.5*2^23 magic
-        // number (|acc| <= D * 127^2 < 2^22), rounded to bf16 into TMEM
-        // (the packed pair e/2 goes to v[e/2], a slot already consumed)
-        const float nm = -m;
+        // P = 2^(acc * c - m) rounded to bf16 into TMEM.  The float with bits
+        // acc + 0x4B400000 is exactly 1.5*2^23 + acc (|acc| <= D*127^2 < 2^22),
+        // so acc*c - m = fma(that, c, -(1.5*2^23*c + m)); the one rounding of
+        // that constant shifts all exponents of this row and half by the same
+        // amount (< 2^-24 relative to 1.5*2^23*c), i.e. scales P and l alike.
+        // The packed pair e/2 goes to v[e/2], a slot already consumed.
+        const float kk = -fmaf(12582912.f, c, m);
+        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const float f0 = __int_as_float((int)v[e] + 0x4B400000) - 12582912.f;
-          const float f1 = __int_as_float((int)v[e + 1] + 0x4B400000) - 12582912.f;
-          float p0 = ex2_approx(fmaf(f0, c, nm));
-          float p1 = ex2_approx(fmaf(f1, c, nm));
+        for (int e = 0; e < 64; e += 4) {
+          float p0 = ex2_approx(fmaf(__int_as_float((int)v[e] + 0x4B400000), c, kk));
+          float p1 = ex2_approx(fmaf(__int_as_float((int)v[e + 1] + 0x4B400000), c, kk));
+          float p2 = ex2_approx(fmaf(__int_as_float((int)v[e + 2] + 0x4B400000), c, kk));
+          float p3 = ex2_approx(fmaf(__int_as_float((int)v[e + 3] + 0x4B400000), c, kk));
           if (partial) {
             p0 = (e < nvalid) ? p0 : 0.f;
             p1 = (e + 1 < nvalid) ? p1 : 0.f;
+            p2 = (e + 2 < nvalid) ? p2 : 0.f;
+            p3 = (e + 3 < nvalid) ? p3 : 0.f;
           }
-          l += p0 + p1;
+          l0 += p0;
+          l1 += p1;
+          l2 += p2;
+          l3 += p3;
           v[e >> 1] = pack_bf16x2(p0, p1);
+          v[(e >> 1) + 1] = pack_bf16x2(p2, p3);
         }
+        l += (l0 + l1) + (l2 + l3);
         SLA_TMEM_ST16(sbuf, v);
         SLA_TMEM_ST16(sbuf + 16, (v + 16));
-        // every PV completion is consumed in order, before the next PV can start
-        if (x > 0 && !pv_waited) {
-          if (!(ok = mbar_wait(&b.pv_done, (g - 1) & 1, abort_flag))) break;
-        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&b.p_full[g & 1]);
@@ -325,7 +333,6 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
       if (!ok) break;
       hg += H;
       if (!(ok = mbar_wait(&b.o_full, item_it & 1, abort_flag))) break;
-      if (!(ok = mbar_wait(&b.pv_done, (hg - 1) & 1, abort_flag))) break;   // the item's last PV
       tc_fence_after();
       const float inv_l = 1.f / l;
       const long long n = (long long)i * BLK + r;

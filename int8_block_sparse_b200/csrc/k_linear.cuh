@@ -10,11 +10,10 @@
 //     [G | g] (NB x (D*D + D)) = notcrit (NB x NB) . [h | z] (NB x (D*D + D))
 // (k_lingemm, tcgen05 bf16 with float32 accumulation; summing the
 // non-selected blocks directly avoids the cancellation of total minus
-// selected).  Then, per query row n of block i (k_linout):
-//     O_lin,n = phi(q_n) G_i / (phi(q_n) . g_i),   out_n = O_sparse,n + O_lin,n W_proj
-// with both products on the tensor cores.  O_lin is split into bf16 high and
-// low parts (O_lin = hi + lo up to float32 rounding) so that O_lin W_proj keeps
-// float32-level accuracy; W_proj itself is exact in bf16.
+// selected).  The states arrive with W_proj folded in (h'_j = h_j W_proj, see
+// k_stats.cuh), so per query row n of block i (k_linout)
+//     out_n = O_sparse,n + phi(q_n) G'_i / (phi(q_n) . g_i),   G'_i = G_i W_proj,
+// one tensor-core product per query block.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -145,29 +144,23 @@ struct LinOutParams {
 
 template <int D>
 struct LinOutCfg {
-  static constexpr int A_BYTES = 128 * D * 2;   // phi(Q) tile, later the high part of O_lin
-  static constexpr int B_BYTES = 128 * D * 2;   // G_i (D x D), later the low part of O_lin (128 x D)
-  static constexpr int G_BYTES = D * D * 2;     // bytes of G_i the TMA delivers
-  static constexpr int W_BYTES = D * D * 2;     // W_proj
-  // at least 60 KB so that no more than 3 CTAs share an SM: each holds 2*D
-  // TMEM columns and an SM has 512
-  static constexpr int SMEM_USED = A_BYTES + B_BYTES + W_BYTES + 1024 + 256;
-  static constexpr int SMEM = SMEM_USED > 61440 ? SMEM_USED : 61440;
+  static constexpr int A_BYTES = 128 * D * 2;   // phi(Q) tile (K-major, 64-column atoms of 16 KB)
+  static constexpr int G_BYTES = D * D * 2;     // G'_i (MN-major)
+  static constexpr int SMEM = A_BYTES + G_BYTES + 1024 + 128 + D * 4;
 };
 
 // One CTA (128 threads, thread = query row) per query block.
 template <int D>
-__global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensorMap tm_g,
-                                                const __grid_constant__ CUtensorMap tm_w, const LinOutParams p) {
+__global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensorMap tm_g, const LinOutParams p) {
   using C = LinOutCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sa = base;
   unsigned char* sg = sa + C::A_BYTES;
-  unsigned char* sw = sg + C::B_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sw + C::W_BYTES);   // 0: loads, 1: mma1, 2: mma2
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  float* sz = reinterpret_cast<float*>(sg + C::G_BYTES);           // z_rest of this query block
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sz + D);            // 0: G load, 1: MMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int i = blockIdx.x;
@@ -176,26 +169,24 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
-    mbar_init(&bars[2], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 2 * D);
+    tmem_alloc(tmem_slot, D);
     tmem_relinquish();
   }
+  if (tid < D) sz[tid] = p.zrest[(bh * p.NB + i) * D + tid];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (tid == 0) {
-    mbar_expect_tx(&bars[0], C::G_BYTES + C::W_BYTES);
+    mbar_expect_tx(&bars[0], C::G_BYTES);
 #pragma unroll
-    for (int hh = 0; hh < D / 64; ++hh) {
+    for (int hh = 0; hh < D / 64; ++hh)
       tma_load_2d(sg + hh * D * 128, &tm_g, &bars[0], hh * 64, int((bh * p.NB + i) * D));
-      tma_load_2d(sw + hh * D * 128, &tm_w, &bars[0], hh * 64, 0);
-    }
   }
 
   const int r = tid;
@@ -205,19 +196,20 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   float den = 0.f;
   {
     const __nv_bfloat16* qrow = p.q + (bh * p.N + n) * D;
-    const float* zr = p.zrest + (bh * p.NB + i) * D;
+    uint4 raw[D / 8];
+#pragma unroll
+    for (int c8 = 0; c8 < D / 8; ++c8)
+      raw[c8] = valid ? *reinterpret_cast<const uint4*>(qrow + c8 * 8) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int c8 = 0; c8 < D / 8; ++c8) {
-      uint4 raw = make_uint4(0, 0, 0, 0);
-      if (valid) raw = *reinterpret_cast<const uint4*>(qrow + c8 * 8);
-      const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
+      const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw[c8]);
       uint32_t pk[4];
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
-        float f0 = valid ? phi_elu1(__uint_as_float(uint32_t(hv[e]) << 16)) : 0.f;
-        float f1 = valid ? phi_elu1(__uint_as_float(uint32_t(hv[e + 1]) << 16)) : 0.f;
-        den = fmaf(f0, zr[c8 * 8 + e], den);
-        den = fmaf(f1, zr[c8 * 8 + e + 1], den);
+        const float f0 = valid ? phi_elu1(__uint_as_float(uint32_t(hv[e]) << 16)) : 0.f;
+        const float f1 = valid ? phi_elu1(__uint_as_float(uint32_t(hv[e + 1]) << 16)) : 0.f;
+        den = fmaf(f0, sz[c8 * 8 + e], den);
+        den = fmaf(f1, sz[c8 * 8 + e + 1], den);
         pk[e >> 1] = pack_bf16x2(f0, f1);
       }
       const int atom = c8 >> 3, chunk = c8 & 7;
@@ -226,11 +218,11 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   }
   fence_async_shared();
   __syncthreads();
-  const uint32_t idesc = idesc_bf16(D, false, true);
   if (tid == 0) {
-    bool ok = mbar_wait(&bars[0], 0, abort_flag);
-    if (ok) {
+    const bool okl = mbar_wait(&bars[0], 0, abort_flag);
+    if (okl) {
       tc_fence_after();
+      const uint32_t idesc = idesc_bf16(D, false, true);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t da = smem_desc(smem_u32(sa + (kk >> 2) * 16384) + (kk & 3) * 32, 16, 1024, 2);
@@ -241,77 +233,33 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
     tc_commit(&bars[1]);
   }
   __syncwarp();
-  bool ok = mbar_wait(&bars[1], 0, abort_flag);
+  const bool ok = mbar_wait(&bars[1], 0, abort_flag);
   tc_fence_after();
   const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
   const float inv_den = (valid && den > 0.f) ? 1.f / den : 0.f;
-  // G_i is consumed (MMA 1 completed), so its buffer takes the low part
-  unsigned char* slo = sg;
-#pragma unroll
-  for (int ch = 0; ch < D / 16; ++ch) {
-    uint32_t v[16];
-    SLA_TMEM_LD16(trow + ch * 16, v);
-    tmem_ld_wait();
-    uint32_t hi[8], lo[8];
-#pragma unroll
-    for (int e = 0; e < 16; e += 2) {
-      const float o0 = __uint_as_float(v[e]) * inv_den, o1 = __uint_as_float(v[e + 1]) * inv_den;
-      hi[e >> 1] = pack_bf16x2(o0, o1);
-      const float h0 = __uint_as_float(hi[e >> 1] << 16), h1 = __uint_as_float(hi[e >> 1] & 0xFFFF0000u);
-      lo[e >> 1] = pack_bf16x2(o0 - h0, o1 - h1);
-    }
-    const int c8 = ch * 2;
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      const int cc = c8 + h2, atom = cc >> 3, chunk = cc & 7;
-      const uint32_t off = atom * 16384 + sw128_offset(r, chunk);
-      *reinterpret_cast<uint4*>(sa + off) = make_uint4(hi[4 * h2], hi[4 * h2 + 1], hi[4 * h2 + 2], hi[4 * h2 + 3]);
-      *reinterpret_cast<uint4*>(slo + off) = make_uint4(lo[4 * h2], lo[4 * h2 + 1], lo[4 * h2 + 2], lo[4 * h2 + 3]);
-    }
-  }
-  fence_async_shared();
-  tc_fence_before();
-  __syncthreads();
-  if (tid == 0) {
-    if (ok) {
-      tc_fence_after();
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        unsigned char* src = part == 0 ? sa : slo;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t da = smem_desc(smem_u32(src + (kk >> 2) * 16384) + (kk & 3) * 32, 16, 1024, 2);
-          const uint64_t db = smem_desc(smem_u32(sw) + kk * 2048, D * 128, 1024, 2);
-          mma_bf16_ss(tmem + D, da, db, idesc, (part > 0 || kk > 0) ? 1u : 0u);
-        }
-      }
-    }
-    tc_commit(&bars[2]);
-  }
-  __syncwarp();
-  ok = mbar_wait(&bars[2], 0, abort_flag) && ok;
-  tc_fence_after();
   const float* os = p.osparse + (bh * p.N + n) * D;
   float* dst = p.out + (bh * p.N + n) * D;
 #pragma unroll
   for (int ch = 0; ch < D / 16; ++ch) {
     uint32_t v[16];
-    SLA_TMEM_LD16(trow + D + ch * 16, v);
+    SLA_TMEM_LD16(trow + ch * 16, v);
     tmem_ld_wait();
     if (valid && ok) {
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const float4 a = *reinterpret_cast<const float4*>(os + ch * 16 + 4 * q4);
         *reinterpret_cast<float4*>(dst + ch * 16 + 4 * q4) =
-            make_float4(a.x + __uint_as_float(v[4 * q4]), a.y + __uint_as_float(v[4 * q4 + 1]),
-                        a.z + __uint_as_float(v[4 * q4 + 2]), a.w + __uint_as_float(v[4 * q4 + 3]));
+            make_float4(fmaf(__uint_as_float(v[4 * q4]), inv_den, a.x),
+                        fmaf(__uint_as_float(v[4 * q4 + 1]), inv_den, a.y),
+                        fmaf(__uint_as_float(v[4 * q4 + 2]), inv_den, a.z),
+                        fmaf(__uint_as_float(v[4 * q4 + 3]), inv_den, a.w));
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 2 * D);
+  if (warp == 0) tmem_dealloc(tmem, D);
 }
 
 }  // namespace sla

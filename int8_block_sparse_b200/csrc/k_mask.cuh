@@ -8,10 +8,12 @@
 // the kc largest scores are the kc largest probabilities; equal scores go to
 // the lower block index.  The kept indices are written in ascending order.
 //
-// One CTA handles ROWS query blocks of one head: it stages the pooled query
-// blocks and, 32 at a time, the pooled key blocks in shared memory, writes
-// the ROWS x NB scores to shared memory, then each warp selects the top kc of
-// a row by a bitwise search for the kc-th largest order-preserving key.
+// One CTA handles R query blocks of one head (R = 8: a warp per row): it stages
+// the pooled query blocks and, 32 at a time, the pooled key blocks in shared
+// memory (each lane takes one key block and four independent partial dot
+// products), writes the R x NB scores to shared memory, then each warp selects
+// the top kc of its row by a bitwise search for the kc-th largest
+// order-preserving key.
 #pragma once
 #include "sm100.cuh"
 
@@ -23,8 +25,8 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qsum, const double* __restrict__ ksum,
-                                             int N, int NB, int BLK, int kc, int rows_per_cta,
+__global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, const double* __restrict__ kbar,
+                                             int NB, int kc, int rows_per_cta,
                                              int32_t* __restrict__ idx, uint8_t* __restrict__ bitmap,
                                              __nv_bfloat16* __restrict__ notcrit, int ncpitch) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -37,39 +39,30 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qsum, c
   const int i0 = blockIdx.x * R;
   const int nrows = min(R, NB - i0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const double rsd = 1.0 / sqrt((double)D);
-  (void)rsd;
   const double sqd = sqrt((double)D);
 
   for (int e = tid; e < R * D; e += 256) {
-    const int r = e / D, c = e % D;
-    double v = 0.0;
-    if (r < nrows) {
-      const int i = i0 + r;
-      const int cnt = min(BLK, N - i * BLK);
-      v = qsum[(bh * NB + i) * (long long)D + c] / (double)cnt;
-    }
-    qb[e] = v;
+    const int r = e / D;
+    qb[e] = (r < nrows) ? qbar[(bh * NB + i0) * (long long)D + e] : 0.0;
   }
   for (int j0 = 0; j0 < NB; j0 += 32) {
     __syncthreads();
     for (int e = tid; e < 32 * D; e += 256) {
       const int r = e / D, c = e % D;
-      const int j = j0 + r;
-      double v = 0.0;
-      if (j < NB) {
-        const int cnt = min(BLK, N - j * BLK);
-        v = ksum[(bh * NB + j) * (long long)D + c] / (double)cnt;
-      }
-      kbs[r * (D + 1) + c] = v;
+      kbs[r * (D + 1) + c] = (j0 + r < NB) ? kbar[(bh * NB + j0 + r) * (long long)D + c] : 0.0;
     }
     __syncthreads();
     const int j = j0 + lane;
     for (int r = warp; r < nrows; r += 8) {
-      double acc = 0.0;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) acc = fma(qb[r * D + c], kbs[lane * (D + 1) + c], acc);
-      if (j < NB) sc[r * NB + j] = acc / sqd;
+      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+#pragma unroll 4
+      for (int c = 0; c < D; c += 4) {
+        a0 = fma(qb[r * D + c], kbs[lane * (D + 1) + c], a0);
+        a1 = fma(qb[r * D + c + 1], kbs[lane * (D + 1) + c + 1], a1);
+        a2 = fma(qb[r * D + c + 2], kbs[lane * (D + 1) + c + 2], a2);
+        a3 = fma(qb[r * D + c + 3], kbs[lane * (D + 1) + c + 3], a3);
+      }
+      if (j < NB) sc[r * NB + j] = ((a0 + a1) + (a2 + a3)) / sqd;
     }
   }
   __syncthreads();

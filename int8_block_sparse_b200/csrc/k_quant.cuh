@@ -7,8 +7,8 @@
 // D channels).  Per block: m = max|x|, s = m / 127 (IEEE float32 division),
 // code = clamp(round_half_even(x / s), -127, 127) with an IEEE division per
 // element; a block with m = 0 has s = 0 and zero codes.  Rows past N (up to
-// NB*BLK) get zero codes.  For Q the kernel also writes the float64 sums of
-// each block (the pooled block means of the mask).
+// NB*BLK) get zero codes.  For Q the kernel also writes the float64 mean of
+// each block's valid rows (the pooled query block of the mask).
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(256) k_quant(const __nv_bfloat16* __restrict__
                                               const __nv_bfloat16* __restrict__ K, const float* __restrict__ mu,
                                               int8_t* __restrict__ qi8, int8_t* __restrict__ ki8,
                                               float* __restrict__ sq, float* __restrict__ sk,
-                                              double* __restrict__ qsum, int N, int NB) {
+                                              double* __restrict__ qbar, int N, int NB) {
   constexpr int VEC = 8;
   constexpr int GROUPS = D / VEC;
   constexpr int NV = BLK * GROUPS / 256;   // 16-byte vectors per thread
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(256) k_quant(const __nv_bfloat16* __restrict__
       mloc = fmaxf(mloc, fabsf(f));
     }
   }
-  if (!isk && qsum != nullptr) {
+  if (!isk && qbar != nullptr) {
     double part[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) part[e] = 0.0;
@@ -75,10 +75,10 @@ __global__ void __launch_bounds__(256) k_quant(const __nv_bfloat16* __restrict__
   const float s = __fdiv_rn(m, 127.0f);
   float* sdst = isk ? sk : sq;
   if (tid == 0 && sdst != nullptr) sdst[bh * NB + j] = s;
-  if (!isk && qsum != nullptr && tid < D) {
+  if (!isk && qbar != nullptr && tid < D) {
     double acc = 0.0;
     for (int q = 0; q < RSTEP; ++q) acc += red[q * D + tid];
-    qsum[(bh * NB + j) * (long long)D + tid] = acc;
+    qbar[(bh * NB + j) * (long long)D + tid] = acc / (double)rows;
   }
   int8_t* dbase = isk ? ki8 : qi8;
   if (dbase == nullptr) return;

@@ -2,17 +2,26 @@
 //
 // For key block j of head (b, h) -- rows [j*BLK, min(N, (j+1)*BLK)) -- it
 // writes
-//   ksum[bh][j][c]   float64 sum of the raw K values of channel c (used for the
-//                    pooled block means of the mask and for the channel mean);
+//   ksum[bh][j][c]   float64 sum of the raw K values of channel c (for the
+//                    channel mean);
+//   kbar[bh][j][c]   float64 mean of those values (the pooled block of the mask);
 //   kexp[bh][j][c]   largest and smallest bf16 exponent field among the nonzero
 //                    K values of the channel (checks that the float64 sums are
 //                    exact);
-//   hstate[bh][j][:] the linear-attention state of the block, bf16:
-//                    h_j = sum_n phi(k_n) v_n^T as a D x D row-major matrix
-//                    followed by z_j = sum_n phi(k_n) (D values), phi = elu + 1.
+//   hstate[bh][j][:] (optional) the block's linear-attention state, bf16:
+//                    h'_j = sum_n phi(k_n) (v_n W_proj)^T as a D x D row-major
+//                    matrix followed by z_j = sum_n phi(k_n) (D values),
+//                    phi = elu + 1.
 // ("Turbo Diffusion：秒级生成与高清保真的视频扩散技术突破", section 三(二) SLA
-// item 2: the non-selected blocks go through an O(N) linear branch; section
-// 三(一) item 1: K smoothing needs the channel mean.)
+// item 2: the non-selected blocks go through an O(N) linear branch with a
+// linear projection; section 三(一) item 1: K smoothing needs the channel mean.)
+//
+// W_proj is folded into the states: O_lin W = phi(q) (sum_j h_j) W / den =
+// phi(q) (sum_j phi(K_j)^T (V_j W)) / den, so the query side needs one product
+// instead of two.  Both products run on the tensor cores (bf16 operands,
+// float32 accumulation): V'_j = V_j W with the TMA-loaded V tile as a K-major A
+// operand, then h'_j = phi(K_j)^T V'_j with phi(K_j)^T built in shared memory as
+// an MN-major A operand and V'_j written back over V_j as an MN-major B operand.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -26,127 +35,254 @@ __device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : 
 __device__ __forceinline__ uint32_t bf16_exp_field(uint16_t b) { return (b >> 7) & 0xFFu; }
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(256) k_kstats(const __nv_bfloat16* __restrict__ K,
-                                               const __nv_bfloat16* __restrict__ V, double* __restrict__ ksum,
-                                               uint8_t* __restrict__ kexp, __nv_bfloat16* __restrict__ hstate,
-                                               int N, int NB, long long hpitch) {
-  constexpr int VEC = 8;             // bf16 per 16-byte load
-  constexpr int GROUPS = D / VEC;    // vector columns per row
-  constexpr int RSTEP = 256 / GROUPS;
-  constexpr int TILE = D / 16;       // each thread owns a TILE x TILE patch of h
+struct StatsCfg {
+  static constexpr int V_BYTES = BLK * D * 2;        // V tile, then V' (MN-major, 64-channel atoms)
+  static constexpr int W_BYTES = D * D * 2;          // W_proj (MN-major B)
+  static constexpr int P_BYTES = 128 * BLK * 2;      // phi(K)^T (MN-major A, 128 rows of a; D=64 pads)
+  static constexpr int GROUPS = D / 8;               // 16-byte vectors per row
+  static constexpr int RG = 128 / GROUPS;            // row groups (threads per channel group)
+  static constexpr int RED_BYTES = RG * D * (8 + 4 + 4);
+  static constexpr int SMEM = V_BYTES + W_BYTES + P_BYTES + RED_BYTES + 1024 + 128;
+};
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensorMap tm_v,
+                                               const __grid_constant__ CUtensorMap tm_w,
+                                               const __nv_bfloat16* __restrict__ K, double* __restrict__ ksum,
+                                               double* __restrict__ kbar, uint8_t* __restrict__ kexp,
+                                               __nv_bfloat16* __restrict__ hstate, int N, int NB,
+                                               long long hpitch) {
+  using C = StatsCfg<D, BLK>;
+  constexpr int GROUPS = C::GROUPS, RG = C::RG;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  float* phk = reinterpret_cast<float*>(smem_raw);                 // [BLK][D]
-  float* vv = phk + BLK * D;                                       // [BLK][D]
-  double* red = reinterpret_cast<double*>(vv + BLK * D);           // [RSTEP][D]
-  uint32_t* ered = reinterpret_cast<uint32_t*>(red + RSTEP * D);   // [RSTEP][D] packed max|min
+  unsigned char* base =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sV = base;
+  unsigned char* sW = sV + C::V_BYTES;
+  unsigned char* sP = sW + C::W_BYTES;
+  double* red = reinterpret_cast<double*>(sP + C::P_BYTES);        // [RG][D]
+  float* redz = reinterpret_cast<float*>(red + RG * D);            // [RG][D]
+  uint32_t* rede = reinterpret_cast<uint32_t*>(redz + RG * D);     // [RG][D] max<<8 | min
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rede + RG * D);     // 0: TMA, 1: MMA0, 2: MMA1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int j = blockIdx.x;
   const long long bh = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int row0 = j * BLK;
   const int rows = min(BLK, N - row0);
-  const __nv_bfloat16* kb = K + (bh * N + row0) * (long long)D;
-  const __nv_bfloat16* vb = V + (bh * N + row0) * (long long)D;
+  const bool states = hstate != nullptr;
 
-  const int g = tid % GROUPS;
-  double part[VEC];
-  uint32_t emax[VEC], emin[VEC];
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    mbar_init(&bars[2], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (states && warp == 0) {
+    tmem_alloc(tmem_slot, 2 * D);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = states ? *tmem_slot : 0u;
+
+  if (states && tid == 0) {
+    mbar_expect_tx(&bars[0], C::V_BYTES + C::W_BYTES);
 #pragma unroll
-  for (int e = 0; e < VEC; ++e) { part[e] = 0.0; emax[e] = 0u; emin[e] = 255u; }
-  for (int r = tid / GROUPS; r < BLK; r += RSTEP) {
-    uint4 kr = make_uint4(0, 0, 0, 0), vr = make_uint4(0, 0, 0, 0);
-    if (r < rows) {
-      kr = *reinterpret_cast<const uint4*>(kb + (long long)r * D + g * VEC);
-      if (hstate != nullptr) vr = *reinterpret_cast<const uint4*>(vb + (long long)r * D + g * VEC);
+    for (int hh = 0; hh < D / 64; ++hh) {
+      tma_load_3d(sV + hh * BLK * 128, &tm_v, &bars[0], hh * 64, row0, (int)bh);
+      tma_load_2d(sW + hh * D * 128, &tm_w, &bars[0], hh * 64, 0);
     }
+  }
+
+  // K rows: float64 sums, exponent range, phi (float32 sums for z, bf16 for h')
+  const __nv_bfloat16* kb = K + (bh * N + row0) * (long long)D;
+  const int g = tid % GROUPS, rg = tid / GROUPS;
+  double part[8];
+  float zp[8];
+  uint32_t emax[8], emin[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { part[e] = 0.0; zp[e] = 0.f; emax[e] = 0u; emin[e] = 255u; }
+  for (int r = rg; r < BLK; r += RG) {
+    uint4 kr = make_uint4(0, 0, 0, 0);
+    if (r < rows) kr = *reinterpret_cast<const uint4*>(kb + (long long)r * D + g * 8);
     const uint16_t* kh = reinterpret_cast<const uint16_t*>(&kr);
-    const uint16_t* vh = reinterpret_cast<const uint16_t*>(&vr);
+    uint32_t pk[4];
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const float kf = __uint_as_float(uint32_t(kh[e]) << 16);
-      const float vf = __uint_as_float(uint32_t(vh[e]) << 16);
-      part[e] += (double)kf;
-      const uint32_t ef = bf16_exp_field(kh[e]);
-      if ((kh[e] & 0x7FFFu) != 0u) { emax[e] = max(emax[e], ef); emin[e] = min(emin[e], ef); }
-      phk[r * D + g * VEC + e] = (r < rows) ? phi_elu1(kf) : 0.f;
-      vv[r * D + g * VEC + e] = vf;
+    for (int e = 0; e < 8; e += 2) {
+      const float k0 = __uint_as_float(uint32_t(kh[e]) << 16), k1 = __uint_as_float(uint32_t(kh[e + 1]) << 16);
+      part[e] += (double)k0;
+      part[e + 1] += (double)k1;
+      if ((kh[e] & 0x7FFFu) != 0u) { emax[e] = max(emax[e], bf16_exp_field(kh[e])); emin[e] = min(emin[e], bf16_exp_field(kh[e])); }
+      if ((kh[e + 1] & 0x7FFFu) != 0u) {
+        emax[e + 1] = max(emax[e + 1], bf16_exp_field(kh[e + 1]));
+        emin[e + 1] = min(emin[e + 1], bf16_exp_field(kh[e + 1]));
+      }
+      const float p0 = (r < rows) ? phi_elu1(k0) : 0.f, p1 = (r < rows) ? phi_elu1(k1) : 0.f;
+      zp[e] += p0;
+      zp[e + 1] += p1;
+      pk[e >> 1] = pack_bf16x2(p0, p1);
+    }
+    if (states) {
+      // phi(K)^T, MN-major: channel a = g*8.. is the M index, row r the K index
+      const int atom = (g * 8) / 64, chunk = ((g * 8) % 64) / 8;
+      *reinterpret_cast<uint4*>(sP + atom * BLK * 128 + sw128_offset(r, chunk)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
-  const int rg = tid / GROUPS;
-#pragma unroll
-  for (int e = 0; e < VEC; ++e) {
-    red[rg * D + g * VEC + e] = part[e];
-    ered[rg * D + g * VEC + e] = (emax[e] << 8) | emin[e];
+  if (states && D == 64) {
+    // rows a = 64..127 of the 128-row A operand are zero
+    for (int e = tid; e < BLK * 128 / 16; e += 128)
+      reinterpret_cast<uint4*>(sP + BLK * 128)[e] = make_uint4(0, 0, 0, 0);
   }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    red[rg * D + g * 8 + e] = part[e];
+    redz[rg * D + g * 8 + e] = zp[e];
+    rede[rg * D + g * 8 + e] = (emax[e] << 8) | emin[e];
+  }
+  fence_async_shared();
   __syncthreads();
   if (tid < D) {
     double s = 0.0;
+    float z = 0.f;
     uint32_t mx = 0u, mn = 255u;
-    for (int q = 0; q < RSTEP; ++q) {
+    for (int q = 0; q < RG; ++q) {
       s += red[q * D + tid];
-      const uint32_t w = ered[q * D + tid];
+      z += redz[q * D + tid];
+      const uint32_t w = rede[q * D + tid];
       mx = max(mx, w >> 8);
       mn = min(mn, w & 0xFFu);
     }
     const long long o = (bh * NB + j) * (long long)D + tid;
     ksum[o] = s;
+    kbar[o] = s / (double)rows;
     kexp[2 * o] = (uint8_t)mx;
     kexp[2 * o + 1] = (uint8_t)mn;
+    if (states) hstate[(bh * (long long)NB + j) * hpitch + D * D + tid] = __float2bfloat16_rn(z);
   }
+  if (!states) return;
 
-  if (hstate == nullptr) return;
-  // h = phi(K)^T V on the CUDA cores (float32 accumulation), then bf16.
-  const int ta = (tid / 16) * TILE, tc = (tid % 16) * TILE;
-  float acc[TILE][TILE];
+  // V' = V W_proj: A = V tile (K-major over channels), B = W_proj (MN-major)
+  if (tid == 0) {
+    bool ok = mbar_wait(&bars[0], 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t id0 = idesc_bf16(D, false, true);
 #pragma unroll
-  for (int x = 0; x < TILE; ++x)
-#pragma unroll
-    for (int y = 0; y < TILE; ++y) acc[x][y] = 0.f;
-  for (int n = 0; n < rows; ++n) {
-    float pa[TILE], pv[TILE];
-#pragma unroll
-    for (int x = 0; x < TILE; ++x) pa[x] = phk[n * D + ta + x];
-#pragma unroll
-    for (int y = 0; y < TILE; ++y) pv[y] = vv[n * D + tc + y];
-#pragma unroll
-    for (int x = 0; x < TILE; ++x)
-#pragma unroll
-      for (int y = 0; y < TILE; ++y) acc[x][y] = fmaf(pa[x], pv[y], acc[x][y]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t da = smem_desc(smem_u32(sV + (kk >> 2) * BLK * 128) + (kk & 3) * 32, 16, 1024, 2);
+        const uint64_t db = smem_desc(smem_u32(sW) + kk * 2048, D * 128, 1024, 2);
+        mma_bf16_ss(tmem, da, db, id0, kk > 0 ? 1u : 0u);
+      }
+    }
+    tc_commit(&bars[1]);
   }
-  __nv_bfloat16* hs = hstate + (bh * (long long)NB + j) * hpitch;
+  __syncwarp();
+  bool ok = mbar_wait(&bars[1], 0, abort_flag);
+  tc_fence_after();
+  // thread = token row n of V': bf16 back over the V tile (same swizzled layout)
+  {
+    const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
 #pragma unroll
-  for (int x = 0; x < TILE; ++x)
+    for (int ch = 0; ch < D / 16; ++ch) {
+      uint32_t v[16];
+      SLA_TMEM_LD16(trow + ch * 16, v);
+      tmem_ld_wait();
+      if (tid < BLK) {
+        uint32_t pk[8];
 #pragma unroll
-    for (int y = 0; y < TILE; ++y) hs[(ta + x) * D + tc + y] = __float2bfloat16_rn(acc[x][y]);
-  if (tid < D) {
-    float z = 0.f;
-    for (int n = 0; n < rows; ++n) z += phk[n * D + tid];
-    hs[D * D + tid] = __float2bfloat16_rn(z);
+        for (int e = 0; e < 16; e += 2) pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        const int c0 = ch * 16, atom = c0 / 64;
+        unsigned char* dst = sV + atom * BLK * 128;
+        *reinterpret_cast<uint4*>(dst + sw128_offset(tid, (c0 % 64) / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(dst + sw128_offset(tid, (c0 % 64) / 8 + 1)) =
+            make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+    }
   }
+  fence_async_shared();
+  tc_fence_before();
+  __syncthreads();
+  // h' = phi(K)^T V': A MN-major (a contiguous), B MN-major (channels contiguous)
+  if (tid == 0) {
+    if (ok) {
+      tc_fence_after();
+      const uint32_t id1 = idesc_bf16(D, true, true);
+#pragma unroll
+      for (int kk = 0; kk < BLK / 16; ++kk) {
+        const uint64_t da = smem_desc(smem_u32(sP) + kk * 2048, BLK * 128, 1024, 2);
+        const uint64_t db = smem_desc(smem_u32(sV) + kk * 2048, BLK * 128, 1024, 2);
+        mma_bf16_ss(tmem + D, da, db, id1, kk > 0 ? 1u : 0u);
+      }
+    }
+    tc_commit(&bars[2]);
+  }
+  __syncwarp();
+  ok = mbar_wait(&bars[2], 0, abort_flag) && ok;
+  tc_fence_after();
+  {
+    const uint32_t trow = tmem + D + (uint32_t(warp * 32) << 16);
+    __nv_bfloat16* hs = hstate + (bh * (long long)NB + j) * hpitch + (long long)tid * D;
+#pragma unroll
+    for (int ch = 0; ch < D / 16; ++ch) {
+      uint32_t v[16];
+      SLA_TMEM_LD16(trow + ch * 16, v);
+      tmem_ld_wait();
+      if (ok && tid < D) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        uint4* d4 = reinterpret_cast<uint4*>(hs + ch * 16);
+        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 2 * D);
 }
 
-template <int D, int BLK>
-constexpr size_t kstats_smem() {
-  return size_t(2) * BLK * D * sizeof(float) + size_t(256 / (D / 8)) * D * (sizeof(double) + sizeof(uint32_t));
-}
-
-// mu[bh][c] = float32 nearest to (sum_j ksum[bh][j][c]) / N.  The block sums
-// are exact when every K value of the channel is a multiple of the smallest
-// one's unit in the last place and the total stays below 2^53 of those units;
-// kexp lets the kernel check that and raise DEV_ERR_INEXACT otherwise.
-__global__ void k_channel_mean(const double* __restrict__ ksum, const uint8_t* __restrict__ kexp,
-                               float* __restrict__ mu, int NB, int D, int N, long long total) {
-  const long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (t >= total) return;
-  const long long bh = t / D;
-  const int c = int(t % D);
+// mu[bh][c] = float32 nearest to (sum_j ksum[bh][j][c]) / N.  One CTA per
+// (batch, head): each thread sums every G-th block of one channel, then the G
+// partial sums are added in a fixed order.  The block sums are exact when every
+// K value of the channel is a multiple of the smallest one's unit in the last
+// place and the total stays below 2^53 of those units, so the order does not
+// matter; kexp lets the kernel check that and raise DEV_ERR_INEXACT otherwise.
+template <int D>
+__global__ void __launch_bounds__(1024) k_channel_mean(const double* __restrict__ ksum,
+                                                      const uint8_t* __restrict__ kexp, float* __restrict__ mu,
+                                                      int NB, int N) {
+  constexpr int G = 1024 / D;
+  __shared__ double rs[G][D];
+  __shared__ uint32_t re[G][D];
+  const long long bh = blockIdx.x;
+  const int c = threadIdx.x % D, gi = threadIdx.x / D;
   double s = 0.0;
   uint32_t mx = 0u, mn = 255u;
-  for (int j = 0; j < NB; ++j) {
+  for (int j = gi; j < NB; j += G) {
     const long long o = (bh * NB + j) * (long long)D + c;
     s += ksum[o];
     mx = max(mx, (uint32_t)kexp[2 * o]);
     mn = min(mn, (uint32_t)kexp[2 * o + 1]);
+  }
+  rs[gi][c] = s;
+  re[gi][c] = (mx << 8) | mn;
+  __syncthreads();
+  if (gi != 0) return;
+  s = 0.0;
+  mx = 0u;
+  mn = 255u;
+  for (int q = 0; q < G; ++q) {
+    s += rs[q][c];
+    mx = max(mx, re[q][c] >> 8);
+    mn = min(mn, re[q][c] & 0xFFu);
   }
   int lgN = 0;
   while ((1LL << lgN) < (long long)N) ++lgN;
@@ -173,7 +309,7 @@ __global__ void k_channel_mean(const double* __restrict__ ksum, const uint8_t* _
       }
     }
   }
-  mu[t] = f;
+  mu[bh * D + c] = f;
 }
 
 }  // namespace sla

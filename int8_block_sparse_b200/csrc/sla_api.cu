@@ -123,7 +123,7 @@ template <class T>
 size_t rounded(size_t count) { return (count * sizeof(T) + 255) & ~size_t(255); }
 
 struct Workspace {
-  double* ksum; uint8_t* kexp; float* mu; double* qsum;
+  double* ksum; double* kbar; uint8_t* kexp; float* mu; double* qbar;
   int8_t* qi8; int8_t* ki8; float* sq; float* sk; int32_t* idx;
   __nv_bfloat16* notcrit; __nv_bfloat16* hstate; __nv_bfloat16* grest; float* zrest;
   long long ncpitch, hpitch;
@@ -133,7 +133,7 @@ struct Workspace {
 size_t workspace_bytes(const Shape& s, int what) {
   const size_t BH = s.BH, NB = s.NB, NP = s.NP, d = s.d, kc = s.kc;
   const size_t ncpitch = (NB + 63) / 64 * 64, hpitch = d * d + d;
-  size_t b = rounded<double>(BH * NB * d) * 2 + rounded<uint8_t>(BH * NB * d * 2) + rounded<float>(BH * d);
+  size_t b = rounded<double>(BH * NB * d) * 3 + rounded<uint8_t>(BH * NB * d * 2) + rounded<float>(BH * d);
   if (what & 1) b += rounded<int8_t>(BH * NP * d) * 2 + rounded<float>(BH * NB) * 2;
   if (what & 2) b += rounded<int32_t>(BH * NB * kc);
   if (what & 8)
@@ -150,7 +150,8 @@ Workspace carve(const Shape& s, int what, char* base) {
   w.ncpitch = (NB + 63) / 64 * 64;
   w.hpitch = d * d + d;
   w.ksum = a.take<double>(BH * NB * d);
-  w.qsum = a.take<double>(BH * NB * d);
+  w.kbar = a.take<double>(BH * NB * d);
+  w.qbar = a.take<double>(BH * NB * d);
   w.kexp = a.take<uint8_t>(BH * NB * d * 2);
   w.mu = a.take<float>(BH * d);
   if (what & 1) {
@@ -205,34 +206,47 @@ struct ProfScope {
 // ------------------------------------------------------------------ launch helpers
 template <int D, int BLK>
 int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                       Workspace& w, bool states, bool kcodes, int8_t* qi8, int8_t* ki8, float* sq, float* sk,
-                       cudaStream_t st) {
-  const size_t sm1 = kstats_smem<D, BLK>();
-  cudaFuncSetAttribute(k_kstats<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+                       const __nv_bfloat16* proj, Workspace& w, bool states, bool kcodes, int8_t* qi8,
+                       int8_t* ki8, float* sq, float* sk, cudaStream_t st) {
+  CUtensorMap mv, mw;
+  std::memset(&mv, 0, sizeof(mv));
+  std::memset(&mw, 0, sizeof(mw));
+  if (states) {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
+    cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)s.N * D * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)BLK, 1u};
+    if (!make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+    cuuint64_t wd[2] = {(cuuint64_t)D, (cuuint64_t)D};
+    cuuint64_t ws[1] = {(cuuint64_t)D * 2};
+    cuuint32_t wb[2] = {64u, (cuuint32_t)D};
+    if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, proj, wd, ws, wb, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  const int sm1 = StatsCfg<D, BLK>::SMEM;
+  cudaFuncSetAttribute(k_kstats<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
   dim3 g1((unsigned)s.NB, (unsigned)s.BH);
   { ProfScope ps(SLA_K_STATS, st);
-  k_kstats<D, BLK><<<g1, 256, sm1, st>>>(k, v, w.ksum, w.kexp, states ? w.hstate : nullptr, s.N, (int)s.NB,
-                                         w.hpitch); }
-  const long long tot = s.BH * D;
+  k_kstats<D, BLK><<<g1, 128, sm1, st>>>(mv, mw, k, w.ksum, w.kbar, w.kexp, states ? w.hstate : nullptr, s.N,
+                                         (int)s.NB, w.hpitch); }
   { ProfScope ps(SLA_K_MEAN, st);
-  k_channel_mean<<<(unsigned)((tot + 255) / 256), 256, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, D, s.N, tot); }
+  k_channel_mean<D><<<(unsigned)s.BH, 1024, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, s.N); }
   dim3 g2((unsigned)s.NB, (unsigned)s.BH, kcodes ? 2u : 1u);
   { ProfScope ps(SLA_K_QUANT, st);
-  k_quant<D, BLK><<<g2, 256, 0, st>>>(q, k, w.mu, qi8, ki8, sq, sk, w.qsum, s.N, (int)s.NB); }
+  k_quant<D, BLK><<<g2, 256, 0, st>>>(q, k, w.mu, qi8, ki8, sq, sk, w.qbar, s.N, (int)s.NB); }
   return cuda_status(cudaGetLastError());
 }
 
 template <int D>
 int launch_mask(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __nv_bfloat16* notcrit,
                 cudaStream_t st) {
-  int rows = 16;
+  int rows = 8;
   while (rows > 1 && mask_smem<D>(rows, (int)s.NB) > 200 * 1024) rows /= 2;
   const size_t sm = mask_smem<D>(rows, (int)s.NB);
   cudaFuncSetAttribute(k_mask<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   dim3 g((unsigned)((s.NB + rows - 1) / rows), (unsigned)s.BH);
   ProfScope ps(SLA_K_MASK, st);
-  k_mask<D><<<g, 256, sm, st>>>(w.qsum, w.ksum, s.N, (int)s.NB, s.block, (int)s.kc, rows, idx, bitmap, notcrit,
-                                (int)w.ncpitch);
+  k_mask<D><<<g, 256, sm, st>>>(w.qbar, w.kbar, (int)s.NB, (int)s.kc, rows, idx, bitmap, notcrit, (int)w.ncpitch);
   return cuda_status(cudaGetLastError());
 }
 
@@ -279,9 +293,9 @@ int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* v, float* o, 
 }
 
 template <int D>
-int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __nv_bfloat16* proj,
-                  const float* osparse, float* out, cudaStream_t st) {
-  CUtensorMap ma, mb, mg, mw;
+int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const float* osparse, float* out,
+                  cudaStream_t st) {
+  CUtensorMap ma, mb, mg;
   {
     cuuint64_t dims[3] = {(cuuint64_t)w.ncpitch, (cuuint64_t)s.NB, (cuuint64_t)s.BH};
     cuuint64_t str[2] = {(cuuint64_t)w.ncpitch * 2, (cuuint64_t)(w.ncpitch * s.NB * 2)};
@@ -303,13 +317,6 @@ int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __
     if (!make_map(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.grest, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return SLA_ERR_CUDA;
   }
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)D};
-    cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)D};
-    if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, proj, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return SLA_ERR_CUDA;
-  }
   LinGemmParams gp;
   gp.grest = w.grest; gp.zrest = w.zrest; gp.NB = (int)s.NB; gp.D = D; gp.E = D * D + D;
   gp.nkt = (int)((s.NB + 63) / 64);
@@ -323,7 +330,7 @@ int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __
   cudaFuncSetAttribute(k_linout<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinOutCfg<D>::SMEM);
   dim3 g2((unsigned)s.NB, (unsigned)s.BH);
   { ProfScope ps(SLA_K_LINOUT, st);
-  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, mw, op); }
+  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, op); }
   return cuda_status(cudaGetLastError());
 }
 
@@ -332,7 +339,7 @@ template <int D, int BLK>
 int run_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
              const __nv_bfloat16* proj, float* out, float* o_sparse, Workspace& w, cudaStream_t st) {
   const bool linear = s.kc < s.NB;
-  int rc = launch_stats_quant<D, BLK>(s, q, k, v, w, linear, true, w.qi8, w.ki8, w.sq, w.sk, st);
+  int rc = launch_stats_quant<D, BLK>(s, q, k, v, proj, w, linear, true, w.qi8, w.ki8, w.sq, w.sk, st);
   if (rc) return rc;
   rc = launch_mask<D>(s, w, w.idx, nullptr, linear ? w.notcrit : nullptr, st);
   if (rc) return rc;
@@ -341,7 +348,7 @@ int run_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, con
   float* osp = (linear && o_sparse != nullptr) ? o_sparse : out;
   rc = launch_attn<D, BLK>(s, w, v, osp, st);
   if (rc) return rc;
-  if (linear) return launch_linear<D>(s, w, q, proj, osp, out, st);
+  if (linear) return launch_linear<D>(s, w, q, osp, out, st);
   if (o_sparse != nullptr)
     return cuda_status(cudaMemcpyAsync(o_sparse, out, (size_t)s.BH * s.N * D * sizeof(float),
                                        cudaMemcpyDeviceToDevice, st));
@@ -372,6 +379,19 @@ struct Scratch {
     if (ptr != nullptr) cudaFreeAsync(ptr, st);
   }
 };
+
+// ------------------------------------------------------------------ failure-path self test
+// One thread waits, with the library's bounded wait, on an mbarrier that no
+// one arrives at; the wait gives up, records DEV_ERR_TIMEOUT and returns.
+__global__ void k_selftest_wait_timeout() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  (void)mbar_wait(&bar, 0, &abort_flag);
+}
 
 // ------------------------------------------------------------------ fixed scratch for sla_mask_noalloc
 // For callers that cannot allocate device memory while they run: the block
@@ -436,8 +456,7 @@ int sla_quant(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q
   return with_dims(d, block, [&](auto D_, auto B_) {
     constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
     return launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                      static_cast<const __nv_bfloat16*>(k), w, false, true, q_i8, k_i8, q_scale,
-                                      k_scale, st);
+                                      nullptr, nullptr, w, false, true, q_i8, k_i8, q_scale, k_scale, st);
   });
 }
 
@@ -457,8 +476,7 @@ int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, in
   return with_dims(d, block, [&](auto D_, auto B_) {
     constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
     int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                       static_cast<const __nv_bfloat16*>(k), w, false, false, nullptr, nullptr,
-                                       nullptr, nullptr, st);
+                                       nullptr, nullptr, w, false, false, nullptr, nullptr, nullptr, nullptr, st);
     if (r) return r;
     return launch_mask<D>(s, w, blk_idx, bitmap, nullptr, st);
   });
@@ -481,8 +499,7 @@ int sla_mask_noalloc(const void* q, const void* k, int32_t* blk_idx, uint8_t* bi
   return with_dims(d, block, [&](auto D_, auto B_) {
     constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
     int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                       static_cast<const __nv_bfloat16*>(k), w, false, false, nullptr, nullptr,
-                                       nullptr, nullptr, st);
+                                       nullptr, nullptr, w, false, false, nullptr, nullptr, nullptr, nullptr, st);
     if (r) return r;
     return launch_mask<D>(s, w, blk_idx, bitmap, nullptr, st);
   });
@@ -583,6 +600,11 @@ int sla_profile_read(double* ms, long long* launches, int n) {
     cudaEventDestroy(r.b);
   }
   return rc;
+}
+
+int sla_selftest_wait_timeout(void* stream) {
+  k_selftest_wait_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return cuda_status(cudaGetLastError());
 }
 
 int sla_get_error(void* stream) {

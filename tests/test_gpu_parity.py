@@ -175,3 +175,18 @@ def test_full_sweep(S, name):
 
 def test_full_720p(S):
     _full_case(S, "720p", per_head=2)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(S):
+    """A kernel whose barrier is never completed gives up after its bounded wait,
+    records SLA_ERR_TIMEOUT and returns; the context stays usable."""
+    import ctypes
+
+    import torch
+
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert S.lib().sla_selftest_wait_timeout(st) == 0
+    assert S.get_error() == 5
+    assert S.get_error() == 0            # the error word was cleared
+    x = make_inputs(1, 1, 256, 128, 6)
+    check_attn(x, 128, 0.5)              # the device still computes correctly
