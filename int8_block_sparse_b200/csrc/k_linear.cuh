@@ -146,7 +146,9 @@ template <int D>
 struct LinOutCfg {
   static constexpr int A_BYTES = 128 * D * 2;   // phi(Q) tile (K-major, 64-column atoms of 16 KB)
   static constexpr int G_BYTES = D * D * 2;     // G'_i (MN-major)
-  static constexpr int SMEM = A_BYTES + G_BYTES + 1024 + 128 + D * 4;
+  // after the product, A and G are reused for the 128 x D float32 result
+  static constexpr int AG_BYTES = (A_BYTES + G_BYTES > 128 * D * 4) ? A_BYTES + G_BYTES : 128 * D * 4;
+  static constexpr int SMEM = AG_BYTES + 1024 + 128 + D * 4;
 };
 
 // One CTA (128 threads, thread = query row) per query block.
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sa = base;
   unsigned char* sg = sa + C::A_BYTES;
-  float* sz = reinterpret_cast<float*>(sg + C::G_BYTES);           // z_rest of this query block
+  float* sz = reinterpret_cast<float*>(sa + C::AG_BYTES);          // z_rest of this query block
   uint64_t* bars = reinterpret_cast<uint64_t*>(sz + D);            // 0: G load, 1: MMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -237,23 +239,38 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   tc_fence_after();
   const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
   const float inv_den = (valid && den > 0.f) ? 1.f / den : 0.f;
-  const float* os = p.osparse + (bh * p.N + n) * D;
-  float* dst = p.out + (bh * p.N + n) * D;
+  // y = phi(q) G' / den, row r -> shared memory (the product is complete, so A
+  // and G are free); 16-byte chunks XOR-swizzled by the row to spread banks
+  constexpr int NCH = D / 4;                       // 16-byte chunks per row
+  float* ys = reinterpret_cast<float*>(sa);
 #pragma unroll
   for (int ch = 0; ch < D / 16; ++ch) {
     uint32_t v[16];
     SLA_TMEM_LD16(trow + ch * 16, v);
     tmem_ld_wait();
-    if (valid && ok) {
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const float4 a = *reinterpret_cast<const float4*>(os + ch * 16 + 4 * q4);
-        *reinterpret_cast<float4*>(dst + ch * 16 + 4 * q4) =
-            make_float4(fmaf(__uint_as_float(v[4 * q4]), inv_den, a.x),
-                        fmaf(__uint_as_float(v[4 * q4 + 1]), inv_den, a.y),
-                        fmaf(__uint_as_float(v[4 * q4 + 2]), inv_den, a.z),
-                        fmaf(__uint_as_float(v[4 * q4 + 3]), inv_den, a.w));
-      }
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const int c4 = ch * 4 + q4;
+      *reinterpret_cast<float4*>(ys + r * D + ((c4 ^ (r & (NCH - 1))) * 4)) =
+          make_float4(__uint_as_float(v[4 * q4]) * inv_den, __uint_as_float(v[4 * q4 + 1]) * inv_den,
+                      __uint_as_float(v[4 * q4 + 2]) * inv_den, __uint_as_float(v[4 * q4 + 3]) * inv_den);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  // out = O_sparse + y, a row at a time per warp with coalesced 16-byte accesses
+  if (ok) {
+    constexpr int RPI = 32 / NCH;                  // rows per warp instruction (1 or 2)
+    const int lane = tid & 31;
+    const int c4 = lane % NCH;
+    const int nrows = min(p.BLK, p.N - i * p.BLK);
+    const long long rowbase = bh * p.N + (long long)i * p.BLK;
+#pragma unroll 4
+    for (int rr = warp * RPI + lane / NCH; rr < nrows; rr += 4 * RPI) {
+      const float4 a = *reinterpret_cast<const float4*>(p.osparse + (rowbase + rr) * D + c4 * 4);
+      const float4 y = *reinterpret_cast<const float4*>(ys + rr * D + ((c4 ^ (rr & (NCH - 1))) * 4));
+      *reinterpret_cast<float4*>(p.out + (rowbase + rr) * D + c4 * 4) =
+          make_float4(a.x + y.x, a.y + y.y, a.z + y.z, a.w + y.w);
     }
   }
   tc_fence_before();

@@ -41,7 +41,7 @@ struct StatsCfg {
   static constexpr int P_BYTES = 128 * BLK * 2;      // phi(K)^T (MN-major A, 128 rows of a; D=64 pads)
   static constexpr int GROUPS = D / 8;               // 16-byte vectors per row
   static constexpr int RG = 128 / GROUPS;            // row groups (threads per channel group)
-  static constexpr int RED_BYTES = RG * D * (8 + 4 + 4);
+  static constexpr int RED_BYTES = 4 * D * (8 + 4 + 4);      // per-warp partials after a shuffle step
   static constexpr int SMEM = V_BYTES + W_BYTES + P_BYTES + RED_BYTES + 1024 + 128;
 };
 
@@ -60,10 +60,10 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
   unsigned char* sV = base;
   unsigned char* sW = sV + C::V_BYTES;
   unsigned char* sP = sW + C::W_BYTES;
-  double* red = reinterpret_cast<double*>(sP + C::P_BYTES);        // [RG][D]
-  float* redz = reinterpret_cast<float*>(red + RG * D);            // [RG][D]
-  uint32_t* rede = reinterpret_cast<uint32_t*>(redz + RG * D);     // [RG][D] max<<8 | min
-  uint64_t* bars = reinterpret_cast<uint64_t*>(rede + RG * D);     // 0: TMA, 1: MMA0, 2: MMA1
+  double* red = reinterpret_cast<double*>(sP + C::P_BYTES);        // [4 warps][D]
+  float* redz = reinterpret_cast<float*>(red + 4 * D);             // [4][D]
+  uint32_t* rede = reinterpret_cast<uint32_t*>(redz + 4 * D);      // [4][D] max<<8 | min
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rede + 4 * D);      // 0: TMA, 1: MMA0, 2: MMA1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -99,18 +99,26 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
     }
   }
 
-  // K rows: float64 sums, exponent range, phi (float32 sums for z, bf16 for h')
+  // K rows: float64 sums, exponent range, phi (float32 sums for z, bf16 for h').
+  // All of the thread's rows are loaded first, so their DRAM latencies overlap.
   const __nv_bfloat16* kb = K + (bh * N + row0) * (long long)D;
   const int g = tid % GROUPS, rg = tid / GROUPS;
+  constexpr int NR = BLK / RG;   // rows per thread
+  uint4 kr[NR];
+#pragma unroll
+  for (int t = 0; t < NR; ++t) {
+    const int r = rg + t * RG;
+    kr[t] = (r < rows) ? *reinterpret_cast<const uint4*>(kb + (long long)r * D + g * 8) : make_uint4(0, 0, 0, 0);
+  }
   double part[8];
   float zp[8];
   uint32_t emax[8], emin[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) { part[e] = 0.0; zp[e] = 0.f; emax[e] = 0u; emin[e] = 255u; }
-  for (int r = rg; r < BLK; r += RG) {
-    uint4 kr = make_uint4(0, 0, 0, 0);
-    if (r < rows) kr = *reinterpret_cast<const uint4*>(kb + (long long)r * D + g * 8);
-    const uint16_t* kh = reinterpret_cast<const uint16_t*>(&kr);
+#pragma unroll
+  for (int t = 0; t < NR; ++t) {
+    const int r = rg + t * RG;
+    const uint16_t* kh = reinterpret_cast<const uint16_t*>(&kr[t]);
     uint32_t pk[4];
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
@@ -139,11 +147,24 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
     for (int e = tid; e < BLK * 128 / 16; e += 128)
       reinterpret_cast<uint4*>(sP + BLK * 128)[e] = make_uint4(0, 0, 0, 0);
   }
+  // lanes of a warp that share a channel group first combine (fixed order)
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    red[rg * D + g * 8 + e] = part[e];
-    redz[rg * D + g * 8 + e] = zp[e];
-    rede[rg * D + g * 8 + e] = (emax[e] << 8) | emin[e];
+  for (int o = GROUPS; o < 32; o <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      part[e] += __shfl_xor_sync(0xffffffffu, part[e], o);
+      zp[e] += __shfl_xor_sync(0xffffffffu, zp[e], o);
+      emax[e] = max(emax[e], __shfl_xor_sync(0xffffffffu, emax[e], o));
+      emin[e] = min(emin[e], __shfl_xor_sync(0xffffffffu, emin[e], o));
+    }
+  }
+  if ((tid & 31) < GROUPS) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      red[warp * D + g * 8 + e] = part[e];
+      redz[warp * D + g * 8 + e] = zp[e];
+      rede[warp * D + g * 8 + e] = (emax[e] << 8) | emin[e];
+    }
   }
   fence_async_shared();
   __syncthreads();
@@ -151,7 +172,7 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
     double s = 0.0;
     float z = 0.f;
     uint32_t mx = 0u, mn = 255u;
-    for (int q = 0; q < RG; ++q) {
+    for (int q = 0; q < 4; ++q) {
       s += red[q * D + tid];
       z += redz[q * D + tid];
       const uint32_t w = rede[q * D + tid];
