@@ -12,7 +12,10 @@
 //
 // One persistent CTA per SM runs two independent pipelines ("tiles"), each
 // working on its own sequence of (head, query block) items:
-//   warp 0 / 2   TMA producer of tile 0 / 1 (Q once per item, K/V ring of 2)
+//   warp 0 / 2   TMA producers of tile 0 / 1: lane 0 loads Q and K, lane 1 V
+//                (two-stage rings; a K stage is released when its block's QK^T
+//                products finish, a V stage when its PV products finish, so
+//                the next K tile is not held up by the PV of the previous one)
 //   warp 1 / 3   tcgen05.mma issuer of tile 0 / 1
 //   warps 4-7    softmax + epilogue of tile 0 (thread = query row = TMEM lane)
 //   warps 8-11   softmax + epilogue of tile 1
@@ -60,7 +63,7 @@ struct AttnCfg {
 struct TileBars {
   uint64_t q_full, q_empty, o_full, o_free;
   uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t kv_full[2], kv_empty[2];
+  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -95,8 +98,10 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
         mbar_init(&b.s_full[s], 1);
         mbar_init(&b.p_full[s], 128);
         mbar_init(&b.pv_done[s], 1);
-        mbar_init(&b.kv_full[s], 1);
-        mbar_init(&b.kv_empty[s], 1);
+        mbar_init(&b.k_full[s], 1);
+        mbar_init(&b.k_empty[s], 1);
+        mbar_init(&b.v_full[s], 1);
+        mbar_init(&b.v_empty[s], 1);
       }
     }
     *abort_flag = 0;
@@ -120,45 +125,45 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
     TileBars& b = bars[u];
     unsigned char* tq = base + u * C::TILE_BYTES;
     if ((warp & 1) == 0) {
-      // ------------------------------------------------------------ producer
-      // The whole warp walks the block list (32 entries per load); lane 0
-      // issues the waits and the TMA copies.
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-      }
-      uint32_t kv_it = 0, item_it = 0;
-      int ok = 1;
-      for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
-        const int bh = item / NB, i = item % NB;
+      // ------------------------------------------------------------ producers
+      // Lane 0 loads Q and the K tiles, lane 1 the V tiles; each walks the
+      // block list on its own, reading the next entry one block ahead.
+      if (lane < 2) {
         if (lane == 0) {
-          ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag);
-          if (ok) {
+          tma_prefetch_desc(&tm_q);
+          tma_prefetch_desc(&tm_k);
+        } else {
+          tma_prefetch_desc(&tm_v);
+        }
+        uint32_t blk_it = 0, item_it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
+          const int bh = item / NB, i = item % NB;
+          if (lane == 0) {
+            if (!(ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag))) break;
             mbar_expect_tx(&b.q_full, C::Q_BYTES);
             tma_load_2d(tq, &tm_q, &b.q_full, 0, bh * p.NP + i * BLK);
           }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
-        int jl = 0;
-        for (int t = 0; t < kc && ok; ++t, ++kv_it) {
-          if ((t & 31) == 0) jl = (t + lane < kc) ? __ldg(lst + t + lane) : 0;
-          const int j = __shfl_sync(0xffffffffu, jl, t & 31);
-          if (lane == 0) {
-            const int s = kv_it & 1;
+          const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
+          int jn = __ldg(lst);
+          for (int t = 0; t < kc; ++t, ++blk_it) {
+            const int j = jn;
+            if (t + 1 < kc) jn = __ldg(lst + t + 1);
+            const int s = blk_it & 1;
+            const uint32_t par = ((blk_it >> 1) & 1) ^ 1;
             unsigned char* tk = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES);
-            unsigned char* tv = tk + C::K_BYTES;
-            ok = mbar_wait(&b.kv_empty[s], ((kv_it >> 1) & 1) ^ 1, abort_flag);
-            if (ok) {
-              mbar_expect_tx(&b.kv_full[s], C::K_BYTES + C::V_BYTES);
-              tma_load_2d(tk, &tm_k, &b.kv_full[s], 0, bh * p.NP + j * BLK);
+            if (lane == 0) {
+              if (!(ok = mbar_wait(&b.k_empty[s], par, abort_flag))) break;
+              mbar_expect_tx(&b.k_full[s], C::K_BYTES);
+              tma_load_2d(tk, &tm_k, &b.k_full[s], 0, bh * p.NP + j * BLK);
+            } else {
+              if (!(ok = mbar_wait(&b.v_empty[s], par, abort_flag))) break;
+              mbar_expect_tx(&b.v_full[s], C::V_BYTES);
 #pragma unroll
               for (int hh = 0; hh < D / 64; ++hh)
-                tma_load_3d(tv + hh * BLK * 128, &tm_v, &b.kv_full[s], hh * 64, j * BLK, bh);
+                tma_load_3d(tk + C::K_BYTES + hh * BLK * 128, &tm_v, &b.v_full[s], hh * 64, j * BLK, bh);
             }
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
         }
       }
     } else {
@@ -181,7 +186,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             const uint32_t blk_it = kv_it + y / NH;
             const int s = blk_it & 1;
             if (y % NH == 0) {
-              if (!mbar_wait(&b.kv_full[s], (blk_it >> 1) & 1, abort_flag)) return false;
+              if (!mbar_wait(&b.k_full[s], (blk_it >> 1) & 1, abort_flag)) return false;
               tc_fence_after();
             }
             unsigned char* tk = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES);
@@ -191,6 +196,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             for (int kk = 0; kk < D / 32; ++kk)
               mma_i8_ss(dS, dq + uint64_t(kk * 2), dk + uint64_t(kk * 2), id_qk, kk > 0 ? 1u : 0u);
             tc_commit(&b.s_full[g & 1]);
+            if (y % NH == NH - 1) tc_commit(&b.k_empty[s]);
             if (y == H - 1) tc_commit(&b.q_empty);
             return true;
           };
@@ -200,8 +206,10 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             const uint32_t g = hg + x;
             if (!(ok = mbar_wait(&b.p_full[g & 1], (g >> 1) & 1, abort_flag))) break;
             if (x == 0 && !(ok = mbar_wait(&b.o_free, (item_it & 1) ^ 1, abort_flag))) break;
+            const uint32_t vblk = kv_it + x / NH;
+            const int s = vblk & 1;
+            if (x % NH == 0 && !(ok = mbar_wait(&b.v_full[s], (vblk >> 1) & 1, abort_flag))) break;
             tc_fence_after();
-            const int s = (kv_it + x / NH) & 1;
             unsigned char* tv = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES) + C::K_BYTES;
             const uint64_t dv = smem_desc(smem_u32(tv) + (x % NH) * C::V_HALF_BYTES, BLK * 128, 1024, 2);
             const uint32_t aP = tS + (g & 1) * 64;
@@ -209,7 +217,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             for (int kk = 0; kk < C::HB / 16; ++kk)
               mma_bf16_ts(tO, aP + kk * 8, dv + uint64_t(kk * (2048 >> 4)), id_pv, (x > 0 || kk > 0) ? 1u : 0u);
             tc_commit(&b.pv_done[g & 1]);
-            if (x % NH == NH - 1) tc_commit(&b.kv_empty[s]);
+            if (x % NH == NH - 1) tc_commit(&b.v_empty[s]);
             if (x == H - 1) tc_commit(&b.o_full);
             if (x + 2 < H) ok = issue_qk(x + 2);
           }

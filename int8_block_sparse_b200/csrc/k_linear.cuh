@@ -258,19 +258,32 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   }
   tc_fence_before();
   __syncthreads();
-  // out = O_sparse + y, a row at a time per warp with coalesced 16-byte accesses
+  // out = O_sparse + y with coalesced 16-byte accesses; each warp takes
+  // RB rows per round and issues all their O_sparse loads before using them
   if (ok) {
     constexpr int RPI = 32 / NCH;                  // rows per warp instruction (1 or 2)
+    constexpr int RB = 8;                          // row groups in flight per warp
     const int lane = tid & 31;
     const int c4 = lane % NCH;
     const int nrows = min(p.BLK, p.N - i * p.BLK);
     const long long rowbase = bh * p.N + (long long)i * p.BLK;
-#pragma unroll 4
-    for (int rr = warp * RPI + lane / NCH; rr < nrows; rr += 4 * RPI) {
-      const float4 a = *reinterpret_cast<const float4*>(p.osparse + (rowbase + rr) * D + c4 * 4);
-      const float4 y = *reinterpret_cast<const float4*>(ys + rr * D + ((c4 ^ (rr & (NCH - 1))) * 4));
-      *reinterpret_cast<float4*>(p.out + (rowbase + rr) * D + c4 * 4) =
-          make_float4(a.x + y.x, a.y + y.y, a.z + y.z, a.w + y.w);
+    for (int r0 = warp * RPI * RB; r0 < nrows; r0 += 4 * RPI * RB) {
+      float4 a[RB];
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+        const int rr = r0 + k * RPI + lane / NCH;
+        a[k] = (rr < nrows) ? *reinterpret_cast<const float4*>(p.osparse + (rowbase + rr) * D + c4 * 4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+        const int rr = r0 + k * RPI + lane / NCH;
+        if (rr < nrows) {
+          const float4 y = *reinterpret_cast<const float4*>(ys + rr * D + ((c4 ^ (rr & (NCH - 1))) * 4));
+          *reinterpret_cast<float4*>(p.out + (rowbase + rr) * D + c4 * 4) =
+              make_float4(a[k].x + y.x, a[k].y + y.y, a[k].z + y.z, a[k].w + y.w);
+        }
+      }
     }
   }
   tc_fence_before();
