@@ -73,8 +73,11 @@ typedef enum {
                                channel's values span more exponents than a float64
                                sum holds exactly (sla_get_error; results are still
                                written)                                            */
-  SLA_ERR_SCRATCH_LIMIT = 7 /* sla_mask_noalloc: the problem needs more scratch than
+  SLA_ERR_SCRATCH_LIMIT = 7, /* sla_mask_noalloc: the problem needs more scratch than
                                its fixed device buffer holds                       */
+  SLA_ERR_SMEM_LAYOUT = 8   /* a kernel's dynamic shared memory did not start on a
+                               boundary that leaves room for its aligned tiles; the
+                               kernel wrote nothing (sla_get_error)                */
 } sla_status;
 
 /* Number of key blocks each query block keeps:
@@ -150,6 +153,7 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device: SLA_ERR_TIMEOUT if a kernel's bounded wait gave up,
  * SLA_ERR_INEXACT_MEAN if a channel mean could not be proven exact,
+ * SLA_ERR_SMEM_LAYOUT if a kernel could not place its shared-memory tiles,
  * SLA_ERR_CUDA if the synchronisation itself failed, else SLA_OK. */
 int sla_get_error(void* stream);
 

@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(HERE, "libsla.so")
 
 SLA_OK = 0
 STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "SLA_ERR_CUDA",
-                4: "SLA_ERR_OOM", 5: "SLA_ERR_TIMEOUT", 6: "SLA_ERR_INEXACT_MEAN", 7: "SLA_ERR_SCRATCH_LIMIT"}
+                4: "SLA_ERR_OOM", 5: "SLA_ERR_TIMEOUT", 6: "SLA_ERR_INEXACT_MEAN", 7: "SLA_ERR_SCRATCH_LIMIT",
+                8: "SLA_ERR_SMEM_LAYOUT"}
 
 EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
            "sla_get_error", "sla_status_string", "sla_profile_enable", "sla_profile_read",

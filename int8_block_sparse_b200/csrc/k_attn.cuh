@@ -51,9 +51,15 @@ struct AttnCfg {
   static constexpr int V_BYTES = BLK * D * 2;    // bf16
   static constexpr int STAGES = 2;
   static constexpr int TILE_BYTES = Q_BYTES + STAGES * (K_BYTES + V_BYTES);
-  // at least 120 KB, so that one CTA (holding all 512 TMEM columns) fills an SM
-  static constexpr int SMEM_USED = 2 * TILE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr int SMEM = SMEM_USED > 122880 ? SMEM_USED : 122880;
+  static constexpr int BAR_BYTES = 2 * 20 * 8 + 16;         // two TileBars, TMEM slot, abort flag
+  static constexpr int SMEM_USED = 2 * TILE_BYTES + BAR_BYTES;
+  static constexpr int SMEM_LIMIT = 232448;                  // 227 KB per CTA
+  static_assert(SMEM_USED <= SMEM_LIMIT, "tile rings do not fit in shared memory");
+  // room to round the base up to 1024 bytes where the limit allows (checked at
+  // run time), and at least 120 KB, so that one CTA (holding all 512 TMEM
+  // columns) fills an SM
+  static constexpr int SMEM_ALIGNED = SMEM_USED + 1024 < SMEM_LIMIT ? SMEM_USED + 1024 : SMEM_LIMIT;
+  static constexpr int SMEM = SMEM_ALIGNED > 122880 ? SMEM_ALIGNED : 122880;
   static constexpr uint32_t KSW = (D == 128) ? 2u : 4u;     // Q/K swizzle: 128B or 64B rows
   static constexpr uint32_t KSBO = (D == 128) ? 1024u : 512u;
   static constexpr uint32_t K_HALF_BYTES = HB * D;          // 64 rows of K (int8)
@@ -64,6 +70,7 @@ struct TileBars {
   uint64_t q_full, q_empty, o_full, o_free;
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t mma_drain, pad;   // end of the MMA issuer: every MMA it issued has finished
 };
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -81,6 +88,11 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  static_assert(sizeof(TileBars) == 20 * 8, "barrier block size");
+  if (uint32_t(base - smem_raw) + C::SMEM_USED > dynamic_smem_bytes()) {
+    if (threadIdx.x == 0) raise_error(DEV_ERR_LAYOUT);
+    return;   // uniform: every thread sees the same base
+  }
   TileBars* bars = reinterpret_cast<TileBars*>(base + 2 * C::TILE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -94,6 +106,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
       mbar_init(&b.q_empty, 1);
       mbar_init(&b.o_full, 1);
       mbar_init(&b.o_free, 128);
+      mbar_init(&b.mma_drain, 1);
       for (int s = 0; s < 2; ++s) {
         mbar_init(&b.s_full[s], 1);
         mbar_init(&b.p_full[s], 128);
@@ -136,6 +149,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
           tma_prefetch_desc(&tm_v);
         }
         uint32_t blk_it = 0, item_it = 0;
+        uint32_t nq = 0, nkv = 0;   // loads issued: Q (lane 0), K or V (lane 0 / lane 1)
         bool ok = true;
         for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
           const int bh = item / NB, i = item % NB;
@@ -143,6 +157,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             if (!(ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag))) break;
             mbar_expect_tx(&b.q_full, C::Q_BYTES);
             tma_load_2d(tq, &tm_q, &b.q_full, 0, bh * p.NP + i * BLK);
+            ++nq;
           }
           const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
           int jn = __ldg(lst);
@@ -156,15 +171,22 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
               if (!(ok = mbar_wait(&b.k_empty[s], par, abort_flag))) break;
               mbar_expect_tx(&b.k_full[s], C::K_BYTES);
               tma_load_2d(tk, &tm_k, &b.k_full[s], 0, bh * p.NP + j * BLK);
+              ++nkv;
             } else {
               if (!(ok = mbar_wait(&b.v_empty[s], par, abort_flag))) break;
               mbar_expect_tx(&b.v_full[s], C::V_BYTES);
 #pragma unroll
               for (int hh = 0; hh < D / 64; ++hh)
                 tma_load_3d(tk + C::K_BYTES + hh * BLK * 128, &tm_v, &b.v_full[s], hh * 64, j * BLK, bh);
+              ++nkv;
             }
           }
         }
+        // Loads still in flight (only after a failed wait) land before the CTA
+        // exits: wait (bounded) for the last phase armed on each barrier.
+        if (lane == 0 && nq > 0) (void)mbar_wait(&b.q_full, (nq - 1) & 1, nullptr);
+        for (uint32_t bb = nkv > 2 ? nkv - 2 : 0; bb < nkv; ++bb)
+          (void)mbar_wait(lane == 0 ? &b.k_full[bb & 1] : &b.v_full[bb & 1], (bb >> 1) & 1, nullptr);
       }
     } else {
       // ------------------------------------------------------------ MMA issuer
@@ -224,6 +246,9 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
           hg += H;
           kv_it += kc;
         }
+        // every MMA issued here finishes before the CTA frees TMEM (bounded)
+        tc_commit(&b.mma_drain);
+        (void)mbar_wait(&b.mma_drain, 0, nullptr);
       }
     }
   } else {

@@ -614,6 +614,7 @@ int sla_get_error(void* stream) {
   if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SLA_ERR_CUDA;
   if (word & DEV_ERR_TIMEOUT) return SLA_ERR_TIMEOUT;
   if (word & DEV_ERR_INEXACT) return SLA_ERR_INEXACT_MEAN;
+  if (word & DEV_ERR_LAYOUT) return SLA_ERR_SMEM_LAYOUT;
   return SLA_OK;
 }
 

@@ -14,7 +14,14 @@ __device__ unsigned int g_error_word;
 enum : unsigned int {
   DEV_ERR_TIMEOUT = 1u,   // a bounded mbarrier wait gave up
   DEV_ERR_INEXACT = 2u,   // a float64 block sum may have rounded (exponent span too wide)
+  DEV_ERR_LAYOUT = 4u,    // dynamic shared memory too small for the aligned layout
 };
+
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t v;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+  return v;
+}
 
 __device__ __forceinline__ void raise_error(unsigned int code) { atomicOr(&g_error_word, code); }
 
