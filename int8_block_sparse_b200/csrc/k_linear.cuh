@@ -30,12 +30,12 @@ struct LinGemmParams {
   int nkt;                // number of 64-wide K steps
 };
 
-constexpr int LG_STAGES = 4;
+constexpr int LG_STAGES = 2;   // two CTAs per SM: one drains its epilogue while the other loads
 constexpr int LG_A_BYTES = 128 * 64 * 2;   // 16 KB
 constexpr int LG_B_BYTES = 64 * 256 * 2;   // 32 KB
 constexpr int LG_SMEM = LG_STAGES * (LG_A_BYTES + LG_B_BYTES) + 1024 + 256;
 
-__global__ void __launch_bounds__(128, 1) k_lingemm(const __grid_constant__ CUtensorMap tm_a,
+__global__ void __launch_bounds__(128, 2) k_lingemm(const __grid_constant__ CUtensorMap tm_a,
                                                     const __grid_constant__ CUtensorMap tm_b,
                                                     const LinGemmParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];

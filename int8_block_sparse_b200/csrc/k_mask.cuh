@@ -8,12 +8,17 @@
 // the kc largest scores are the kc largest probabilities; equal scores go to
 // the lower block index.  The kept indices are written in ascending order.
 //
-// One CTA handles R query blocks of one head (R = 8: a warp per row): it stages
-// the pooled query blocks and, 32 at a time, the pooled key blocks in shared
-// memory (each lane takes one key block and four independent partial dot
-// products), writes the R x NB scores to shared memory, then each warp selects
-// the top kc of its row by a bitwise search for the kc-th largest
-// order-preserving key.
+// One CTA handles R query blocks of one head (R <= 8: a warp per row in the
+// selection; R = 8 unless the scores of a long sequence need a smaller R to fit
+// in shared memory).  Scores: thread t takes key blocks t, t + 256, ... and computes
+// the R dot products of its key block with the R pooled query blocks (staged
+// in shared memory, read as broadcasts), each as four interleaved partial sums
+// over the channels (c mod 4) added as (a0 + a1) + (a2 + a3); its pooled key
+// block is read once, straight from global memory.  Selection: each warp turns
+// its row into order-preserving 64-bit keys and finds the kc-th largest by a
+// bitwise search over the high 32 bits (warp reductions with redux.sync), then
+// over the low 32 bits of the keys tied at that high half, if they are not all
+// kept.
 #pragma once
 #include "sm100.cuh"
 
@@ -24,16 +29,14 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
   return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
-template <int D>
+template <int D, int R>
 __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, const double* __restrict__ kbar,
-                                             int NB, int kc, int rows_per_cta,
-                                             int32_t* __restrict__ idx, uint8_t* __restrict__ bitmap,
+                                             int NB, int kc, int32_t* __restrict__ idx, uint8_t* __restrict__ bitmap,
                                              __nv_bfloat16* __restrict__ notcrit, int ncpitch) {
+  static_assert(R >= 1 && R <= 8, "one warp per row in the selection");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const int R = rows_per_cta;
   double* qb = reinterpret_cast<double*>(smem_raw);   // [R][D]
-  double* kbs = qb + R * D;                           // [32][D+1]
-  double* sc = kbs + 32 * (D + 1);                    // [R][NB]
+  double* sc = qb + R * D;                            // [R][NB]
 
   const long long bh = blockIdx.y;
   const int i0 = blockIdx.x * R;
@@ -45,43 +48,73 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, c
     const int r = e / D;
     qb[e] = (r < nrows) ? qbar[(bh * NB + i0) * (long long)D + e] : 0.0;
   }
-  for (int j0 = 0; j0 < NB; j0 += 32) {
-    __syncthreads();
-    for (int e = tid; e < 32 * D; e += 256) {
-      const int r = e / D, c = e % D;
-      kbs[r * (D + 1) + c] = (j0 + r < NB) ? kbar[(bh * NB + j0 + r) * (long long)D + c] : 0.0;
-    }
-    __syncthreads();
-    const int j = j0 + lane;
-    for (int r = warp; r < nrows; r += 8) {
-      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-#pragma unroll 4
-      for (int c = 0; c < D; c += 4) {
-        a0 = fma(qb[r * D + c], kbs[lane * (D + 1) + c], a0);
-        a1 = fma(qb[r * D + c + 1], kbs[lane * (D + 1) + c + 1], a1);
-        a2 = fma(qb[r * D + c + 2], kbs[lane * (D + 1) + c + 2], a2);
-        a3 = fma(qb[r * D + c + 3], kbs[lane * (D + 1) + c + 3], a3);
+  __syncthreads();
+  for (int j = tid; j < NB; j += 256) {
+    const double2* kr = reinterpret_cast<const double2*>(kbar + (bh * NB + j) * (long long)D);
+    double a[R][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0.0;
+#pragma unroll 2
+    for (int c = 0; c < D; c += 4) {
+      const double2 k01 = __ldg(kr + c / 2), k23 = __ldg(kr + c / 2 + 1);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const double2 q01 = *reinterpret_cast<const double2*>(qb + r * D + c);
+        const double2 q23 = *reinterpret_cast<const double2*>(qb + r * D + c + 2);
+        a[r][0] = fma(q01.x, k01.x, a[r][0]);
+        a[r][1] = fma(q01.y, k01.y, a[r][1]);
+        a[r][2] = fma(q23.x, k23.x, a[r][2]);
+        a[r][3] = fma(q23.y, k23.y, a[r][3]);
       }
-      if (j < NB) sc[r * NB + j] = ((a0 + a1) + (a2 + a3)) / sqd;
     }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (r < nrows) sc[r * NB + j] = ((a[r][0] + a[r][1]) + (a[r][2] + a[r][3])) / sqd;
   }
   __syncthreads();
 
   for (int r = warp; r < nrows; r += 8) {
     const int i = i0 + r;
-    const double* row = sc + r * NB;
-    // kc-th largest key
-    unsigned long long T = 0ull;
-    for (int bit = 63; bit >= 0; --bit) {
-      const unsigned long long cand = T | (1ull << bit);
-      int cnt = 0;
-      for (int j = lane; j < NB; j += 32) cnt += (order_key(row[j]) >= cand) ? 1 : 0;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-      if (cnt >= kc) T = cand;
+    // scores -> order-preserving 64-bit keys, in place
+    unsigned long long* rk = reinterpret_cast<unsigned long long*>(sc + r * NB);
+    for (int j = lane; j < NB; j += 32) rk[j] = order_key(sc[r * NB + j]);
+    __syncwarp();
+    const uint32_t* w32 = reinterpret_cast<const uint32_t*>(rk);   // word 2j: low half, 2j+1: high half
+    // T = the kc-th largest key: first the kc-th largest high half Th, then,
+    // among the keys whose high half is Th, the (kc - #above)-th largest low half
+    uint32_t Th = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = Th | (1u << bit);
+      uint32_t cnt = 0u;
+      for (int j = lane; j < NB; j += 32) cnt += (w32[2 * j + 1] >= cand) ? 1u : 0u;
+      if (__reduce_add_sync(0xffffffffu, cnt) >= (uint32_t)kc) Th = cand;
     }
+    uint32_t above = 0u, tied = 0u, tied_min = 0xFFFFFFFFu;
+    for (int j = lane; j < NB; j += 32) {
+      const uint32_t h = w32[2 * j + 1];
+      above += (h > Th) ? 1u : 0u;
+      if (h == Th) {
+        ++tied;
+        tied_min = min(tied_min, w32[2 * j]);
+      }
+    }
+    above = __reduce_add_sync(0xffffffffu, above);
+    tied = __reduce_add_sync(0xffffffffu, tied);
+    tied_min = __reduce_min_sync(0xffffffffu, tied_min);
+    const uint32_t need = (uint32_t)kc - above;   // >= 1: at least kc high halves are >= Th
+    uint32_t Tl = tied_min;                       // all tied keys are kept
+    if (tied != need) {
+      Tl = 0u;
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = Tl | (1u << bit);
+        uint32_t cnt = 0u;
+        for (int j = lane; j < NB; j += 32) cnt += (w32[2 * j + 1] == Th && w32[2 * j] >= cand) ? 1u : 0u;
+        if (__reduce_add_sync(0xffffffffu, cnt) >= need) Tl = cand;
+      }
+    }
+    const unsigned long long T = ((unsigned long long)Th << 32) | Tl;
     int gt = 0;
-    for (int j = lane; j < NB; j += 32) gt += (order_key(row[j]) > T) ? 1 : 0;
+    for (int j = lane; j < NB; j += 32) gt += (rk[j] > T) ? 1 : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
     const int need_eq = kc - gt;
@@ -89,7 +122,7 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, c
     int32_t* dst = idx + (bh * NB + i) * (long long)kc;
     for (int j0 = 0; j0 < NB; j0 += 32) {
       const int j = j0 + lane;
-      const unsigned long long key = (j < NB) ? order_key(row[j]) : 0ull;
+      const unsigned long long key = (j < NB) ? rk[j] : 0ull;
       const bool inb = j < NB;
       const bool eq = inb && key == T;
       const unsigned eqmask = __ballot_sync(0xffffffffu, eq);
@@ -113,7 +146,7 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, c
 
 template <int D>
 size_t mask_smem(int rows, int NB) {
-  return (size_t(rows) * D + 32 * (D + 1) + size_t(rows) * NB) * sizeof(double);
+  return (size_t(rows) * D + size_t(rows) * NB) * sizeof(double);
 }
 
 }  // namespace sla

@@ -39,14 +39,18 @@ struct StatsCfg {
   static constexpr int V_BYTES = BLK * D * 2;        // V tile, then V' (MN-major, 64-channel atoms)
   static constexpr int W_BYTES = D * D * 2;          // W_proj (MN-major B)
   static constexpr int P_BYTES = 128 * BLK * 2;      // phi(K)^T (MN-major A, 128 rows of a; D=64 pads)
+  static constexpr int THREADS = 256;
+  static constexpr int WARPS = THREADS / 32;
   static constexpr int GROUPS = D / 8;               // 16-byte vectors per row
-  static constexpr int RG = 128 / GROUPS;            // row groups (threads per channel group)
-  static constexpr int RED_BYTES = 4 * D * (8 + 4 + 4);      // per-warp partials after a shuffle step
+  static constexpr int RG = THREADS / GROUPS;        // row groups (threads per channel group)
+  static constexpr int RED_BYTES = WARPS * D * (8 + 4 + 2);  // per-warp partials after a shuffle step
+  // two CTAs per SM (228 KB, 1 KB of it reserved per CTA)
   static constexpr int SMEM = V_BYTES + W_BYTES + P_BYTES + RED_BYTES + 1024 + 128;
+  static_assert(D != 128 || BLK != 128 || 2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensorMap tm_v,
+__global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUtensorMap tm_v,
                                                const __grid_constant__ CUtensorMap tm_w,
                                                const __nv_bfloat16* __restrict__ K, double* __restrict__ ksum,
                                                double* __restrict__ kbar, uint8_t* __restrict__ kexp,
@@ -60,10 +64,10 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
   unsigned char* sV = base;
   unsigned char* sW = sV + C::V_BYTES;
   unsigned char* sP = sW + C::W_BYTES;
-  double* red = reinterpret_cast<double*>(sP + C::P_BYTES);        // [4 warps][D]
-  float* redz = reinterpret_cast<float*>(red + 4 * D);             // [4][D]
-  uint32_t* rede = reinterpret_cast<uint32_t*>(redz + 4 * D);      // [4][D] max<<8 | min
-  uint64_t* bars = reinterpret_cast<uint64_t*>(rede + 4 * D);      // 0: TMA, 1: MMA0, 2: MMA1
+  double* red = reinterpret_cast<double*>(sP + C::P_BYTES);        // [WARPS][D]
+  float* redz = reinterpret_cast<float*>(red + C::WARPS * D);      // [WARPS][D]
+  uint16_t* rede = reinterpret_cast<uint16_t*>(redz + C::WARPS * D);   // [WARPS][D] max<<8 | min
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rede + C::WARPS * D);   // 0: TMA, 1: MMA0, 2: MMA1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -144,7 +148,7 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
   }
   if (states && D == 64) {
     // rows a = 64..127 of the 128-row A operand are zero
-    for (int e = tid; e < BLK * 128 / 16; e += 128)
+    for (int e = tid; e < BLK * 128 / 16; e += C::THREADS)
       reinterpret_cast<uint4*>(sP + BLK * 128)[e] = make_uint4(0, 0, 0, 0);
   }
   // lanes of a warp that share a channel group first combine (fixed order)
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
     for (int e = 0; e < 8; ++e) {
       red[warp * D + g * 8 + e] = part[e];
       redz[warp * D + g * 8 + e] = zp[e];
-      rede[warp * D + g * 8 + e] = (emax[e] << 8) | emin[e];
+      rede[warp * D + g * 8 + e] = uint16_t((emax[e] << 8) | emin[e]);
     }
   }
   fence_async_shared();
@@ -172,7 +176,7 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
     double s = 0.0;
     float z = 0.f;
     uint32_t mx = 0u, mn = 255u;
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < C::WARPS; ++q) {
       s += red[q * D + tid];
       z += redz[q * D + tid];
       const uint32_t w = rede[q * D + tid];
@@ -206,22 +210,26 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
   __syncwarp();
   bool ok = mbar_wait(&bars[1], 0, abort_flag);
   tc_fence_after();
-  // thread = token row n of V': bf16 back over the V tile (same swizzled layout)
+  // token row n of V' = TMEM lane (warps w and w + 4 share a lane quarter and
+  // take half of the columns each): bf16 back over the V tile (same swizzled layout)
+  const int lrow = (warp & 3) * 32 + (tid & 31);
+  const int chalf = warp >> 2;
   {
-    const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t trow = tmem + (uint32_t((warp & 3) * 32) << 16);
 #pragma unroll
-    for (int ch = 0; ch < D / 16; ++ch) {
+    for (int cq = 0; cq < D / 32; ++cq) {
+      const int ch = chalf * (D / 32) + cq;
       uint32_t v[16];
       SLA_TMEM_LD16(trow + ch * 16, v);
       tmem_ld_wait();
-      if (tid < BLK) {
+      if (lrow < BLK) {
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
         const int c0 = ch * 16, atom = c0 / 64;
         unsigned char* dst = sV + atom * BLK * 128;
-        *reinterpret_cast<uint4*>(dst + sw128_offset(tid, (c0 % 64) / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(dst + sw128_offset(tid, (c0 % 64) / 8 + 1)) =
+        *reinterpret_cast<uint4*>(dst + sw128_offset(lrow, (c0 % 64) / 8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(dst + sw128_offset(lrow, (c0 % 64) / 8 + 1)) =
             make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
     }
@@ -247,14 +255,15 @@ __global__ void __launch_bounds__(128) k_kstats(const __grid_constant__ CUtensor
   ok = mbar_wait(&bars[2], 0, abort_flag) && ok;
   tc_fence_after();
   {
-    const uint32_t trow = tmem + D + (uint32_t(warp * 32) << 16);
-    __nv_bfloat16* hs = hstate + (bh * (long long)NB + j) * hpitch + (long long)tid * D;
+    const uint32_t trow = tmem + D + (uint32_t((warp & 3) * 32) << 16);
+    __nv_bfloat16* hs = hstate + (bh * (long long)NB + j) * hpitch + (long long)lrow * D;
 #pragma unroll
-    for (int ch = 0; ch < D / 16; ++ch) {
+    for (int cq = 0; cq < D / 32; ++cq) {
+      const int ch = chalf * (D / 32) + cq;
       uint32_t v[16];
       SLA_TMEM_LD16(trow + ch * 16, v);
       tmem_ld_wait();
-      if (ok && tid < D) {
+      if (ok && lrow < D) {
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));

@@ -227,27 +227,48 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
   cudaFuncSetAttribute(k_kstats<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm1);
   dim3 g1((unsigned)s.NB, (unsigned)s.BH);
   { ProfScope ps(SLA_K_STATS, st);
-  k_kstats<D, BLK><<<g1, 128, sm1, st>>>(mv, mw, k, w.ksum, w.kbar, w.kexp, states ? w.hstate : nullptr, s.N,
+  k_kstats<D, BLK><<<g1, StatsCfg<D, BLK>::THREADS, sm1, st>>>(mv, mw, k, w.ksum, w.kbar, w.kexp, states ? w.hstate : nullptr, s.N,
                                          (int)s.NB, w.hpitch); }
   { ProfScope ps(SLA_K_MEAN, st);
   k_channel_mean<D><<<(unsigned)s.BH, 1024, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, s.N); }
+  CUtensorMap mq, mk;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
+    cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)s.N * D * 2};
+    cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)BLK, 1u};
+    if (!make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return SLA_ERR_CUDA;
+    if (!make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return SLA_ERR_CUDA;
+  }
+  const int sm2 = QuantCfg<D, BLK>::SMEM;
+  cudaFuncSetAttribute(k_quant<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2);
   dim3 g2((unsigned)s.NB, (unsigned)s.BH, kcodes ? 2u : 1u);
   { ProfScope ps(SLA_K_QUANT, st);
-  k_quant<D, BLK><<<g2, 256, 0, st>>>(q, k, w.mu, qi8, ki8, sq, sk, w.qbar, s.N, (int)s.NB); }
+  k_quant<D, BLK><<<g2, 256, sm2, st>>>(mq, mk, w.mu, qi8, ki8, sq, sk, w.qbar, s.N, (int)s.NB); }
+  return cuda_status(cudaGetLastError());
+}
+
+template <int D, int R>
+int launch_mask_rows(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __nv_bfloat16* notcrit,
+                     cudaStream_t st) {
+  const size_t sm = mask_smem<D>(R, (int)s.NB);
+  cudaFuncSetAttribute(k_mask<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  dim3 g((unsigned)((s.NB + R - 1) / R), (unsigned)s.BH);
+  ProfScope ps(SLA_K_MASK, st);
+  k_mask<D, R><<<g, 256, sm, st>>>(w.qbar, w.kbar, (int)s.NB, (int)s.kc, idx, bitmap, notcrit, (int)w.ncpitch);
   return cuda_status(cudaGetLastError());
 }
 
 template <int D>
 int launch_mask(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __nv_bfloat16* notcrit,
                 cudaStream_t st) {
-  int rows = 8;
-  while (rows > 1 && mask_smem<D>(rows, (int)s.NB) > 200 * 1024) rows /= 2;
-  const size_t sm = mask_smem<D>(rows, (int)s.NB);
-  cudaFuncSetAttribute(k_mask<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  dim3 g((unsigned)((s.NB + rows - 1) / rows), (unsigned)s.BH);
-  ProfScope ps(SLA_K_MASK, st);
-  k_mask<D><<<g, 256, sm, st>>>(w.qbar, w.kbar, (int)s.NB, (int)s.kc, rows, idx, bitmap, notcrit, (int)w.ncpitch);
-  return cuda_status(cudaGetLastError());
+  // rows per CTA: 8 unless the R x NB float64 scores would not fit
+  const size_t lim = 200 * 1024;
+  if (mask_smem<D>(8, (int)s.NB) <= lim) return launch_mask_rows<D, 8>(s, w, idx, bitmap, notcrit, st);
+  if (mask_smem<D>(4, (int)s.NB) <= lim) return launch_mask_rows<D, 4>(s, w, idx, bitmap, notcrit, st);
+  if (mask_smem<D>(2, (int)s.NB) <= lim) return launch_mask_rows<D, 2>(s, w, idx, bitmap, notcrit, st);
+  return launch_mask_rows<D, 1>(s, w, idx, bitmap, notcrit, st);
 }
 
 int num_sms() {
