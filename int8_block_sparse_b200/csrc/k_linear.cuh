@@ -137,8 +137,6 @@ __global__ void __launch_bounds__(128, 2) k_lingemm(const __grid_constant__ CUte
 struct LinOutParams {
   const __nv_bfloat16* q;      // [BH][N][D]
   const float* zrest;          // [BH][NB][D]
-  const float* osparse;        // [BH][N][D] float32 (may be the same buffer as out)
-  float* out;                  // [BH][N][D] float32
   int N, NB, BLK;
 };
 
@@ -146,14 +144,19 @@ template <int D>
 struct LinOutCfg {
   static constexpr int A_BYTES = 128 * D * 2;   // phi(Q) tile (K-major, 64-column atoms of 16 KB)
   static constexpr int G_BYTES = D * D * 2;     // G'_i (MN-major)
-  // after the product, A and G are reused for the 128 x D float32 result
-  static constexpr int AG_BYTES = (A_BYTES + G_BYTES > 128 * D * 4) ? A_BYTES + G_BYTES : 128 * D * 4;
+  // after the product, A and G are reused for the 128 x D float32 result y,
+  // as D/32 column chunks of 32 floats (128-byte rows, 128-byte swizzle)
+  static constexpr int Y_BYTES = 128 * D * 4;
+  static constexpr int AG_BYTES = (A_BYTES + G_BYTES > Y_BYTES) ? A_BYTES + G_BYTES : Y_BYTES;
   static constexpr int SMEM = AG_BYTES + 1024 + 128 + D * 4;
 };
 
-// One CTA (128 threads, thread = query row) per query block.
+// One CTA (128 threads, thread = query row) per query block.  out holds
+// O_sparse on entry; y = phi(q) G' / den is staged in shared memory and added
+// to out by TMA reductions (float32 add in L2, one add per element).
 template <int D>
-__global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensorMap tm_g, const LinOutParams p) {
+__global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensorMap tm_g,
+                                               const __grid_constant__ CUtensorMap tm_out, const LinOutParams p) {
   using C = LinOutCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int i = blockIdx.x;
-  const long long bh = blockIdx.y;
+  const int bh = blockIdx.y;
 
   if (tid == 0) {
     mbar_init(&bars[0], 1);
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
     tmem_alloc(tmem_slot, D);
     tmem_relinquish();
   }
-  if (tid < D) sz[tid] = p.zrest[(bh * p.NB + i) * D + tid];
+  if (tid < D) sz[tid] = p.zrest[((long long)bh * p.NB + i) * D + tid];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
     mbar_expect_tx(&bars[0], C::G_BYTES);
 #pragma unroll
     for (int hh = 0; hh < D / 64; ++hh)
-      tma_load_2d(sg + hh * D * 128, &tm_g, &bars[0], hh * 64, int((bh * p.NB + i) * D));
+      tma_load_2d(sg + hh * D * 128, &tm_g, &bars[0], hh * 64, int(((long long)bh * p.NB + i) * D));
   }
 
   const int r = tid;
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   // phi(q) -> bf16 A tile (K-major, 128-byte swizzle, 64-column atoms of 16 KB)
   float den = 0.f;
   {
-    const __nv_bfloat16* qrow = p.q + (bh * p.N + n) * D;
+    const __nv_bfloat16* qrow = p.q + ((long long)bh * p.N + n) * D;
     uint4 raw[D / 8];
 #pragma unroll
     for (int c8 = 0; c8 < D / 8; ++c8)
@@ -235,60 +238,38 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
     tc_commit(&bars[1]);
   }
   __syncwarp();
-  const bool ok = mbar_wait(&bars[1], 0, abort_flag);
+  const bool ok = __syncthreads_and(mbar_wait(&bars[1], 0, abort_flag));
   tc_fence_after();
+  // y row r = phi(q_r) G' / den_r -> shared memory over A and G (the product
+  // is complete): chunk c holds columns [32c, 32c + 32) as 128-byte rows
   const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
   const float inv_den = (valid && den > 0.f) ? 1.f / den : 0.f;
-  // y = phi(q) G' / den, row r -> shared memory (the product is complete, so A
-  // and G are free); 16-byte chunks XOR-swizzled by the row to spread banks
-  constexpr int NCH = D / 4;                       // 16-byte chunks per row
-  float* ys = reinterpret_cast<float*>(sa);
 #pragma unroll
   for (int ch = 0; ch < D / 16; ++ch) {
     uint32_t v[16];
     SLA_TMEM_LD16(trow + ch * 16, v);
     tmem_ld_wait();
+    unsigned char* chunk = base + (ch >> 1) * 16384;
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int c4 = ch * 4 + q4;
-      *reinterpret_cast<float4*>(ys + r * D + ((c4 ^ (r & (NCH - 1))) * 4)) =
+    for (int q4 = 0; q4 < 4; ++q4)
+      *reinterpret_cast<float4*>(chunk + sw128_offset(r, (ch & 1) * 4 + q4)) =
           make_float4(__uint_as_float(v[4 * q4]) * inv_den, __uint_as_float(v[4 * q4 + 1]) * inv_den,
                       __uint_as_float(v[4 * q4 + 2]) * inv_den, __uint_as_float(v[4 * q4 + 3]) * inv_den);
-    }
   }
+  fence_async_shared();
   tc_fence_before();
   __syncthreads();
-  // out = O_sparse + y with coalesced 16-byte accesses; each warp takes
-  // RB rows per round and issues all their O_sparse loads before using them
-  if (ok) {
-    constexpr int RPI = 32 / NCH;                  // rows per warp instruction (1 or 2)
-    constexpr int RB = 8;                          // row groups in flight per warp
-    const int lane = tid & 31;
-    const int c4 = lane % NCH;
-    const int nrows = min(p.BLK, p.N - i * p.BLK);
-    const long long rowbase = bh * p.N + (long long)i * p.BLK;
-    for (int r0 = warp * RPI * RB; r0 < nrows; r0 += 4 * RPI * RB) {
-      float4 a[RB];
+  if (tid == 0) {
+    if (ok) {
+      // rows past N are dropped by the TMA; the box is BLK rows high
 #pragma unroll
-      for (int k = 0; k < RB; ++k) {
-        const int rr = r0 + k * RPI + lane / NCH;
-        a[k] = (rr < nrows) ? *reinterpret_cast<const float4*>(p.osparse + (rowbase + rr) * D + c4 * 4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int k = 0; k < RB; ++k) {
-        const int rr = r0 + k * RPI + lane / NCH;
-        if (rr < nrows) {
-          const float4 y = *reinterpret_cast<const float4*>(ys + rr * D + ((c4 ^ (rr & (NCH - 1))) * 4));
-          *reinterpret_cast<float4*>(p.out + (rowbase + rr) * D + c4 * 4) =
-              make_float4(a[k].x + y.x, a[k].y + y.y, a[k].z + y.z, a[k].w + y.w);
-        }
-      }
+      for (int c = 0; c < D / 32; ++c) tma_reduce_add_3d(&tm_out, base + c * 16384, c * 32, i * p.BLK, bh);
+      bulk_commit_group();
     }
+    bulk_wait_group_read0();
   }
-  tc_fence_before();
-  __syncthreads();
   tc_fence_after();
+  __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, D);
 }
 

@@ -345,13 +345,26 @@ int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const fl
   dim3 g1((unsigned)((gp.E + 255) / 256), (unsigned)((s.NB + 127) / 128), (unsigned)s.BH);
   { ProfScope ps(SLA_K_LINGEMM, st);
   k_lingemm<<<g1, 128, LG_SMEM, st>>>(ma, mb, gp); }
+  // out = O_sparse + y: out must hold O_sparse before the TMA adds y to it
+  if (osparse != out &&
+      cudaMemcpyAsync(out, osparse, (size_t)s.BH * s.N * D * sizeof(float), cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess)
+    return SLA_ERR_CUDA;
+  CUtensorMap mo;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
+    cuuint64_t str[2] = {(cuuint64_t)D * 4, (cuuint64_t)s.N * D * 4};
+    cuuint32_t box[3] = {32u, (cuuint32_t)s.block, 1u};
+    if (!make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
   LinOutParams op;
-  op.q = q; op.zrest = w.zrest; op.osparse = osparse; op.out = out;
+  op.q = q; op.zrest = w.zrest;
   op.N = s.N; op.NB = (int)s.NB; op.BLK = s.block;
   cudaFuncSetAttribute(k_linout<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinOutCfg<D>::SMEM);
   dim3 g2((unsigned)s.NB, (unsigned)s.BH);
   { ProfScope ps(SLA_K_LINOUT, st);
-  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, op); }
+  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, mo, op); }
   return cuda_status(cudaGetLastError());
 }
 
