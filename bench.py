@@ -217,23 +217,25 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle sample
 
-def oracle_sample(w, nq: int):
-    """Time the CPU oracle on head 0 of the workload: its quantisation, mask and
-    states plus the outputs of nq query blocks.  Returns (seconds, ops, sample)."""
+def oracle_sample(w, nh: int):
+    """Time the CPU oracle on every query block of the first nh heads of the
+    workload (quantisation, mask, linear states and outputs).  Returns
+    (seconds, ops, sample)."""
     import numpy as np
 
     import oracle as O
     from synth import make_workload
 
-    x = make_workload(w, heads=[0])
-    items = [(0, 0, i) for i in np.linspace(0, w.nblk - 1, nq).astype(int)]
+    nh = max(1, min(nh, w.H))
+    x = make_workload(w, heads=list(range(nh)))
+    items = [(0, h, i) for h in range(nh) for i in range(w.nblk)]
     t0 = time.perf_counter()
     O.sla_attention(x["q"], x["k"], x["v"], x["proj"], w.block, w.topk_frac, items=items)
     dt = time.perf_counter() - t0
-    ops = nq * 4.0 * w.block * w.N * w.d   # dense-equivalent ops of nq query blocks
-    return dt, ops, (f"CPU oracle on head 0 of {w.name}: per-head quantisation, mask and linear "
-                     f"states, then {nq} query blocks of {w.block} rows; value = dense-equivalent "
-                     f"ops of those rows / wall time")
+    ops = nh * 4.0 * w.N * w.N * w.d   # dense-equivalent ops of those heads
+    return dt, ops, (f"CPU oracle on heads 0..{nh - 1} of {w.name} (all {w.nblk} query blocks of "
+                     f"{w.block} rows each, with their quantisation, mask and linear states); "
+                     f"value = dense-equivalent ops of those heads / wall time")
 
 
 def blas_threads() -> int:
@@ -336,7 +338,7 @@ def run_ours(args, dist):
         "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "e2e": e2e,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
-        dt, cops, sample = oracle_sample(w, args.cpu_query_blocks)
+        dt, cops, sample = oracle_sample(w, args.cpu_heads)
         line["cpu_baseline"] = {"value": round(cops / dt / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
                                 "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
     return line
@@ -429,7 +431,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--cpu-query-blocks", type=int, default=64)
+    ap.add_argument("--cpu-heads", type=int, default=6,
+                    help="heads of the workload the CPU oracle baseline runs in full (about 10-20 s)")
     ap.add_argument("--heads", type=int, default=0,
                     help="keep only the first H heads (a smaller case for profiling; not the headline)")
     args = ap.parse_args(argv)
