@@ -123,6 +123,29 @@ def test_mask_bitmap_and_list_agree(S):
     assert np.all(np.diff(idx, axis=-1) > 0)
 
 
+def test_mask_exact_ties_go_to_the_lower_block(S):
+    """Seven identical key blocks share the top score of every query row and
+    kc = 4: the kept list must be the four lowest of them, exactly as the
+    oracle's tie rule says (exact ties are not exempt here)."""
+    from synth.workloads import f32_to_bf16_bits
+
+    B, H, N, d, block, frac = 1, 1, 1024, 64, 64, 0.25   # nblk 16, kc 4
+    rng = np.random.default_rng(21)
+    k = rng.standard_normal((B, H, N, d)).astype(np.float32)
+    q = rng.standard_normal((B, H, N, d)).astype(np.float32) * 0.1
+    k[..., 64:128, 0] += 6.0                 # key block 1: large channel-0 mean
+    for j in (3, 5, 7, 9, 11, 13):           # six exact copies of key block 1
+        k[..., j * 64:(j + 1) * 64, :] = k[..., 64:128, :]
+    q[..., 0] += 1.0                          # every query block prefers channel 0
+    qb, kb = f32_to_bf16_bits(q), f32_to_bf16_bits(k)
+    ref = O.block_mask(qb, kb, block, frac)
+    assert ref["kc"] == 4
+    assert np.all(ref["idx"] == np.array([1, 3, 5, 7], dtype=ref["idx"].dtype))
+    idx = S.sla_mask(to_dev(qb), to_dev(kb), block, frac).cpu().numpy()
+    assert S.get_error() == 0
+    assert np.array_equal(idx, ref["idx"])
+
+
 def test_host_buffers_match_device_path(S):
     import torch
 
