@@ -105,24 +105,29 @@ __global__ void __launch_bounds__(128, 2) k_lingemm(const __grid_constant__ CUte
   const int row = m0 + tid;
   const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
   const int DD = p.D * p.D;
-  {
-    for (int ch = 0; ch < 16; ++ch) {
-      uint32_t v[16];
-      SLA_TMEM_LD16(taddr + ch * 16, v);   // warp-collective: every lane loads
-      tmem_ld_wait();
-      const int e0 = n0 + ch * 16;
+  // four 16-column TMEM loads in flight per wait (the loads, not the stores,
+  // are what the epilogue waits on)
+  for (int c4 = 0; c4 < 4; ++c4) {
+    uint32_t v[4][16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) SLA_TMEM_LD16(taddr + (c4 * 4 + q) * 16, v[q]);   // warp-collective
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e0 = n0 + (c4 * 4 + q) * 16;
       if (ok && row < p.NB && e0 < p.E) {
         if (e0 < DD) {
           uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) pk[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+          for (int e = 0; e < 16; e += 2)
+            pk[e >> 1] = pack_bf16x2(__uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
           uint4* dst = reinterpret_cast<uint4*>(p.grest + ((long long)bh * p.NB + row) * DD + e0);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         } else {
           float* dst = p.zrest + ((long long)bh * p.NB + row) * p.D + (e0 - DD);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) dst[e] = __uint_as_float(v[e]);
+          for (int e = 0; e < 16; ++e) dst[e] = __uint_as_float(v[q][e]);
         }
       }
     }
@@ -155,7 +160,8 @@ struct LinOutCfg {
 // O_sparse on entry; y = phi(q) G' / den is staged in shared memory and added
 // to out by TMA reductions (float32 add in L2, one add per element).
 template <int D>
-__global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensorMap tm_g,
+__global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensorMap tm_q,
+                                               const __grid_constant__ CUtensorMap tm_g,
                                                const __grid_constant__ CUtensorMap tm_out, const LinOutParams p) {
   using C = LinOutCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -188,26 +194,29 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
   const uint32_t tmem = *tmem_slot;
 
   if (tid == 0) {
-    mbar_expect_tx(&bars[0], C::G_BYTES);
+    // the query tile lands in the A operand's own layout (K-major, 128-byte
+    // swizzle, 64-column atoms of 16 KB); rows past N arrive as zeros
+    mbar_expect_tx(&bars[0], C::G_BYTES + C::A_BYTES);
 #pragma unroll
-    for (int hh = 0; hh < D / 64; ++hh)
+    for (int hh = 0; hh < D / 64; ++hh) {
       tma_load_2d(sg + hh * D * 128, &tm_g, &bars[0], hh * 64, int(((long long)bh * p.NB + i) * D));
+      tma_load_3d(sa + hh * 16384, &tm_q, &bars[0], hh * 64, i * p.BLK, bh);
+    }
   }
 
   const int r = tid;
   const long long n = (long long)i * p.BLK + r;
   const bool valid = r < p.BLK && n < p.N;
-  // phi(q) -> bf16 A tile (K-major, 128-byte swizzle, 64-column atoms of 16 KB)
+  const bool landed = __syncthreads_and(mbar_wait(&bars[0], 0, abort_flag));
+  // phi(q) in place: each thread rewrites its own row of the A tile
   float den = 0.f;
   {
-    const __nv_bfloat16* qrow = p.q + ((long long)bh * p.N + n) * D;
-    uint4 raw[D / 8];
-#pragma unroll
-    for (int c8 = 0; c8 < D / 8; ++c8)
-      raw[c8] = valid ? *reinterpret_cast<const uint4*>(qrow + c8 * 8) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int c8 = 0; c8 < D / 8; ++c8) {
-      const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw[c8]);
+      const int atom = c8 >> 3, chunk = c8 & 7;
+      uint4* slot = reinterpret_cast<uint4*>(sa + atom * 16384 + sw128_offset(r, chunk));
+      const uint4 raw = *slot;
+      const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
       uint32_t pk[4];
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
@@ -217,15 +226,13 @@ __global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensor
         den = fmaf(f1, sz[c8 * 8 + e + 1], den);
         pk[e >> 1] = pack_bf16x2(f0, f1);
       }
-      const int atom = c8 >> 3, chunk = c8 & 7;
-      *reinterpret_cast<uint4*>(sa + atom * 16384 + sw128_offset(r, chunk)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *slot = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
   fence_async_shared();
   __syncthreads();
   if (tid == 0) {
-    const bool okl = mbar_wait(&bars[0], 0, abort_flag);
-    if (okl) {
+    if (landed) {
       tc_fence_after();
       const uint32_t idesc = idesc_bf16(D, false, true);
 #pragma unroll

@@ -350,7 +350,14 @@ int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const fl
       cudaMemcpyAsync(out, osparse, (size_t)s.BH * s.N * D * sizeof(float), cudaMemcpyDeviceToDevice, st) !=
           cudaSuccess)
     return SLA_ERR_CUDA;
-  CUtensorMap mo;
+  CUtensorMap mo, mq;
+  {
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
+    cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)s.N * D * 2};
+    cuuint32_t box[3] = {64u, 128u, 1u};
+    if (!make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
   {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
     cuuint64_t str[2] = {(cuuint64_t)D * 4, (cuuint64_t)s.N * D * 4};
@@ -364,7 +371,7 @@ int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const fl
   cudaFuncSetAttribute(k_linout<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinOutCfg<D>::SMEM);
   dim3 g2((unsigned)s.NB, (unsigned)s.BH);
   { ProfScope ps(SLA_K_LINOUT, st);
-  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mg, mo, op); }
+  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mq, mg, mo, op); }
   return cuda_status(cudaGetLastError());
 }
 
