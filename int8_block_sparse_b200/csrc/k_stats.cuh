@@ -280,20 +280,24 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
 }
 
 // mu[bh][c] = float32 nearest to (sum_j ksum[bh][j][c]) / N.  One CTA per
-// (batch, head): each thread sums every G-th block of one channel, then the G
-// partial sums are added in a fixed order.  The block sums are exact when every
-// K value of the channel is a multiple of the smallest one's unit in the last
-// place and the total stays below 2^53 of those units, so the order does not
-// matter; kexp lets the kernel check that and raise DEV_ERR_INEXACT otherwise.
+// (batch, head, group of CG channels): thread (gi, c) sums every G-th block of
+// channel c, then the G partial sums are added in a fixed order.  The block
+// sums are exact when every K value of the channel is a multiple of the
+// smallest one's unit in the last place and the total stays below 2^53 of
+// those units, so the order does not matter; kexp lets the kernel check that
+// and raise DEV_ERR_INEXACT otherwise.
+constexpr int kMeanCG = 8;   // channels per CTA
+
 template <int D>
 __global__ void __launch_bounds__(1024) k_channel_mean(const double* __restrict__ ksum,
                                                       const uint8_t* __restrict__ kexp, float* __restrict__ mu,
                                                       int NB, int N) {
-  constexpr int G = 1024 / D;
-  __shared__ double rs[G][D];
-  __shared__ uint32_t re[G][D];
+  constexpr int CG = kMeanCG;
+  constexpr int G = 1024 / CG;
+  __shared__ double rs[G][CG];
+  __shared__ uint32_t re[G][CG];
   const long long bh = blockIdx.x;
-  const int c = threadIdx.x % D, gi = threadIdx.x / D;
+  const int c = blockIdx.y * CG + threadIdx.x % CG, gi = threadIdx.x / CG;
   double s = 0.0;
   uint32_t mx = 0u, mn = 255u;
   for (int j = gi; j < NB; j += G) {
@@ -302,17 +306,17 @@ __global__ void __launch_bounds__(1024) k_channel_mean(const double* __restrict_
     mx = max(mx, (uint32_t)kexp[2 * o]);
     mn = min(mn, (uint32_t)kexp[2 * o + 1]);
   }
-  rs[gi][c] = s;
-  re[gi][c] = (mx << 8) | mn;
+  rs[gi][threadIdx.x % CG] = s;
+  re[gi][threadIdx.x % CG] = (mx << 8) | mn;
   __syncthreads();
   if (gi != 0) return;
   s = 0.0;
   mx = 0u;
   mn = 255u;
   for (int q = 0; q < G; ++q) {
-    s += rs[q][c];
-    mx = max(mx, re[q][c] >> 8);
-    mn = min(mn, re[q][c] & 0xFFu);
+    s += rs[q][threadIdx.x];
+    mx = max(mx, re[q][threadIdx.x] >> 8);
+    mn = min(mn, re[q][threadIdx.x] & 0xFFu);
   }
   int lgN = 0;
   while ((1LL << lgN) < (long long)N) ++lgN;

@@ -230,7 +230,7 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
   k_kstats<D, BLK><<<g1, StatsCfg<D, BLK>::THREADS, sm1, st>>>(mv, mw, k, w.ksum, w.kbar, w.kexp, states ? w.hstate : nullptr, s.N,
                                          (int)s.NB, w.hpitch); }
   { ProfScope ps(SLA_K_MEAN, st);
-  k_channel_mean<D><<<(unsigned)s.BH, 1024, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, s.N); }
+  k_channel_mean<D><<<dim3((unsigned)s.BH, D / kMeanCG), 1024, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, s.N); }
   CUtensorMap mq, mk;
   {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
