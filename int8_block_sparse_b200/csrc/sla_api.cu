@@ -477,6 +477,7 @@ const char* sla_status_string(int status) {
     case SLA_ERR_TIMEOUT: return "a kernel wait timed out";
     case SLA_ERR_INEXACT_MEAN: return "K channel mean not proven exact";
     case SLA_ERR_SCRATCH_LIMIT: return "problem larger than the fixed no-allocation scratch buffer";
+    case SLA_ERR_SMEM_LAYOUT: return "a kernel could not place its shared-memory tiles";
     default: return "unknown status";
   }
 }
