@@ -28,8 +28,11 @@ def test_library_exports_every_declared_function():
 
 
 def test_status_strings():
-    for code in range(0, 8):
-        assert S.status_string(code)
+    header = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    declared = {int(v): n for n, v in re.findall(r"\b(SLA_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", header)}
+    assert declared == S.STATUS_NAMES
+    for code in declared:
+        assert S.status_string(code) and S.status_string(code) != "unknown status", code
     assert S.status_string(99) == "unknown status"
 
 
