@@ -6,17 +6,16 @@
 // quantisation parameters -- here one float32 scale per block of BLK tokens x
 // D channels).  Per block: m = max|x|, s = m / 127 (IEEE float32 division),
 // code = clamp(round_half_even(float32(x / s)), -127, 127) (the clamp never
-// acts: see pack_i8x4); a block with m = 0
-// has s = 0 and zero codes.  Rows past N (up to NB*BLK) get zero codes.  For Q
-// the kernel also writes the float64 mean of each block's valid rows (the
-// pooled query block of the mask).
+// acts: see pack_i8x4); a block with m = 0 has s = 0 and zero codes.  Rows
+// past N (up to NB*BLK) get zero codes.  For Q the kernel also writes the
+// float64 mean of each block's valid rows (the pooled query block of the mask).
 //
 // The smoothed K value is recomputed (one float32 subtraction) when it is
-// quantised.  The quotient
-// x / s is taken as y0 = x * (1/s): with y = float32(x / s), |y - y0| < 2e-5
-// for |x / s| <= 128 (two float32 roundings of relative size 2^-24 plus half
-// an ulp of y), so round_half_even(y) = round_half_even(y0) unless y0 lies
-// within 3e-5 of a half-integer; only then is the IEEE division done.
+// quantised.  The quotient x / s is taken as y0 = x * (1/s): with
+// y = float32(x / s), |y - y0| < 2e-5 for |x / s| <= 128 (two float32
+// roundings of relative size 2^-24 plus half an ulp of y), so
+// round_half_even(y) = round_half_even(y0) unless y0 lies within 3e-5 of a
+// half-integer; only then is the IEEE division done.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
