@@ -1,0 +1,35 @@
+"""Builds the plain C++ CPU oracle (libsla_oracle.so) with g++.
+
+Test infrastructure: the library this builds is loaded only by the tests, the
+package's smoke check and the benchmark's CPU-baseline leg (through
+oracle/cpp_oracle.py).  -ffp-contract=off keeps every float32 and float64
+operation a separately rounded IEEE operation, as the oracle's readings state
+(and, without -ffast-math, the compiler keeps the order of every sum).
+
+Usage: python -m oracle.build   (or build() from Python).
+"""
+
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "sla_oracle.cpp")
+LIB = os.path.join(HERE, "libsla_oracle.so")
+
+
+def build(force: bool = False) -> str:
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= max(os.path.getmtime(SRC),
+                                                                         os.path.getmtime(__file__)):
+        return LIB
+    cxx = os.environ.get("CXX") or shutil.which("g++") or "g++"
+    tmp = LIB + ".tmp"
+    subprocess.run([cxx, "-O3", "-std=c++17", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
+                    "-fno-fast-math", "-o", tmp, SRC], check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))

@@ -3,7 +3,9 @@
 Each test checks one oracle function against a closed form, a library
 routine, a brute force or a hand-derived case (tests/golden/), chosen so that
 a dropped term, a wrong sign or index, or a transposed operand fails one of
-them.  No GPU needed.
+them.  Tests taking the `impl` fixture run against both oracles, the numpy
+statement (oracle/sla_oracle.py) and the plain C++ one (oracle/sla_oracle.cpp);
+the rest pin helpers only the numpy statement has.  No GPU needed.
 """
 
 import itertools
@@ -18,10 +20,19 @@ import scipy.special
 import torch
 
 import oracle as O
+from oracle import cpp_oracle as C
 from synth import make_inputs
 from synth.workloads import f32_to_bf16_bits
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+IMPLS = {"numpy": O, "cpp": C}
+
+
+@pytest.fixture(params=sorted(IMPLS))
+def impl(request):
+    """The oracle under test: the numpy statement or the plain C++ one."""
+    return IMPLS[request.param]
 
 
 def golden(name):
@@ -39,7 +50,7 @@ def bits(x):
 
 # --- number formats --------------------------------------------------------
 
-def test_round_bf16_special_values():
+def test_round_bf16_special_values(impl):
     e = 2.0 ** -8
     cases = {
         1.0: 1.0,
@@ -52,14 +63,14 @@ def test_round_bf16_special_values():
         0.0: 0.0,
     }
     for x, y in cases.items():
-        assert O.round_bf16(np.array([x]))[0] == y, x
+        assert impl.round_bf16(np.array([x]))[0] == y, x
 
 
-def test_round_bf16_matches_torch_on_float32_inputs():
+def test_round_bf16_matches_torch_on_float32_inputs(impl):
     rng = np.random.default_rng(5)
     x = (rng.standard_normal(200000) * np.exp(rng.uniform(-20, 20, 200000))).astype(np.float32)
     ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
-    assert np.array_equal(O.round_bf16(x.astype(np.float64)), ref)
+    assert np.array_equal(impl.round_bf16(x.astype(np.float64)), ref)
 
 
 def _nearest_f32_bruteforce(fr: Fraction) -> float:
@@ -86,22 +97,22 @@ def test_round_rational_to_f32_bruteforce():
 
 # --- smoothing -------------------------------------------------------------
 
-def test_channel_mean_is_exact_where_float64_summation_is_not():
+def test_channel_mean_is_exact_where_float64_summation_is_not(impl):
     # per channel: 2**100, 1, -2**100  -> exact sum 1; a float64 running sum gives 0
     k = np.zeros((1, 1, 3, 2), dtype=np.float32)
     k[0, 0, :, 0] = [2.0 ** 100, 1.0, -(2.0 ** 100)]
     k[0, 0, :, 1] = [3.0, -1.0, 2.0 ** -60]
-    mu = O.channel_mean(bits(k))
+    mu = impl.channel_mean(bits(k))
     assert mu[0, 0, 0] == np.float32(1.0 / 3.0)
     assert mu[0, 0, 1] == _nearest_f32_bruteforce((Fraction(2) + Fraction(2) ** -60) / 3)
 
 
-def test_channel_mean_matches_exact_rationals():
+def test_channel_mean_matches_exact_rationals(impl):
     rng = np.random.default_rng(11)
     x = (rng.standard_normal((2, 1, 37, 3)) * np.exp(rng.uniform(-30, 30, (2, 1, 37, 3)))).astype(np.float32)
     b = f32_to_bf16_bits(x)
     vals = O.bf16_to_f64(b)
-    mu = O.channel_mean(b)
+    mu = impl.channel_mean(b)
     for i in range(2):
         for c in range(3):
             ex = sum(Fraction(float(t)) for t in vals[i, 0, :, c]) / 37
@@ -110,15 +121,15 @@ def test_channel_mean_matches_exact_rationals():
 
 # --- quantisation ----------------------------------------------------------
 
-def test_quant_ties_golden():
+def test_quant_ties_golden(impl):
     g = golden("quant_ties.json")
     x = np.array(g["x"], dtype=np.float32).reshape(1, 1, -1, 1)
-    codes, scales = O.quantize_blocks(x, g["block"])
+    codes, scales = impl.quantize_blocks(x, g["block"])
     assert scales[0, 0, 0] == g["scale"]
     assert codes[0, 0, :, 0].tolist() == g["codes"]
 
 
-def test_quant_round_trip_of_representable_blocks():
+def test_quant_round_trip_of_representable_blocks(impl):
     rng = np.random.default_rng(3)
     block, d, nblk = 16, 8, 5
     m = rng.integers(-127, 128, size=(1, 1, nblk * block, d))
@@ -126,15 +137,15 @@ def test_quant_round_trip_of_representable_blocks():
         m[0, 0, r * block, 0] = 127 if r % 2 else -127
     s = 2.0 ** -np.arange(3, 3 + nblk)
     x = (m * np.repeat(s, block)[None, None, :, None]).astype(np.float32)
-    codes, scales = O.quantize_blocks(x, block)
+    codes, scales = impl.quantize_blocks(x, block)
     assert np.array_equal(codes.astype(np.int64), m)
     assert np.array_equal(scales[0, 0], s.astype(np.float32))
 
 
-def test_quant_zero_block_partial_block_and_padding():
+def test_quant_zero_block_partial_block_and_padding(impl):
     x = np.zeros((1, 1, 10, 4), dtype=np.float32)
     x[0, 0, 8:10] = [[1, -2, 3, 0.5], [0, 0, -3, 1]]
-    codes, scales = O.quantize_blocks(x, 4)            # blocks [0,4) [4,8) zero, [8,10) partial
+    codes, scales = impl.quantize_blocks(x, 4)            # blocks [0,4) [4,8) zero, [8,10) partial
     assert codes.shape == (1, 1, 12, 4)
     assert scales[0, 0].tolist() == [0.0, 0.0, np.float32(3.0) / np.float32(127.0)]
     assert not codes[0, 0, :8].any() and not codes[0, 0, 10:].any()
@@ -143,22 +154,22 @@ def test_quant_zero_block_partial_block_and_padding():
 
 # --- mask ------------------------------------------------------------------
 
-def test_topk_counts_golden():
+def test_topk_counts_golden(impl):
     for c in golden("topk_counts.json")["cases"]:
-        assert O.topk_count(c["nblk"], c["frac"]) == c["kc"], c
+        assert impl.topk_count(c["nblk"], c["frac"]) == c["kc"], c
     with pytest.raises(ValueError):
-        O.topk_count(10, 0.0)
+        impl.topk_count(10, 0.0)
     with pytest.raises(ValueError):
-        O.topk_count(10, 1.5)
+        impl.topk_count(10, 1.5)
 
 
-def test_select_topk_bruteforce_over_all_subsets():
+def test_select_topk_bruteforce_over_all_subsets(impl):
     rng = np.random.default_rng(2)
     for trial in range(300):
         n = int(rng.integers(1, 9))
         kc = int(rng.integers(1, n + 1))
         p = rng.integers(0, 4, size=n).astype(np.float64)   # many exact ties
-        idx, _ = O.select_topk(p[None, :], kc)
+        idx, _ = impl.select_topk(p[None, :], kc)
         winners = []
         for sub in itertools.combinations(range(n), kc):
             rest = [j for j in range(n) if j not in sub]
@@ -168,32 +179,32 @@ def test_select_topk_bruteforce_over_all_subsets():
         assert idx[0].tolist() == winners[0]
 
 
-def test_near_tie_flag():
+def test_near_tie_flag(impl):
     p = np.array([[0.5, 0.3, 0.3 * (1 - 1e-12), 0.1], [0.5, 0.3, 0.29, 0.1]])
-    _, tie = O.select_topk(p, 2)
+    _, tie = impl.select_topk(p, 2)
     assert tie.tolist() == [True, False]
 
 
-def test_block_means_closed_form_with_partial_block():
+def test_block_means_closed_form_with_partial_block(impl):
     N, block, d = 10, 4, 3
     x = np.zeros((1, 1, N, d), dtype=np.float32)
     for n in range(N):
         x[0, 0, n] = [n, -2 * n, 1.0]
-    means = O.block_means(bits(x), block)
+    means = impl.block_means(bits(x), block)
     assert means[0, 0].tolist() == [[1.5, -3.0, 1.0], [5.5, -11.0, 1.0], [8.5, -17.0, 1.0]]
 
 
-def test_block_probs_matches_scipy_softmax():
+def test_block_probs_matches_scipy_softmax(impl):
     rng = np.random.default_rng(4)
     qb, kb = rng.standard_normal((2, 3, 7, 16)), rng.standard_normal((2, 3, 7, 16))
     ref = scipy.special.softmax(np.einsum("bhic,bhjc->bhij", qb, kb) / 4.0, axis=-1)
-    assert np.allclose(O.block_probs(qb, kb), ref, rtol=0, atol=1e-15)
+    assert np.allclose(impl.block_probs(qb, kb), ref, rtol=0, atol=1e-15)
 
 
-def test_mask_hand_case():
+def test_mask_hand_case(impl):
     g = golden("linear_hand_case.json")
     q, k = bits(np.array(g["q"])[None, None]), bits(np.array(g["k"])[None, None])
-    m = O.block_mask(q, k, g["block"], g["topk_frac"])
+    m = impl.block_mask(q, k, g["block"], g["topk_frac"])
     assert m["idx"][0, 0].tolist() == g["idx"]
 
 
@@ -226,7 +237,7 @@ def test_linear_states_skip_rows_past_n():
     assert h[1].tolist() == [[16.0, 18.0], [16.0, 18.0]]
 
 
-def test_whole_operator_closed_form_q_k_zero():
+def test_whole_operator_closed_form_q_k_zero(impl):
     """Q = K = 0: every score ties, so the lowest kc key blocks are kept; all
     codes are 0, so P = 1 on every kept key and phi = 1 elsewhere:
     out = mean(V over kept keys) + mean(V over the other keys) . W."""
@@ -236,8 +247,8 @@ def test_whole_operator_closed_form_q_k_zero():
     w = rng.standard_normal((d, d)).astype(np.float32) / 4
     vb, wb = f32_to_bf16_bits(v), f32_to_bf16_bits(w)
     z = np.zeros((B, H, N, d), dtype=np.uint16)
-    res = O.sla_attention(z, z, vb, wb, block, frac)
-    kc = O.topk_count(7, frac)
+    res = impl.sla_attention(z, z, vb, wb, block, frac)
+    kc = impl.topk_count(7, frac)
     V, W = O.bf16_to_f64(vb), O.bf16_to_f64(wb)
     for h in range(H):
         assert (res["mask"]["idx"][0, h] == np.arange(kc)).all()
@@ -247,9 +258,9 @@ def test_whole_operator_closed_form_q_k_zero():
             assert np.allclose(rows, np.broadcast_to(expect, rows.shape), rtol=0, atol=1e-12)
 
 
-def test_all_blocks_critical_means_no_linear_part():
+def test_all_blocks_critical_means_no_linear_part(impl):
     x = make_inputs(1, 1, 96, 16, seed=1)
-    res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 32, 1.0)
+    res = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 32, 1.0)
     for key, ol in res["o_lin"].items():
         assert not ol.any()
         assert np.array_equal(res["out"][key], res["o_sparse"][key])
@@ -264,9 +275,9 @@ def _sdpa64(q, k, v):
 
 
 @pytest.mark.parametrize("N,block", [(256, 64), (200, 64), (130, 32)])
-def test_dense_unquantised_equals_library_attention(N, block):
+def test_dense_unquantised_equals_library_attention(impl, N, block):
     x = make_inputs(1, 2, N, 32, seed=N)
-    res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, 1.0,
+    res = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, 1.0,
                           quant=False, pcast=False)
     Q, K, V = (O.bf16_to_f64(x[t]) for t in ("q", "k", "v"))
     for h in range(2):
@@ -275,17 +286,17 @@ def test_dense_unquantised_equals_library_attention(N, block):
         assert np.max(np.abs(got - ref)) <= 1e-10
 
 
-def test_smoothing_does_not_change_unquantised_output():
+def test_smoothing_does_not_change_unquantised_output(impl):
     x = make_inputs(1, 2, 320, 32, seed=5)
-    a = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.4, quant=False, pcast=False)
-    b = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.4, quant=False, pcast=False,
+    a = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.4, quant=False, pcast=False)
+    b = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.4, quant=False, pcast=False,
                         smooth=False)
     assert np.array_equal(a["mask"]["idx"], b["mask"]["idx"])
     for key in a["out"]:
         assert np.max(np.abs(a["out"][key] - b["out"][key])) <= 1e-12
 
 
-def test_quantised_path_on_losslessly_quantisable_inputs():
+def test_quantised_path_on_losslessly_quantisable_inputs(impl):
     """Blocks of integers times 2**-6 with max |int| = 127 quantise without loss,
     and K rows in +- pairs have channel mean 0, so smoothing is the identity:
     the INT8 path then equals float64 attention up to float32 rounding of S."""
@@ -305,28 +316,28 @@ def test_quantised_path_on_losslessly_quantisable_inputs():
     v = rng.standard_normal((1, 1, N, d)).astype(np.float32)
     qb, kb, vb = bits(qv), bits(kv), f32_to_bf16_bits(v)
     wb = f32_to_bf16_bits(np.eye(d, dtype=np.float32))
-    qz = O.quantize(qb, kb, block)
+    qz = impl.quantize(qb, kb, block)
     assert not qz["mu"].any()
     assert np.array_equal(qz["q_i8"].astype(np.int64), qi)
     assert np.array_equal(qz["k_i8"].astype(np.int64), ki)
-    a = O.sla_attention(qb, kb, vb, wb, block, 0.5, pcast=False)
-    b = O.sla_attention(qb, kb, vb, wb, block, 0.5, pcast=False, quant=False)
+    a = impl.sla_attention(qb, kb, vb, wb, block, 0.5, pcast=False)
+    b = impl.sla_attention(qb, kb, vb, wb, block, 0.5, pcast=False, quant=False)
     for key in a["out"]:
         assert np.max(np.abs(a["o_sparse"][key] - b["o_sparse"][key])) <= 1e-5
 
 
-def test_bf16_cast_of_p_error_bound():
+def test_bf16_cast_of_p_error_bound(impl):
     """Rounding P to bf16 changes each P by at most 2**-9 of itself, so O moves by
     at most 2**-9 * max |V|."""
     x = make_inputs(1, 1, 512, 32, seed=8)
-    a = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.25)
-    b = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.25, pcast=False)
+    a = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.25)
+    b = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.25, pcast=False)
     vmax = np.abs(O.bf16_to_f64(x["v"])).max()
     worst = max(np.abs(a["o_sparse"][k] - b["o_sparse"][k]).max() for k in a["o_sparse"])
     assert 0 < worst <= 2.0 ** -9 * vmax
 
 
-def test_projection_multiplies_on_the_right():
+def test_projection_multiplies_on_the_right(impl):
     """W_proj = identity gives out = O_sparse + O_lin; W_proj = 0 gives O_sparse; a
     permutation matrix permutes the columns of O_lin."""
     x = make_inputs(1, 1, 256, 16, seed=21)
@@ -334,9 +345,9 @@ def test_projection_multiplies_on_the_right():
     eye = f32_to_bf16_bits(np.eye(d, dtype=np.float32))
     zero = np.zeros((d, d), dtype=np.uint16)
     perm = np.roll(np.eye(d, dtype=np.float32), 1, axis=1)          # e_a -> e_{a+1}
-    a = O.sla_attention(x["q"], x["k"], x["v"], eye, 32, 0.25)
-    b = O.sla_attention(x["q"], x["k"], x["v"], zero, 32, 0.25)
-    c = O.sla_attention(x["q"], x["k"], x["v"], f32_to_bf16_bits(perm), 32, 0.25)
+    a = impl.sla_attention(x["q"], x["k"], x["v"], eye, 32, 0.25)
+    b = impl.sla_attention(x["q"], x["k"], x["v"], zero, 32, 0.25)
+    c = impl.sla_attention(x["q"], x["k"], x["v"], f32_to_bf16_bits(perm), 32, 0.25)
     for key in a["out"]:
         assert np.array_equal(a["out"][key], a["o_sparse"][key] + a["o_lin"][key])
         assert np.array_equal(b["out"][key], b["o_sparse"][key])
@@ -344,13 +355,13 @@ def test_projection_multiplies_on_the_right():
                            rtol=0, atol=1e-15)
 
 
-def test_quant_codes_match_exact_rational_division():
+def test_quant_codes_match_exact_rational_division(impl):
     """Each code is the float32 nearest to x / s (exact rational arithmetic),
     rounded half to even; s is the float32 nearest to max|x| / 127."""
     rng = np.random.default_rng(17)
     x = (rng.standard_normal((1, 1, 64, 32)) * 3).astype(np.float32)
     x = O.bf16_to_f32(f32_to_bf16_bits(x))
-    codes, scales = O.quantize_blocks(x[:, :, :, :], 16)
+    codes, scales = impl.quantize_blocks(x[:, :, :, :], 16)
     for r in range(4):
         blk = x[0, 0, r * 16:(r + 1) * 16]
         m = Fraction(float(np.abs(blk).max()))
@@ -360,3 +371,19 @@ def test_quant_codes_match_exact_rational_division():
             qf = _nearest_f32_bruteforce(Fraction(float(val)) / Fraction(s))
             want = max(-127, min(127, int(np.rint(qf))))
             assert codes[0, 0, r * 16 + n, c] == want
+
+
+def test_linear_hand_case_through_the_whole_operator(impl):
+    """The hand-derived linear branch again, through the whole operator with
+    W_proj = I (every value of the case is exact in bf16)."""
+    g = golden("linear_hand_case.json")
+    q = bits(np.array(g["q"])[None, None])
+    k = bits(np.array(g["k"])[None, None])
+    v = bits(np.array(g["v"])[None, None])
+    w = bits(np.eye(g["d"]))
+    res = impl.sla_attention(q, k, v, w, g["block"], g["topk_frac"])
+    assert res["mask"]["idx"][0, 0].tolist() == g["idx"]
+    e = math.e
+    expect = np.array([[eval(s, {"e": e}) for s in row] for row in g["o_lin_expr"]])
+    got = np.concatenate([res["o_lin"][(0, 0, i)] for i in range(2)])
+    assert np.allclose(got, expect, rtol=1e-14, atol=0)
