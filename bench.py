@@ -4,15 +4,19 @@ and ms per call at the 480P video-DiT shape (B=1, H=12, N=32768, d=128,
 block=128, top-10%), one call of the whole operator per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 480p|720p|dense|sweep0.05|sweep0.10|sweep0.20|sweep0.40|tiny]
+
+--workload picks another of the seeded synthetic workloads (default: the
+480P headline); the JSON line's metric string names the workload's shape.
 
 One process per GPU (torchrun for N > 1).  Every (batch, head) problem is
 independent, so each rank runs its own full-size problem with no collective
 on the data path ("scaling": "weak"); ranks only meet at the timing barriers
 and the max-over-ranks of the elapsed time.  Rank 0 prints one JSON line.
 
---impl reference times the CPU oracle (oracle/, the plain statement of the
-method, run as it stands on the host cores) on a bounded sample of the same
-workload: one query block of a head per step.
+--impl reference times the CPU oracle (the plain C++ statement of the method
+under oracle/, run as it stands on the host cores) on a bounded sample of the
+same workload: one whole head per step.
 """
 
 from __future__ import annotations
@@ -44,21 +48,57 @@ ATTN_SOURCE = os.path.join(ROOT, "int8_block_sparse_b200", "csrc", "k_attn.cuh")
 
 # ---------------------------------------------------------------- work accounting
 
+def metric_for(w) -> str:
+    """The headline metric string, or the same wording for another workload's shape."""
+    if w.name == WORKLOAD:
+        return METRIC
+    pct = f"{w.topk_frac * 100:g}%"
+    return (f"effective sparse-attn TOPS & ms/call, B={w.B} N={w.N} H={w.H} d={w.d} top-{pct}, 1 B200 "
+            f"({w.name} workload)")
+
+
 def dense_equivalent_ops(B, H, N, d):
     """4 * B * H * N^2 * d: QK^T and PV of dense attention, 2 ops per MAC each."""
     return 4.0 * B * H * N * N * d
 
 
-def critical_ops(B, H, N, d, block, kc):
-    """Ops of the critical-block work: int8 QK^T and bf16 PV, 2*rows*keys*d each.
+def critical_ops(idx, N, d, block):
+    """Ops of the critical-block work counted from the block lists idx
+    [B, H, nblk, kc]: int8 QK^T and bf16 PV, 2 * rows_i * keys_j * d each for
+    every kept (query block i, key block j), with the valid rows and keys of
+    a partial last block."""
+    import numpy as np
 
-    With a full last block (N a multiple of block) every selected pair is
-    block x block; otherwise the count is an upper bound by at most one
-    partial block per row (the 480P workload has no partial block)."""
-    nblk = (N + block - 1) // block
-    pairs = B * H * nblk * kc
-    per = 2.0 * block * block * d
-    return pairs * per, pairs * per
+    nblk = idx.shape[-2]
+    sizes = np.minimum(block, N - np.arange(nblk) * block).astype(np.float64)
+    keys = sizes[idx.astype(np.int64)].sum(axis=-1)          # [B, H, nblk]
+    ops = float((2.0 * d * sizes[None, None, :] * keys).sum())
+    return ops, ops
+
+
+def algorithmic_bytes(B, H, N, d, nblk, kc):
+    """Bytes a call must move at least: q, k, v in (bf16), out (bf16), the
+    INT8 codes written and read once, and the float32 linear states written
+    and read once (none when every block is kept)."""
+    b = B * H * N * d * (3 * 2 + 2 + 2 * 1 * 2)
+    if kc < nblk:
+        b += 2 * B * H * nblk * (d * d + d) * 4
+    return float(b)
+
+
+def call_roofline(qk_ops, pv_flops, bytes_alg, ms, peaks):
+    """Roofline of the whole call: the slower of the critical-block work at the
+    tensor peaks and the algorithmic bytes at the HBM peak, over the measured
+    time per call."""
+    bf16 = float(peaks["bf16_tflops"]) if peaks else FALLBACK_BF16_TFLOPS
+    hbm = float(peaks["hbm_gbs"]) if peaks else FALLBACK_HBM_GBS
+    t_tensor = qk_ops / (2.0 * bf16 * 1e12) + pv_flops / (bf16 * 1e12)
+    t_hbm = bytes_alg / (hbm * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    return {"bound": "tensor" if t_tensor >= t_hbm else "hbm", "t_roof_ms": round(t_roof * 1e3, 4),
+            "t_tensor_ms": round(t_tensor * 1e3, 4), "t_hbm_ms": round(t_hbm * 1e3, 4),
+            "bytes_alg": bytes_alg, "frac": round(t_roof * 1e3 / ms, 4),
+            "peaks": "measured (MEASURED_PEAKS.json)" if peaks else "fallback"}
 
 
 def attn_roofline(qk_ops, pv_flops, peaks):
@@ -217,35 +257,46 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle sample
 
-def oracle_sample(w, nh: int):
-    """Time the CPU oracle on every query block of the first nh heads of the
-    workload (quantisation, mask, linear states and outputs).  Returns
-    (seconds, ops, sample)."""
-    import numpy as np
+def oracle_sample(w, x, max_heads: int, budget_s: float):
+    """Time the CPU oracle on every query block of whole heads of the workload
+    (their quantisation, mask, linear states and outputs), head 0 first, until
+    max_heads heads or about budget_s seconds.  Returns (seconds, ops, sample)."""
+    from oracle import cpp_oracle as O
 
-    import oracle as O
-    from synth import make_workload
-
-    nh = max(1, min(nh, w.H))
-    x = make_workload(w, heads=list(range(nh)))
-    items = [(0, h, i) for h in range(nh) for i in range(w.nblk)]
-    t0 = time.perf_counter()
-    O.sla_attention(x["q"], x["k"], x["v"], x["proj"], w.block, w.topk_frac, items=items)
-    dt = time.perf_counter() - t0
+    dt, nh = 0.0, 0
+    for h in range(min(max_heads, w.H)):
+        xs = {k: (v[:1, h:h + 1] if v.ndim == 4 else v) for k, v in x.items()}
+        t0 = time.perf_counter()
+        O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, w.topk_frac)
+        dt += time.perf_counter() - t0
+        nh += 1
+        if dt >= budget_s:
+            break
     ops = nh * 4.0 * w.N * w.N * w.d   # dense-equivalent ops of those heads
-    return dt, ops, (f"CPU oracle on heads 0..{nh - 1} of {w.name} (all {w.nblk} query blocks of "
-                     f"{w.block} rows each, with their quantisation, mask and linear states); "
+    return dt, ops, (f"CPU oracle on heads 0..{nh - 1} of batch 0 of {w.name} (all {w.nblk} query blocks "
+                     f"of {w.block} rows each, with their quantisation, mask and linear states); "
                      f"value = dense-equivalent ops of those heads / wall time")
 
 
-def blas_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
+def mask_parity(w, x, gidx):
+    """The GPU's block lists against the oracle's over the whole workload:
+    rows, rows the oracle marks as near ties, rows whose lists differ, and
+    rows that differ without being near ties (must be 0)."""
+    import numpy as np
 
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return int(max(n)) if n else 1
-    except Exception:
-        return len(os.sched_getaffinity(0))
+    from oracle import cpp_oracle as O
+
+    ref = O.block_mask(x["q"], x["k"], w.block, w.topk_frac)
+    diff = np.any(gidx != ref["idx"], axis=-1)
+    return {"rows": int(diff.size), "near_tie_rows": int(ref["near_tie"].sum()),
+            "differing_rows": int(diff.sum()), "differing_off_near_tie": int((diff & ~ref["near_tie"]).sum())}
+
+
+def oracle_threads() -> int:
+    """Worker threads of the C++ CPU oracle (every core this process may use)."""
+    from oracle import cpp_oracle
+
+    return cpp_oracle.threads()
 
 
 # ---------------------------------------------------------------- arms
@@ -262,16 +313,16 @@ def run_ours(args, dist):
     S.lib()
     dev = torch.device("cuda", dist.local)
     torch.cuda.set_device(dev)
-    w = CONFIGS[WORKLOAD]
+    w = CONFIGS[args.workload]
     if args.heads:
         import dataclasses
 
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}-first{args.heads}heads")
-        x = make_workload(CONFIGS[WORKLOAD], heads=list(range(args.heads)))
+        x = make_workload(CONFIGS[args.workload], heads=list(range(args.heads)))
     else:
         x = make_workload(w)
     t = {k: torch.from_numpy(x[k].view(np.int16)).view(torch.bfloat16).to(dev) for k in ("q", "k", "v", "proj")}
-    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, device=dev)
+    out = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -309,7 +360,8 @@ def run_ours(args, dist):
     ops = dense_equivalent_ops(w.B, w.H, w.N, w.d)
     value = weak_scaling_value(ops, dist.world, ms / 1e3)
     kc = S.topk_count(w.N, w.block, w.topk_frac)
-    qk, pv = critical_ops(w.B, w.H, w.N, w.d, w.block, kc)
+    gidx = S.sla_mask(t["q"], t["k"], w.block, w.topk_frac).cpu().numpy()
+    qk, pv = critical_ops(gidx, w.N, w.d, w.block)
     peaks = load_peaks()
     peak, peak_src = attn_roofline(qk, pv, peaks)
     attn_ms, attn_n = prof["attn"]
@@ -317,7 +369,7 @@ def run_ours(args, dist):
     achieved = (qk + pv) / (attn_avg / 1e3) / 1e12
     roof = {"bound": "tensor", "kernel": "k_attn<128,128> (critical-block attention)",
             "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+            "frac": round(achieved / peak, 4), "traffic": profiled_traffic() if w.name == WORKLOAD else None,
             "peak_source": peak_src, "ops_per_launch": qk + pv,
             "kernel_ms": round(attn_avg, 4)}
     launches = int(sum(n for _, n in prof.values()))
@@ -328,19 +380,24 @@ def run_ours(args, dist):
         e2e = run_e2e(S, t, w, args, dist)
 
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": dist.world,
+        "metric": metric_for(w), "value": round(value, 2), "unit": UNIT, "n_gpus": dist.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8,bf16 (f32 accumulate)",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8,bf16 (f32 accumulate; bf16 out)",
         "data": "synthetic (seeded field-plus-noise, see synth/workloads.py)",
         "config": {"workload": w.describe(), "kc": kc,
                    "parallelism": f"replicas x{dist.world} (independent problems per rank)",
                    "l2": "inputs larger than L2 (q, k, v: 302 MB; ~1 GB moved per call), no flush"},
-        "roofline": roof, "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "e2e": e2e,
+        "roofline": roof,
+        "roofline_call": call_roofline(qk, pv, algorithmic_bytes(w.B, w.H, w.N, w.d, w.nblk, kc), ms, peaks),
+        "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "e2e": e2e,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
-        dt, cops, sample = oracle_sample(w, args.cpu_heads)
-        line["cpu_baseline"] = {"value": round(cops / dt / 1e12, 6), "unit": UNIT, "cores": blas_threads(),
+        dt, cops, sample = oracle_sample(w, x, args.cpu_heads, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(cops / dt / 1e12, 6), "unit": UNIT, "cores": oracle_threads(),
                                 "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+        # near ties of the block mask (CPU oracle leg): every differing row must be one
+        line["mask_parity"] = mask_parity(w, x, gidx)
+        line["near_tie_rows"] = line["mask_parity"]["near_tie_rows"]
     return line
 
 
@@ -351,7 +408,7 @@ def run_e2e(S, t, w, args, dist):
     import torch
 
     host = {k: v.cpu().pin_memory() for k, v in t.items()}
-    hout = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32).pin_memory()
+    hout = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16).pin_memory()
     S.sla_attn_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block, topk_frac=w.topk_frac)
     n = max(1, min(args.steps, args.e2e_steps))
     dist.barrier()
@@ -369,55 +426,42 @@ def run_e2e(S, t, w, args, dist):
 
 
 def run_reference(args, dist):
-    """The CPU oracle as the reference arm: one query block per step."""
-    import numpy as np
-
-    import oracle as O
+    """The CPU oracle as the reference arm: the plain C++ oracle, as it stands,
+    on the host cores; each step is the whole operator on one head of the
+    workload (every query block of it, with its quantisation, mask and linear
+    states), the heads taken in turn."""
+    from oracle import cpp_oracle as O
     from synth import CONFIGS, make_workload
 
-    w = CONFIGS[WORKLOAD]
+    w = CONFIGS[args.workload]
     if dist.rank != 0:
         return None
-    x = make_workload(w, heads=[0])
-    # per-head preparation (quantisation, mask, linear states) is timed once
-    # and amortised over the workload's query blocks in the reported value
-    t0 = time.perf_counter()
-    res0 = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], w.block, w.topk_frac, items=[(0, 0, 0)])
-    prep = time.perf_counter() - t0
-    rng = np.random.default_rng(0)
-    blocks = rng.integers(0, w.nblk, size=args.warmup + args.steps)
-    q64 = O.bf16_to_f64(x["q"][0, 0])
-    k64 = O.bf16_to_f64(x["k"][0, 0])
-    v64 = O.bf16_to_f64(x["v"][0, 0])
-    w64 = O.bf16_to_f64(x["proj"])
-    hst, zst = O.linear_states(k64, v64, w.block)
-    qz, mask = res0["quant"], res0["mask"]
+    n = args.warmup + args.steps
+    heads = sorted({s % w.H for s in range(n)})
+    x = make_workload(w, heads=heads)
+    pos = {h: t for t, h in enumerate(heads)}
 
-    def step(i):
-        crit = mask["idx"][0, 0, i]
-        lo, hi = i * w.block, min(w.N, (i + 1) * w.block)
-        os_ = O.critical_rows(qz["q_i8"][0, 0, lo:lo + w.block], qz["q_scale"][0, 0, i], qz["k_i8"][0, 0],
-                              qz["k_scale"][0, 0], v64, crit, w.N, w.block)[:hi - lo]
-        return os_ + np.matmul(O.linear_rows(q64[lo:hi], hst, zst, crit), w64)
+    def step(s):
+        h = pos[s % w.H]
+        xs = {k: (v[:1, h:h + 1] if v.ndim == 4 else v) for k, v in x.items()}
+        O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, w.topk_frac)
 
-    for i in blocks[:args.warmup]:
-        step(int(i))
+    for s_ in range(args.warmup):
+        step(s_)
     t0 = time.perf_counter()
-    for i in blocks[args.warmup:]:
-        step(int(i))
-    per = (time.perf_counter() - t0) / max(args.steps, 1)
-    per_block = per + prep / w.nblk
-    ops = 4.0 * w.block * w.N * w.d
-    value = ops / per_block / 1e12
-    ms_call = per_block * w.nblk * w.B * w.H * 1e3
-    sample = (f"CPU oracle, {args.steps} steps of one query block ({w.block} rows) of head 0 of {w.name}; "
-              f"per-head preparation {prep:.2f} s amortised over its {w.nblk} query blocks")
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": dist.world,
+    for s_ in range(args.warmup, n):
+        step(s_)
+    per_head = (time.perf_counter() - t0) / max(args.steps, 1)
+    value = 4.0 * w.N * w.N * w.d / per_head / 1e12
+    ms_call = per_head * w.B * w.H * 1e3
+    sample = (f"C++ CPU oracle, {args.steps} steps of one whole head of batch 0 of {w.name} (all {w.nblk} "
+              f"query blocks with the head's quantisation, mask and linear states), heads in turn")
+    return {"impl": "reference", "metric": metric_for(w), "value": round(value, 6), "unit": UNIT, "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_call, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (int8 codes)",
             "data": "synthetic (seeded field-plus-noise, see synth/workloads.py)",
             "config": {"workload": w.describe(), "note": "ms_per_step = projected time of one full call"},
-            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -431,8 +475,12 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["tiny", "480p", "720p", "dense", "sweep0.05", "sweep0.10", "sweep0.20", "sweep0.40"])
     ap.add_argument("--cpu-heads", type=int, default=6,
-                    help="heads of the workload the CPU oracle baseline runs in full (about 10-20 s)")
+                    help="most heads of the workload the CPU oracle baseline runs in full")
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds after which the CPU oracle baseline stops adding heads")
     ap.add_argument("--heads", type=int, default=0,
                     help="keep only the first H heads (a smaller case for profiling; not the headline)")
     args = ap.parse_args(argv)

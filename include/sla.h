@@ -12,7 +12,7 @@
  *        (--attention_type sagesla, --sla_topk 0.1 = keep 10%).
  * The pages give no formulas; the exact semantics implemented here are:
  *   1. mu = per-channel mean of K over the N tokens (exact sum, rounded once to
- *      float32); K_s = float32(K) - mu.  ([P1] 三(一) item 1, "outlier smoothing")
+ *      float32, for every finite input); K_s = float32(K) - mu.  ([P1] 三(一) item 1, "outlier smoothing")
  *   2. Q and K_s are quantised to INT8 per block of `block` tokens x d channels:
  *      s = max|x| / 127 (float32), code = clamp(round_half_even(x / s), +-127).
  *      ([P1] 三(一) item 2)
@@ -28,13 +28,13 @@
  *      O_lin = phi(q) (sum h_j) / (phi(q) . sum z_j) with per-key-block states
  *      h_j = sum phi(k) v^T, z_j = sum phi(k) of the raw K; none when every
  *      block is kept.  ([P1] 三(二) item 2)
- *   6. out = O_sparse + O_lin . W_proj in float32 (the accumulation
- *      precision; the pages name no output rounding).  ([P1] 三(二) item 2,
+ *   6. out = O_sparse + O_lin . W_proj, formed in float32 and stored as bf16
+ *      (round to nearest even; float32 on request).  ([P1] 三(二) item 2,
  *      "linear projection")
  *
  * Conventions for every entry point:
  *   - Tensors are row-major.  q, k, v: bf16 [B, H, N, d] (d innermost); out:
- *     float32 [B, H, N, d].
+ *     bf16 [B, H, N, d] (float32 through sla_attn_ex).
  *     proj (W_proj): bf16 [d, d], used as O_lin . proj (row vectors).
  *   - All tensor pointers are DEVICE pointers except where an entry point says
  *     HOST.  They must be 16-byte aligned.  The caller owns all memory; the
@@ -49,8 +49,12 @@
  *     returns an error code and touches no memory.  Faults inside the kernels
  *     surface at the caller's next synchronisation or through
  *     sla_get_error().
- *   - Thread safety: calls are re-entrant; concurrent calls on different
- *     streams are independent.
+ *   - Thread safety: calls are re-entrant, and concurrent calls on different
+ *     streams compute independently, with two exceptions: sla_mask_noalloc
+ *     calls share one scratch buffer (see there), and the device error word
+ *     that sla_get_error() reads is one word per device, not per stream, so a
+ *     failure recorded by one stream's kernels is reported to (and cleared by)
+ *     whichever caller reads it first.
  */
 #ifndef SLA_H_
 #define SLA_H_
@@ -69,10 +73,6 @@ typedef enum {
   SLA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                   */
   SLA_ERR_OOM = 4,          /* temporary device memory could not be obtained       */
   SLA_ERR_TIMEOUT = 5,      /* a kernel's bounded wait gave up (sla_get_error)     */
-  SLA_ERR_INEXACT_MEAN = 6, /* the K channel mean could not be proven exact: some
-                               channel's values span more exponents than a float64
-                               sum holds exactly (sla_get_error; results are still
-                               written)                                            */
   SLA_ERR_SCRATCH_LIMIT = 7, /* sla_mask_noalloc: the problem needs more scratch than
                                its fixed device buffer holds                       */
   SLA_ERR_SMEM_LAYOUT = 8   /* a kernel's dynamic shared memory did not start on a
@@ -120,9 +120,12 @@ int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, in
  * (for example B*H = 12, nblk = 256, d = 128 fits; B*H = 40, nblk = 591
  * does not); larger ones return SLA_ERR_SCRATCH_LIMIT before any work is
  * enqueued.
- *   The first call on a device looks up the buffer's device address (once
- * per device, with that device current); make that first call before any
- * stream capture.  No allocation happens on that or any later call (keep
+ *   The first call on a device looks up the buffer's device address and
+ * loads every kernel this entry point can launch (once per device, with that
+ * device current; with CUDA's lazy module loading that is where the buffer
+ * and the kernels' code are placed on the device); make that first call
+ * during start-up, before the caller stops allowing allocation and before any
+ * stream capture.  No later call allocates, whatever its shape (keep
  * sla_profile_enable off, its default: profiling creates CUDA events).
  *   All calls on a device share the one buffer and it keeps the last call's
  * contents; every scratch element is written before it is read, so nothing
@@ -134,25 +137,36 @@ int sla_mask_noalloc(const void* q, const void* k, int32_t* blk_idx, uint8_t* bi
 /* The whole operator, steps 1-6 ([P1] 三(二) 3, SageSLA).
  *   q, k, v : in,  bf16 [B,H,N,d]
  *   proj    : in,  bf16 [d,d]
- *   out     : out, float [B,H,N,d], fully overwritten */
+ *   out     : out, bf16 [B,H,N,d], fully overwritten (float32 result rounded
+ *             to nearest even) */
 int sla_attn(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N,
              int d, int block, float topk_frac, void* stream);
 
-/* sla_attn that also returns the critical-block part before the projection
- * and the sum (for inspection and tests):
- *   o_sparse : out, float [B,H,N,d] = O_sparse of step 4, or NULL. */
-int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, void* out, float* o_sparse,
-                int B, int H, int N, int d, int block, float topk_frac, void* stream);
+/* Output element types of sla_attn_ex. */
+#define SLA_OUT_BF16 0
+#define SLA_OUT_F32 1
+
+/* sla_attn with a choice of output type and, for inspection and tests, the
+ * two parts of step 6 on their own:
+ *   out       : out, [B,H,N,d] of type out_dtype (SLA_OUT_BF16 or SLA_OUT_F32)
+ *   o_sparse  : out, float [B,H,N,d] = O_sparse of step 4, or NULL
+ *   o_lin     : out, float [B,H,N,d] = O_lin . W_proj of steps 5-6 (zero when
+ *               every block is kept), or NULL
+ * Each part asked for costs one more pass of the attention kernel. */
+int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, void* out, int out_dtype,
+                float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, float topk_frac,
+                void* stream);
 
 /* sla_attn on HOST buffers (pageable or pinned): copies q, k, v, proj to the
  * device, runs the operator on an internal stream of the current device,
- * copies out back and returns when it is in host memory. */
+ * copies out (bf16) back and returns when it is in host memory. */
 int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
                   int N, int d, int block, float topk_frac);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
- * current device: SLA_ERR_TIMEOUT if a kernel's bounded wait gave up,
- * SLA_ERR_INEXACT_MEAN if a channel mean could not be proven exact,
+ * current device.  The word is shared by every stream of the device: a code
+ * recorded by kernels on another stream is reported here as well, and cleared.
+ * Returns SLA_ERR_TIMEOUT if a kernel's bounded wait gave up,
  * SLA_ERR_SMEM_LAYOUT if a kernel could not place its shared-memory tiles,
  * SLA_ERR_CUDA if the synchronisation itself failed, else SLA_OK. */
 int sla_get_error(void* stream);
@@ -163,10 +177,9 @@ typedef enum {
   SLA_K_MEAN = 1,    /* per-channel mean of K                        */
   SLA_K_QUANT = 2,   /* smoothing + INT8 quantisation (+ Q block sums) */
   SLA_K_MASK = 3,    /* pooled scores + top-k                        */
-  SLA_K_ATTN = 4,    /* critical-block attention                     */
+  SLA_K_ATTN = 4,    /* critical-block attention + linear part       */
   SLA_K_LINGEMM = 5, /* sums of the non-selected states              */
-  SLA_K_LINOUT = 6,  /* linear branch, projection, add               */
-  SLA_K_COUNT = 7
+  SLA_K_COUNT = 6
 } sla_kernel_kind;
 
 /* Measurement support (no counterpart on the pages).  While enabled, every

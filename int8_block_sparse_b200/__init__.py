@@ -17,14 +17,16 @@ LIB_PATH = os.path.join(HERE, "libsla.so")
 
 SLA_OK = 0
 STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "SLA_ERR_CUDA",
-                4: "SLA_ERR_OOM", 5: "SLA_ERR_TIMEOUT", 6: "SLA_ERR_INEXACT_MEAN", 7: "SLA_ERR_SCRATCH_LIMIT",
+                4: "SLA_ERR_OOM", 5: "SLA_ERR_TIMEOUT", 7: "SLA_ERR_SCRATCH_LIMIT",
                 8: "SLA_ERR_SMEM_LAYOUT"}
 
 EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
            "sla_get_error", "sla_status_string", "sla_profile_enable", "sla_profile_read",
            "sla_mask_noalloc", "sla_selftest_wait_timeout")
 
-KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm", "linout")
+KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm")
+
+OUT_BF16, OUT_F32 = 0, 1
 
 
 class SlaError(RuntimeError):
@@ -50,7 +52,7 @@ def lib() -> ctypes.CDLL:
         L.sla_mask_noalloc.argtypes = [vp] * 4 + [i] * 5 + [f, vp]
         L.sla_selftest_wait_timeout.argtypes = [vp]
         L.sla_attn.argtypes = [vp] * 5 + [i] * 5 + [f, vp]
-        L.sla_attn_ex.argtypes = [vp] * 6 + [i] * 5 + [f, vp]
+        L.sla_attn_ex.argtypes = [vp] * 5 + [i] + [vp] * 2 + [i] * 5 + [f, vp]
         L.sla_attn_host.argtypes = [vp] * 5 + [i] * 5 + [f]
         L.sla_get_error.argtypes = [vp]
         L.sla_status_string.argtypes = [i]
@@ -101,7 +103,15 @@ def nblk(N: int, block: int) -> int:
     return (N + block - 1) // block
 
 
-def sla_quant(q, k, block: int, stream=None):
+def _after(check: bool, stream, where: str) -> None:
+    """With check=True, wait for the call and raise on a device-side status
+    (a timed-out wait, a shared-memory layout failure); without it, such a
+    status is only seen by a later get_error()."""
+    if check:
+        _check(get_error(stream), where)
+
+
+def sla_quant(q, k, block: int, stream=None, check: bool = False):
     """Smoothing + INT8 quantisation.  Returns (q_i8, k_i8, q_scale, k_scale, k_mean)."""
     import torch
 
@@ -115,10 +125,11 @@ def sla_quant(q, k, block: int, stream=None):
     mu = torch.empty((B, H, d), dtype=torch.float32, device=dev)
     _check(lib().sla_quant(_ptr(q), _ptr(k), _ptr(qi8), _ptr(ki8), _ptr(sq), _ptr(sk), _ptr(mu),
                            B, H, N, d, block, _stream(stream)), "sla_quant")
+    _after(check, stream, "sla_quant")
     return qi8, ki8, sq, sk, mu
 
 
-def sla_mask(q, k, block: int, topk_frac: float, bitmap: bool = False, stream=None):
+def sla_mask(q, k, block: int, topk_frac: float, bitmap: bool = False, stream=None, check: bool = False):
     """Pooled top-k block mask.  Returns idx [B,H,nblk,kc] int32 (and the uint8 bitmap)."""
     import torch
 
@@ -129,29 +140,38 @@ def sla_mask(q, k, block: int, topk_frac: float, bitmap: bool = False, stream=No
     bm = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=q.device) if bitmap else None
     _check(lib().sla_mask(_ptr(q), _ptr(k), _ptr(idx), _ptr(bm), B, H, N, d, block, float(topk_frac),
                           _stream(stream)), "sla_mask")
+    _after(check, stream, "sla_mask")
     return (idx, bm) if bitmap else idx
 
 
-def sla_attn(q, k, v, proj, block: int = 128, topk_frac: float = 0.1, out=None, o_sparse=None,
-             stream=None):
-    """SageSLA attention; q, k, v bf16 [B,H,N,d], proj bf16 [d,d] on the GPU.  Returns out (float32)."""
+def sla_attn(q, k, v, proj, block: int = 128, topk_frac: float = 0.1, out=None, out_dtype=None,
+             o_sparse=None, o_lin=None, stream=None, check: bool = False):
+    """SageSLA attention; q, k, v bf16 [B,H,N,d], proj bf16 [d,d] on the GPU.
+
+    Returns out [B,H,N,d], bf16 by default (out_dtype=torch.float32, or a
+    float32 `out`, for the unrounded result).  o_sparse / o_lin (float32,
+    optional) receive the two parts, O_sparse and O_lin . W_proj."""
     import torch
 
     B, H, N, d = _shape(q)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device)
-    if o_sparse is None:
+        out = torch.empty((B, H, N, d), dtype=out_dtype or torch.bfloat16, device=q.device)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bf16 or float32")
+    if out.dtype == torch.bfloat16 and o_sparse is None and o_lin is None:
         rc = lib().sla_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
                             float(topk_frac), _stream(stream))
     else:
-        rc = lib().sla_attn_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), _ptr(o_sparse), B, H, N, d,
-                               block, float(topk_frac), _stream(stream))
+        kind = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+        rc = lib().sla_attn_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), kind, _ptr(o_sparse),
+                               _ptr(o_lin), B, H, N, d, block, float(topk_frac), _stream(stream))
     _check(rc, "sla_attn")
+    _after(check, stream, "sla_attn")
     return out
 
 
 def sla_attn_host(q, k, v, proj, out, block: int = 128, topk_frac: float = 0.1) -> None:
-    """SageSLA attention on host (CPU) tensors (out: float32); copies in and out inside the call."""
+    """SageSLA attention on host (CPU) tensors (out: bf16); copies in and out inside the call."""
     B, H, N, d = _shape(q)
     _check(lib().sla_attn_host(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
                                float(topk_frac)), "sla_attn_host")

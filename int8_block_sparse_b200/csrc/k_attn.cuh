@@ -1,21 +1,30 @@
-// K4: critical-block attention on the 5th-generation tensor cores.
+// K4: critical-block attention plus the linear part, on the 5th-generation
+// tensor cores.
 //
 // "Turbo Diffusion：秒级生成与高清保真的视频扩散技术突破", section 三(一) item 3
-// (attention re-tiled to 128x128 tensor-core tiles with a parallel softmax) and
+// (attention re-tiled to 128x128 tensor-core tiles with a parallel softmax),
 // section 三(二) item 3 (SageSLA: after the block selection, INT8 computation
-// on the selected blocks).  For query block i of head (b, h) and each selected
-// key block j (ascending):
+// on the selected blocks) and item 2 (the rest through a linear branch and a
+// linear projection).  For query block i of head (b, h) and each selected key
+// block j (ascending):
 //     S = int32(Qi8_i . Ki8_j^T) * sq_i * sk_j / sqrt(D)   (tcgen05 kind::i8)
 //     online softmax in float32 (exp2 domain), P rounded to bf16
 //     O += P . V_j                                        (tcgen05 kind::f16)
-// and finally O_sparse = O / l, l being the sum of the unrounded P.
+// then the linear part of the non-selected blocks, with W_proj folded into the
+// states (G'_i = sum_{j not selected} h_j W_proj, g_i = sum z_j):
+//     O += A . G'_i,  A = bf16(phi(q) * l / den),  den = phi(q) . g_i
+// (one more kind::f16 product, A taken from TMEM like P), so that
+//     out = O / l = O_sparse + phi(q) G'_i / den,
+// l being the sum of the unrounded P; out is written as bf16 (round to nearest
+// even) or float32.  Either part can be switched off (p.sparse, p.lin): with
+// the linear part alone l = 1.
 //
 // One persistent CTA per SM runs two independent pipelines ("tiles"), each
 // working on its own sequence of (head, query block) items:
 //   warp 0 / 2   TMA producers of tile 0 / 1: lane 0 loads Q and K, lane 1 V
-//                (two-stage rings; a K stage is released when its block's QK^T
-//                products finish, a V stage when its PV products finish, so
-//                the next K tile is not held up by the PV of the previous one)
+//                and G'_i (two-stage rings; G'_i goes through the V ring as
+//                one more block; a K stage is released when its block's QK^T
+//                products finish, a V stage when its PV products finish)
 //   warp 1 / 3   tcgen05.mma issuer of tile 0 / 1
 //   warps 4-7    softmax + epilogue of tile 0 (thread = query row = TMEM lane)
 //   warps 8-11   softmax + epilogue of tile 1
@@ -25,7 +34,9 @@
 // S) and O in [256u+128, 256u+128+D).  With two S buffers the QK^T of the next
 // half is already queued on the tensor core while the softmax of this half
 // runs.  The tensor core executes one CTA's MMAs in issue order, so a QK^T
-// issued after a PV may overwrite the S buffer that PV reads P from.
+// issued after a PV may overwrite the S buffer that PV reads P from.  A (D/2
+// columns) goes to the S buffer the next item's first QK^T will use, after the
+// PV that last read it has finished.
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
@@ -33,12 +44,17 @@
 namespace sla {
 
 struct AttnParams {
-  const int32_t* idx;   // [BH][NB][kc]
-  const float* sq;      // [BH][NB]
-  const float* sk;      // [BH][NB]
-  float* o;             // [BH][N][D] float32: O_sparse
+  const int32_t* idx;          // [BH][NB][kc]
+  const float* sq;             // [BH][NB]
+  const float* sk;             // [BH][NB]
+  const __nv_bfloat16* q;      // [BH][N][D] raw queries (phi(q) of the linear part)
+  const float* zrest;          // [BH][NB][D] g_i: z sums over the non-selected blocks
+  void* out;                   // [BH][N][D], bf16 or float32
   int N, NB, NP, kc, items;
-  float qk_scale;       // log2(e) / sqrt(D)
+  int sparse;                  // the selected blocks (softmax attention) take part
+  int lin;                     // the linear part is added
+  int out_f32;                 // float32 output (else bf16)
+  float qk_scale;              // log2(e) / sqrt(D)
 };
 
 template <int D, int BLK>
@@ -64,14 +80,26 @@ struct AttnCfg {
   static constexpr uint32_t KSBO = (D == 128) ? 1024u : 512u;
   static constexpr uint32_t K_HALF_BYTES = HB * D;          // 64 rows of K (int8)
   static constexpr uint32_t V_HALF_BYTES = HB * 128;        // 64 rows of one 64-channel V atom
+  // G'_i (D x D bf16, rows = the K dimension of A . G'_i) passes through the V
+  // ring in LC chunks of LROWS rows, laid out like V blocks
+  static constexpr int LROWS = D < BLK ? D : BLK;
+  static constexpr int LC = D / LROWS;
+  static constexpr int G_CHUNK_BYTES = LROWS * D * 2;
+  static_assert(G_CHUNK_BYTES <= V_BYTES, "a G' chunk fits in a V stage");
 };
 
 struct TileBars {
   uint64_t q_full, q_empty, o_full, o_free;
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t mma_drain, pad;   // end of the MMA issuer: every MMA it issued has finished
+  uint64_t mma_drain;   // end of the MMA issuer: every MMA it issued has finished
+  uint64_t a_full;      // A of the linear part is in TMEM
 };
+
+// The running row maximum is raised (and O, l rescaled) only when a new
+// maximum exceeds it by more than this many powers of two; until then P may
+// reach 2^kRescaleLog2, far inside the range of bf16 P and float32 sums.
+constexpr float kRescaleLog2 = 16.f;
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -79,10 +107,40 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// phi = elu + 1 of a bf16 value (raw bits): x + 1 for x > 0, else e^x.
+__device__ __forceinline__ float phi_bf16(uint16_t bits) {
+  const float x = __uint_as_float(uint32_t(bits) << 16);
+  return x > 0.f ? x + 1.f : ex2_approx(x * 1.4426950408889634f);
+}
+
+// den = phi(q) . g for one query row (zero for a row past the block or N).
+template <int D>
+__device__ __forceinline__ float linear_den(const __nv_bfloat16* qrow, const float* g, bool valid) {
+  float d0 = 0.f, d1 = 0.f;
+  if (valid) {
+#pragma unroll 4
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(qrow) + c8);
+      const float4 g0 = __ldg(reinterpret_cast<const float4*>(g) + 2 * c8);
+      const float4 g1 = __ldg(reinterpret_cast<const float4*>(g) + 2 * c8 + 1);
+      d0 = fmaf(phi_bf16(uint16_t(raw.x)), g0.x, d0);
+      d1 = fmaf(phi_bf16(uint16_t(raw.x >> 16)), g0.y, d1);
+      d0 = fmaf(phi_bf16(uint16_t(raw.y)), g0.z, d0);
+      d1 = fmaf(phi_bf16(uint16_t(raw.y >> 16)), g0.w, d1);
+      d0 = fmaf(phi_bf16(uint16_t(raw.z)), g1.x, d0);
+      d1 = fmaf(phi_bf16(uint16_t(raw.z >> 16)), g1.y, d1);
+      d0 = fmaf(phi_bf16(uint16_t(raw.w)), g1.z, d0);
+      d1 = fmaf(phi_bf16(uint16_t(raw.w >> 16)), g1.w, d1);
+    }
+  }
+  return d0 + d1;
+}
+
 template <int D, int BLK>
 __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtensorMap tm_q,
                                                  const __grid_constant__ CUtensorMap tm_k,
-                                                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                                                 const __grid_constant__ CUtensorMap tm_v,
+                                                 const __grid_constant__ CUtensorMap tm_g, const AttnParams p) {
   using C = AttnCfg<D, BLK>;
   constexpr int NH = C::NH;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -107,6 +165,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
       mbar_init(&b.o_full, 1);
       mbar_init(&b.o_free, 128);
       mbar_init(&b.mma_drain, 1);
+      mbar_init(&b.a_full, 128);
       for (int s = 0; s < 2; ++s) {
         mbar_init(&b.s_full[s], 1);
         mbar_init(&b.p_full[s], 128);
@@ -132,60 +191,76 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
   const int kc = p.kc;
   const int NB = p.NB;
   const int tiles_total = 2 * gridDim.x;
+  const bool sparse = p.sparse != 0, lin = p.lin != 0;
+  const int H = sparse ? kc * NH : 0;   // halves per item
 
   if (warp < 4) {
     const int u = warp >> 1;
     TileBars& b = bars[u];
     unsigned char* tq = base + u * C::TILE_BYTES;
+    auto k_stage = [&](int s) { return tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES); };
+    auto v_stage = [&](int s) { return tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES) + C::K_BYTES; };
     if ((warp & 1) == 0) {
       // ------------------------------------------------------------ producers
-      // Lane 0 loads Q and the K tiles, lane 1 the V tiles; each walks the
-      // block list on its own, reading the next entry one block ahead.
+      // Lane 0 loads Q and the K tiles, lane 1 the V tiles and G'_i; each walks
+      // the block list on its own, reading the next entry one block ahead.
       if (lane < 2) {
         if (lane == 0) {
           tma_prefetch_desc(&tm_q);
           tma_prefetch_desc(&tm_k);
         } else {
           tma_prefetch_desc(&tm_v);
+          if (lin) tma_prefetch_desc(&tm_g);
         }
-        uint32_t blk_it = 0, item_it = 0;
-        uint32_t nq = 0, nkv = 0;   // loads issued: Q (lane 0), K or V (lane 0 / lane 1)
+        uint32_t item_it = 0, nq = 0, nl = 0;   // nl: K loads (lane 0) or V-ring loads (lane 1)
         bool ok = true;
         for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
           const int bh = item / NB, i = item % NB;
-          if (lane == 0) {
-            if (!(ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag))) break;
-            mbar_expect_tx(&b.q_full, C::Q_BYTES);
-            tma_load_2d(tq, &tm_q, &b.q_full, 0, bh * p.NP + i * BLK);
-            ++nq;
-          }
-          const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
-          int jn = __ldg(lst);
-          for (int t = 0; t < kc; ++t, ++blk_it) {
-            const int j = jn;
-            if (t + 1 < kc) jn = __ldg(lst + t + 1);
-            const int s = blk_it & 1;
-            const uint32_t par = ((blk_it >> 1) & 1) ^ 1;
-            unsigned char* tk = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES);
+          if (sparse) {
             if (lane == 0) {
-              if (!(ok = mbar_wait(&b.k_empty[s], par, abort_flag))) break;
-              mbar_expect_tx(&b.k_full[s], C::K_BYTES);
-              tma_load_2d(tk, &tm_k, &b.k_full[s], 0, bh * p.NP + j * BLK);
-              ++nkv;
-            } else {
-              if (!(ok = mbar_wait(&b.v_empty[s], par, abort_flag))) break;
-              mbar_expect_tx(&b.v_full[s], C::V_BYTES);
+              if (!(ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag))) break;
+              mbar_expect_tx(&b.q_full, C::Q_BYTES);
+              tma_load_2d(tq, &tm_q, &b.q_full, 0, bh * p.NP + i * BLK);
+              ++nq;
+            }
+            const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
+            int jn = __ldg(lst);
+            for (int t = 0; t < kc; ++t) {
+              const int j = jn;
+              if (t + 1 < kc) jn = __ldg(lst + t + 1);
+              const int s = nl & 1;
+              const uint32_t par = ((nl >> 1) & 1) ^ 1;
+              if (lane == 0) {
+                if (!(ok = mbar_wait(&b.k_empty[s], par, abort_flag))) break;
+                mbar_expect_tx(&b.k_full[s], C::K_BYTES);
+                tma_load_2d(k_stage(s), &tm_k, &b.k_full[s], 0, bh * p.NP + j * BLK);
+              } else {
+                if (!(ok = mbar_wait(&b.v_empty[s], par, abort_flag))) break;
+                mbar_expect_tx(&b.v_full[s], C::V_BYTES);
+#pragma unroll
+                for (int hh = 0; hh < D / 64; ++hh)
+                  tma_load_3d(v_stage(s) + hh * BLK * 128, &tm_v, &b.v_full[s], hh * 64, j * BLK, bh);
+              }
+              ++nl;
+            }
+          }
+          if (lin && lane == 1) {
+            for (int ch = 0; ch < C::LC && ok; ++ch) {
+              const int s = nl & 1;
+              if (!(ok = mbar_wait(&b.v_empty[s], ((nl >> 1) & 1) ^ 1, abort_flag))) break;
+              mbar_expect_tx(&b.v_full[s], C::G_CHUNK_BYTES);
 #pragma unroll
               for (int hh = 0; hh < D / 64; ++hh)
-                tma_load_3d(tk + C::K_BYTES + hh * BLK * 128, &tm_v, &b.v_full[s], hh * 64, j * BLK, bh);
-              ++nkv;
+                tma_load_2d(v_stage(s) + hh * BLK * 128, &tm_g, &b.v_full[s], hh * 64,
+                            int(((long long)bh * NB + i) * D + ch * C::LROWS));
+              ++nl;
             }
           }
         }
         // Loads still in flight (only after a failed wait) land before the CTA
         // exits: wait (bounded) for the last phase armed on each barrier.
         if (lane == 0 && nq > 0) (void)mbar_wait(&b.q_full, (nq - 1) & 1, nullptr);
-        for (uint32_t bb = nkv > 2 ? nkv - 2 : 0; bb < nkv; ++bb)
+        for (uint32_t bb = nl > 2 ? nl - 2 : 0; bb < nl; ++bb)
           (void)mbar_wait(lane == 0 ? &b.k_full[bb & 1] : &b.v_full[bb & 1], (bb >> 1) & 1, nullptr);
       }
     } else {
@@ -196,55 +271,75 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
         const uint32_t id_qk = idesc_i8(C::HB);
         const uint32_t id_pv = idesc_bf16(D, false, true);
         const uint64_t dq = smem_desc(smem_u32(tq), 16, C::KSBO, C::KSW);
-        uint32_t kv_it = 0, item_it = 0, hg = 0;   // hg: halves of the items before this one
+        uint32_t kit = 0, vit = 0, item_it = 0, hg = 0;   // hg: halves of the items before this one
         bool ok = true;
         for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
-          const int H = kc * NH;
-          if (!(ok = mbar_wait(&b.q_full, item_it & 1, abort_flag))) break;
-          // S(y) = Q K_half(y)^T into buffer (hg + y) % 2; at the first half of a
-          // key block it first waits for that block's K/V stage
-          auto issue_qk = [&](int y) -> bool {
-            const uint32_t g = hg + y;
-            const uint32_t blk_it = kv_it + y / NH;
-            const int s = blk_it & 1;
-            if (y % NH == 0) {
-              if (!mbar_wait(&b.k_full[s], (blk_it >> 1) & 1, abort_flag)) return false;
+          if (sparse) {
+            if (!(ok = mbar_wait(&b.q_full, item_it & 1, abort_flag))) break;
+            // S(y) = Q K_half(y)^T into buffer (hg + y) % 2; at the first half of a
+            // key block it first waits for that block's K stage
+            auto issue_qk = [&](int y) -> bool {
+              const uint32_t g = hg + y;
+              const uint32_t blk = kit + y / NH;
+              const int s = blk & 1;
+              if (y % NH == 0) {
+                if (!mbar_wait(&b.k_full[s], (blk >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+              }
+              const uint64_t dk = smem_desc(smem_u32(k_stage(s)) + (y % NH) * C::K_HALF_BYTES, 16, C::KSBO, C::KSW);
+              const uint32_t dS = tS + (g & 1) * 64;
+#pragma unroll
+              for (int kk = 0; kk < D / 32; ++kk)
+                mma_i8_ss(dS, dq + uint64_t(kk * 2), dk + uint64_t(kk * 2), id_qk, kk > 0 ? 1u : 0u);
+              tc_commit(&b.s_full[g & 1]);
+              if (y % NH == NH - 1) tc_commit(&b.k_empty[s]);
+              if (y == H - 1) tc_commit(&b.q_empty);
+              return true;
+            };
+            ok = issue_qk(0);
+            if (ok && H > 1) ok = issue_qk(1);
+            for (int x = 0; x < H && ok; ++x) {
+              const uint32_t g = hg + x;
+              if (!(ok = mbar_wait(&b.p_full[g & 1], (g >> 1) & 1, abort_flag))) break;
+              if (x == 0 && !(ok = mbar_wait(&b.o_free, (item_it & 1) ^ 1, abort_flag))) break;
+              const uint32_t vb = vit + x / NH;
+              const int s = vb & 1;
+              if (x % NH == 0 && !(ok = mbar_wait(&b.v_full[s], (vb >> 1) & 1, abort_flag))) break;
               tc_fence_after();
+              const uint64_t dv = smem_desc(smem_u32(v_stage(s)) + (x % NH) * C::V_HALF_BYTES, BLK * 128, 1024, 2);
+              const uint32_t aP = tS + (g & 1) * 64;
+#pragma unroll
+              for (int kk = 0; kk < C::HB / 16; ++kk)
+                mma_bf16_ts(tO, aP + kk * 8, dv + uint64_t(kk * (2048 >> 4)), id_pv, (x > 0 || kk > 0) ? 1u : 0u);
+              tc_commit(&b.pv_done[g & 1]);
+              if (x % NH == NH - 1) tc_commit(&b.v_empty[s]);
+              if (x + 2 < H) ok = issue_qk(x + 2);
             }
-            unsigned char* tk = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES);
-            const uint64_t dk = smem_desc(smem_u32(tk) + (y % NH) * C::K_HALF_BYTES, 16, C::KSBO, C::KSW);
-            const uint32_t dS = tS + (g & 1) * 64;
-#pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk)
-              mma_i8_ss(dS, dq + uint64_t(kk * 2), dk + uint64_t(kk * 2), id_qk, kk > 0 ? 1u : 0u);
-            tc_commit(&b.s_full[g & 1]);
-            if (y % NH == NH - 1) tc_commit(&b.k_empty[s]);
-            if (y == H - 1) tc_commit(&b.q_empty);
-            return true;
-          };
-          ok = issue_qk(0);
-          if (ok && H > 1) ok = issue_qk(1);
-          for (int x = 0; x < H && ok; ++x) {
-            const uint32_t g = hg + x;
-            if (!(ok = mbar_wait(&b.p_full[g & 1], (g >> 1) & 1, abort_flag))) break;
-            if (x == 0 && !(ok = mbar_wait(&b.o_free, (item_it & 1) ^ 1, abort_flag))) break;
-            const uint32_t vblk = kv_it + x / NH;
-            const int s = vblk & 1;
-            if (x % NH == 0 && !(ok = mbar_wait(&b.v_full[s], (vblk >> 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            unsigned char* tv = tq + C::Q_BYTES + s * (C::K_BYTES + C::V_BYTES) + C::K_BYTES;
-            const uint64_t dv = smem_desc(smem_u32(tv) + (x % NH) * C::V_HALF_BYTES, BLK * 128, 1024, 2);
-            const uint32_t aP = tS + (g & 1) * 64;
-#pragma unroll
-            for (int kk = 0; kk < C::HB / 16; ++kk)
-              mma_bf16_ts(tO, aP + kk * 8, dv + uint64_t(kk * (2048 >> 4)), id_pv, (x > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&b.pv_done[g & 1]);
-            if (x % NH == NH - 1) tc_commit(&b.v_empty[s]);
-            if (x == H - 1) tc_commit(&b.o_full);
-            if (x + 2 < H) ok = issue_qk(x + 2);
+            if (!ok) break;
+            kit += kc;
+            vit += kc;
           }
+          if (lin) {
+            // O += A . G'_i, A (bf16, D/2 columns) in the S buffer of half hg + H
+            if (H == 0 && !(ok = mbar_wait(&b.o_free, (item_it & 1) ^ 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&b.a_full, item_it & 1, abort_flag))) break;
+            const uint32_t aL = tS + ((hg + H) & 1) * 64;
+            for (int ch = 0; ch < C::LC && ok; ++ch) {
+              const int s = vit & 1;
+              if (!(ok = mbar_wait(&b.v_full[s], (vit >> 1) & 1, abort_flag))) break;
+              tc_fence_after();
+              const uint64_t dv = smem_desc(smem_u32(v_stage(s)), BLK * 128, 1024, 2);
+#pragma unroll
+              for (int kk = 0; kk < C::LROWS / 16; ++kk)
+                mma_bf16_ts(tO, aL + (ch * (C::LROWS / 16) + kk) * 8, dv + uint64_t(kk * (2048 >> 4)), id_pv,
+                            (H > 0 || ch > 0 || kk > 0) ? 1u : 0u);
+              tc_commit(&b.v_empty[s]);
+              ++vit;
+            }
+            if (!ok) break;
+          }
+          tc_commit(&b.o_full);
           hg += H;
-          kv_it += kc;
         }
         // every MMA issued here finishes before the CTA frees TMEM (bounded)
         tc_commit(&b.mma_drain);
@@ -264,11 +359,20 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
     const int part_rows = p.N % BLK;                // rows of a partial last block (0: none)
     for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
       const int bh = item / NB, i = item % NB;
-      const float sq_i = __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale;
-      const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
-      const int H = kc * NH;
+      const long long n = (long long)i * BLK + r;
+      const bool valid = r < BLK && n < p.N;
+      const __nv_bfloat16* qrow = p.q + ((long long)bh * p.N + (valid ? n : 0)) * D;
+      const float* grow = p.zrest + ((long long)bh * NB + i) * D;
       // running maximum m (log2 domain) and normaliser l of this row
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = sparse ? 0.f : 1.f;
+      float den = 0.f;
+      if (lin) {
+        if (!sparse) den = linear_den<D>(qrow, grow, valid);
+        else if (valid)   // read after the first half
+          for (int c = 0; c < D; c += 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + c));
+      }
+      const float sq_i = sparse ? __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale : 0.f;
+      const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
       float cl = 0.f;
       int jl = 0;
       for (int x = 0; x < H; ++x) {
@@ -292,24 +396,31 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
         SLA_TMEM_LD32(sbuf, v);
         SLA_TMEM_LD32(sbuf + 32, (v + 32));
         tmem_ld_wait();
-        // row maximum of the int32 scores (c >= 0 keeps the order)
-        int amax = INT_MIN;
-        if (!partial) {
+        // The float with bits acc + 0x4B400000 is exactly 1.5*2^23 + acc
+        // (|acc| <= D*127^2 < 2^22); c >= 0, so its maximum gives the row's.
 #pragma unroll
-          for (int e = 0; e < 64; ++e) amax = max(amax, (int)v[e]);
-        } else {
+        for (int e = 0; e < 64; ++e) v[e] += 0x4B400000u;
+        if (partial) {   // keys past N (a partial last block): out of the maximum
 #pragma unroll
           for (int e = 0; e < 64; ++e)
-            if (e < nvalid) amax = max(amax, (int)v[e]);
+            if (e >= nvalid) v[e] = 0xFF800000u;   // -inf
         }
-        const float mx = (nvalid > 0) ? (float)amax * c : -INFINITY;
+        float xm[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) xm[q] = fmax3(__uint_as_float(v[3 * q]), __uint_as_float(v[3 * q + 1]),
+                                                  __uint_as_float(v[3 * q + 2]));
+#pragma unroll
+        for (int e = 24; e < 64; e += 2)
+          xm[(e / 2) & 7] = fmax3(xm[(e / 2) & 7], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        const float xmax = fmaxf(fmax3(xm[0], xm[1], xm[2]), fmax3(fmax3(xm[3], xm[4], xm[5]), xm[6], xm[7]));
+        const float mx = (xmax - 12582912.f) * c;   // exact difference; -inf when no key is valid
         if (x == 0) {
           m = mx;
-        } else if (__any_sync(0xffffffffu, mx > m + 8.f)) {
-          // Some row's maximum grew by more than 2^8: once the previous PV has
-          // finished, the warp rescales O (tcgen05.ld/st are warp-collective);
-          // rows whose maximum did not grow keep alpha = 1.  Otherwise the
-          // stale maximum stays (P <= 2^8).
+        } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+          // Some row's maximum grew by more than 2^kRescaleLog2: once the
+          // previous PV has finished, the warp rescales O (tcgen05.ld/st are
+          // warp-collective).  Otherwise the stale maximum stays
+          // (P <= 2^kRescaleLog2).
           // PV(g-2) and older are complete (QK(g) was issued after PV(g-2) and
           // its S is ready); PV(g-1) uses buffer (g-1)&1, whose uses before it
           // are complete, so this parity names PV(g-1) without ambiguity.
@@ -329,47 +440,79 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             SLA_TMEM_ST16(tO + ch * 16, w);
           }
         }
-        // P = 2^(acc * c - m) rounded to bf16 into TMEM.  The float with bits
-        // acc + 0x4B400000 is exactly 1.5*2^23 + acc (|acc| <= D*127^2 < 2^22),
-        // so acc*c - m = fma(that, c, -(1.5*2^23*c + m)); the one rounding of
-        // that constant shifts all exponents of this row and half by the same
+        // P = 2^(acc * c - m) = 2^((1.5*2^23 + acc) * c - (1.5*2^23 * c + m)):
+        // one FMA per key (two per packed instruction); the one rounding of
+        // the constant shifts all exponents of this row and half by the same
         // amount (< 2^-24 relative to 1.5*2^23*c), i.e. scales P and l alike.
-        // The packed pair e/2 goes to v[e/2], a slot already consumed.
         const float kk = -fmaf(12582912.f, c, m);
-        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+        const uint64_t c2 = f32x2(c, c), k2 = f32x2(kk, kk);
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          float y0, y1;
+          f32x2_split(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), c2, k2), y0, y1);
+          v[e] = __float_as_uint(ex2_approx(y0));
+          v[e + 1] = __float_as_uint(ex2_approx(y1));
+        }
+        if (partial) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (e >= nvalid) v[e] = 0u;
+        }
+        // l sums the unrounded P (four packed partial sums); the bf16 pair
+        // e/2 goes to v[e/2], a slot already consumed
+        uint64_t la = f32x2(0.f, 0.f), lb = la;
 #pragma unroll
         for (int e = 0; e < 64; e += 4) {
-          float p0 = ex2_approx(fmaf(__int_as_float((int)v[e] + 0x4B400000), c, kk));
-          float p1 = ex2_approx(fmaf(__int_as_float((int)v[e + 1] + 0x4B400000), c, kk));
-          float p2 = ex2_approx(fmaf(__int_as_float((int)v[e + 2] + 0x4B400000), c, kk));
-          float p3 = ex2_approx(fmaf(__int_as_float((int)v[e + 3] + 0x4B400000), c, kk));
-          if (partial) {
-            p0 = (e < nvalid) ? p0 : 0.f;
-            p1 = (e + 1 < nvalid) ? p1 : 0.f;
-            p2 = (e + 2 < nvalid) ? p2 : 0.f;
-            p3 = (e + 3 < nvalid) ? p3 : 0.f;
-          }
-          l0 += p0;
-          l1 += p1;
-          l2 += p2;
-          l3 += p3;
-          v[e >> 1] = pack_bf16x2(p0, p1);
-          v[(e >> 1) + 1] = pack_bf16x2(p2, p3);
+          la = add_f32x2(la, f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])));
+          lb = add_f32x2(lb, f32x2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])));
+          v[e >> 1] = pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+          v[(e >> 1) + 1] = pack_bf16x2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
         }
-        l += (l0 + l1) + (l2 + l3);
+        {
+          float a0, a1, b0, b1;
+          f32x2_split(la, a0, a1);
+          f32x2_split(lb, b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
         SLA_TMEM_ST16(sbuf, v);
         SLA_TMEM_ST16(sbuf + 16, (v + 16));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&b.p_full[g & 1]);
+        // den of the linear part, while the tensor core runs this half's PV
+        if (lin && x == 0) den = linear_den<D>(qrow, grow, valid);
       }
       if (!ok) break;
+      if (lin) {
+        // A = bf16(phi(q) * l / den) into the S buffer of half hg + H, once the
+        // PV that last read that buffer (half hg + H - 2 of this item) is done;
+        // an earlier reader finished before the previous o_full
+        const float sc = (valid && den > 0.f) ? l / den : 0.f;
+        uint32_t a[D / 2];
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          const uint4 raw = valid ? __ldg(reinterpret_cast<const uint4*>(qrow) + c8) : make_uint4(0, 0, 0, 0);
+          a[4 * c8 + 0] = pack_bf16x2(phi_bf16(uint16_t(raw.x)) * sc, phi_bf16(uint16_t(raw.x >> 16)) * sc);
+          a[4 * c8 + 1] = pack_bf16x2(phi_bf16(uint16_t(raw.y)) * sc, phi_bf16(uint16_t(raw.y >> 16)) * sc);
+          a[4 * c8 + 2] = pack_bf16x2(phi_bf16(uint16_t(raw.z)) * sc, phi_bf16(uint16_t(raw.z >> 16)) * sc);
+          a[4 * c8 + 3] = pack_bf16x2(phi_bf16(uint16_t(raw.w)) * sc, phi_bf16(uint16_t(raw.w >> 16)) * sc);
+        }
+        if (H >= 2) {
+          const uint32_t gp = hg + H - 2;
+          if (!(ok = mbar_wait(&b.pv_done[gp & 1], (gp >> 1) & 1, abort_flag))) break;
+        }
+        tc_fence_after();
+        const uint32_t abuf = tS + ((hg + H) & 1) * 64;
+#pragma unroll
+        for (int c = 0; c < D / 2; c += 16) SLA_TMEM_ST16(abuf + c, (a + c));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&b.a_full);
+      }
       hg += H;
       if (!(ok = mbar_wait(&b.o_full, item_it & 1, abort_flag))) break;
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const long long n = (long long)i * BLK + r;
-      const bool valid = r < BLK && n < p.N;
       const long long obase = ((long long)bh * p.N + n) * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -377,11 +520,21 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
         SLA_TMEM_LD32(tO + ch * 32, w);
         tmem_ld_wait();
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(p.o + obase + ch * 32);
+          if (p.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + obase + ch * 32);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(w[4 * q]) * inv_l, __uint_as_float(w[4 * q + 1]) * inv_l,
-                                 __uint_as_float(w[4 * q + 2]) * inv_l, __uint_as_float(w[4 * q + 3]) * inv_l);
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(__uint_as_float(w[4 * q]) * inv_l, __uint_as_float(w[4 * q + 1]) * inv_l,
+                                   __uint_as_float(w[4 * q + 2]) * inv_l, __uint_as_float(w[4 * q + 3]) * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + ch * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              dst[q] = make_uint4(pack_bf16x2(__uint_as_float(w[8 * q]) * inv_l, __uint_as_float(w[8 * q + 1]) * inv_l),
+                                  pack_bf16x2(__uint_as_float(w[8 * q + 2]) * inv_l, __uint_as_float(w[8 * q + 3]) * inv_l),
+                                  pack_bf16x2(__uint_as_float(w[8 * q + 4]) * inv_l, __uint_as_float(w[8 * q + 5]) * inv_l),
+                                  pack_bf16x2(__uint_as_float(w[8 * q + 6]) * inv_l, __uint_as_float(w[8 * q + 7]) * inv_l));
+          }
         }
       }
       tc_fence_before();

@@ -11,13 +11,12 @@
 // (k_lingemm, tcgen05 bf16 with float32 accumulation; summing the
 // non-selected blocks directly avoids the cancellation of total minus
 // selected).  The states arrive with W_proj folded in (h'_j = h_j W_proj, see
-// k_stats.cuh), so per query row n of block i (k_linout)
+// k_stats.cuh), so per query row n of block i
 //     out_n = O_sparse,n + phi(q_n) G'_i / (phi(q_n) . g_i),   G'_i = G_i W_proj,
-// one tensor-core product per query block.
+// one tensor-core product per query block, done inside k_attn (k_attn.cuh).
 #pragma once
 #include <cuda_bf16.h>
 #include "sm100.cuh"
-#include "k_stats.cuh"
 
 namespace sla {
 
@@ -136,148 +135,6 @@ __global__ void __launch_bounds__(128, 2) k_lingemm(const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, 256);
-}
-
-// ------------------------------------------------------------------ k_linout
-struct LinOutParams {
-  const __nv_bfloat16* q;      // [BH][N][D]
-  const float* zrest;          // [BH][NB][D]
-  int N, NB, BLK;
-};
-
-template <int D>
-struct LinOutCfg {
-  static constexpr int A_BYTES = 128 * D * 2;   // phi(Q) tile (K-major, 64-column atoms of 16 KB)
-  static constexpr int G_BYTES = D * D * 2;     // G'_i (MN-major)
-  // after the product, A and G are reused for the 128 x D float32 result y,
-  // as D/32 column chunks of 32 floats (128-byte rows, 128-byte swizzle)
-  static constexpr int Y_BYTES = 128 * D * 4;
-  static constexpr int AG_BYTES = (A_BYTES + G_BYTES > Y_BYTES) ? A_BYTES + G_BYTES : Y_BYTES;
-  static constexpr int SMEM = AG_BYTES + 1024 + 128 + D * 4;
-};
-
-// One CTA (128 threads, thread = query row) per query block.  out holds
-// O_sparse on entry; y = phi(q) G' / den is staged in shared memory and added
-// to out by TMA reductions (float32 add in L2, one add per element).
-template <int D>
-__global__ void __launch_bounds__(128) k_linout(const __grid_constant__ CUtensorMap tm_q,
-                                               const __grid_constant__ CUtensorMap tm_g,
-                                               const __grid_constant__ CUtensorMap tm_out, const LinOutParams p) {
-  using C = LinOutCfg<D>;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* base =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sa = base;
-  unsigned char* sg = sa + C::A_BYTES;
-  float* sz = reinterpret_cast<float*>(sa + C::AG_BYTES);          // z_rest of this query block
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sz + D);            // 0: G load, 1: MMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int i = blockIdx.x;
-  const int bh = blockIdx.y;
-
-  if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, D);
-    tmem_relinquish();
-  }
-  if (tid < D) sz[tid] = p.zrest[((long long)bh * p.NB + i) * D + tid];
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (tid == 0) {
-    // the query tile lands in the A operand's own layout (K-major, 128-byte
-    // swizzle, 64-column atoms of 16 KB); rows past N arrive as zeros
-    mbar_expect_tx(&bars[0], C::G_BYTES + C::A_BYTES);
-#pragma unroll
-    for (int hh = 0; hh < D / 64; ++hh) {
-      tma_load_2d(sg + hh * D * 128, &tm_g, &bars[0], hh * 64, int(((long long)bh * p.NB + i) * D));
-      tma_load_3d(sa + hh * 16384, &tm_q, &bars[0], hh * 64, i * p.BLK, bh);
-    }
-  }
-
-  const int r = tid;
-  const long long n = (long long)i * p.BLK + r;
-  const bool valid = r < p.BLK && n < p.N;
-  const bool landed = __syncthreads_and(mbar_wait(&bars[0], 0, abort_flag));
-  // phi(q) in place: each thread rewrites its own row of the A tile
-  float den = 0.f;
-  {
-#pragma unroll
-    for (int c8 = 0; c8 < D / 8; ++c8) {
-      const int atom = c8 >> 3, chunk = c8 & 7;
-      uint4* slot = reinterpret_cast<uint4*>(sa + atom * 16384 + sw128_offset(r, chunk));
-      const uint4 raw = *slot;
-      const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const float f0 = valid ? phi_elu1(__uint_as_float(uint32_t(hv[e]) << 16)) : 0.f;
-        const float f1 = valid ? phi_elu1(__uint_as_float(uint32_t(hv[e + 1]) << 16)) : 0.f;
-        den = fmaf(f0, sz[c8 * 8 + e], den);
-        den = fmaf(f1, sz[c8 * 8 + e + 1], den);
-        pk[e >> 1] = pack_bf16x2(f0, f1);
-      }
-      *slot = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-  }
-  fence_async_shared();
-  __syncthreads();
-  if (tid == 0) {
-    if (landed) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16(D, false, true);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t da = smem_desc(smem_u32(sa + (kk >> 2) * 16384) + (kk & 3) * 32, 16, 1024, 2);
-        const uint64_t db = smem_desc(smem_u32(sg) + kk * 2048, D * 128, 1024, 2);
-        mma_bf16_ss(tmem, da, db, idesc, kk > 0 ? 1u : 0u);
-      }
-    }
-    tc_commit(&bars[1]);
-  }
-  __syncwarp();
-  const bool ok = __syncthreads_and(mbar_wait(&bars[1], 0, abort_flag));
-  tc_fence_after();
-  // y row r = phi(q_r) G' / den_r -> shared memory over A and G (the product
-  // is complete): chunk c holds columns [32c, 32c + 32) as 128-byte rows
-  const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
-  const float inv_den = (valid && den > 0.f) ? 1.f / den : 0.f;
-#pragma unroll
-  for (int ch = 0; ch < D / 16; ++ch) {
-    uint32_t v[16];
-    SLA_TMEM_LD16(trow + ch * 16, v);
-    tmem_ld_wait();
-    unsigned char* chunk = base + (ch >> 1) * 16384;
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4)
-      *reinterpret_cast<float4*>(chunk + sw128_offset(r, (ch & 1) * 4 + q4)) =
-          make_float4(__uint_as_float(v[4 * q4]) * inv_den, __uint_as_float(v[4 * q4 + 1]) * inv_den,
-                      __uint_as_float(v[4 * q4 + 2]) * inv_den, __uint_as_float(v[4 * q4 + 3]) * inv_den);
-  }
-  fence_async_shared();
-  tc_fence_before();
-  __syncthreads();
-  if (tid == 0) {
-    if (ok) {
-      // rows past N are dropped by the TMA; the box is BLK rows high
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tma_reduce_add_3d(&tm_out, base + c * 16384, c * 32, i * p.BLK, bh);
-      bulk_commit_group();
-    }
-    bulk_wait_group_read0();
-  }
-  tc_fence_after();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, D);
 }
 
 }  // namespace sla

@@ -91,7 +91,13 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
   for (int e = 0; e < VEC; ++e) muc[e] = isk ? mu[(long long)bh * D + g * VEC + e] : 0.f;
   __syncthreads();   // barrier initialised before anyone waits on it
   const bool landed = mbar_wait(bar, 0, nullptr);
-  if (!__syncthreads_and(landed)) return;   // uniform exit if the load did not land in time
+  if (!__syncthreads_and(landed)) {
+    // uniform exit if the load did not land in time; the copy may still be in
+    // flight, so one thread waits for it once more (bounded) before the CTA's
+    // shared memory is handed on
+    if (tid == 0) (void)mbar_wait(bar, 0, nullptr);
+    return;
+  }
 
   // pass 1: block maximum of |x| (K: x - mu on valid rows) and, for Q, float64 channel sums
   float mloc = 0.f;

@@ -24,6 +24,7 @@
 // an MN-major A operand and V'_j written back over V_j as an MN-major B operand.
 #pragma once
 #include <cuda_bf16.h>
+#include "exact_mean.cuh"
 #include "sm100.cuh"
 
 namespace sla {
@@ -279,25 +280,34 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
   if (warp == 0) tmem_dealloc(tmem, 2 * D);
 }
 
-// mu[bh][c] = float32 nearest to (sum_j ksum[bh][j][c]) / N.  One CTA per
-// (batch, head, group of CG channels): thread (gi, c) sums every G-th block of
-// channel c, then the G partial sums are added in a fixed order.  The block
-// sums are exact when every K value of the channel is a multiple of the
-// smallest one's unit in the last place and the total stays below 2^53 of
-// those units, so the order does not matter; kexp lets the kernel check that
-// and raise DEV_ERR_INEXACT otherwise.
+// mu[bh][c] = float32 nearest to (sum of the N values of K[bh][:][c]) / N.
+// One CTA per (batch, head, group of CG channels).
+//
+// Fast path: thread (gi, c) sums every G-th float64 block sum of channel c,
+// then the G partial sums are added in a fixed order.  The block sums are
+// exact when every K value of the channel is a multiple of the smallest one's
+// unit in the last place and the total stays below 2^53 of those units, so the
+// order does not matter; kexp (largest and smallest exponent field per block)
+// shows whether that holds.
+// Exact path, for a channel where it does not: the CTA re-reads the channel's
+// N values and sums them as 320-bit integers (exact_mean.cuh), then rounds the
+// exact quotient once.  Either way mu is the correctly rounded exact mean.
 constexpr int kMeanCG = 8;   // channels per CTA
 
 template <int D>
 __global__ void __launch_bounds__(1024) k_channel_mean(const double* __restrict__ ksum,
-                                                      const uint8_t* __restrict__ kexp, float* __restrict__ mu,
+                                                      const uint8_t* __restrict__ kexp,
+                                                      const __nv_bfloat16* __restrict__ K, float* __restrict__ mu,
                                                       int NB, int N) {
   constexpr int CG = kMeanCG;
   constexpr int G = 1024 / CG;
   __shared__ double rs[G][CG];
   __shared__ uint32_t re[G][CG];
+  __shared__ int need_exact[CG];
+  __shared__ Wide320 wpart[32][CG][2];   // per warp and channel: positive, negative part
   const long long bh = blockIdx.x;
-  const int c = blockIdx.y * CG + threadIdx.x % CG, gi = threadIdx.x / CG;
+  const int cc = threadIdx.x % CG, gi = threadIdx.x / CG;
+  const int c = blockIdx.y * CG + cc;
   double s = 0.0;
   uint32_t mx = 0u, mn = 255u;
   for (int j = gi; j < NB; j += G) {
@@ -306,44 +316,89 @@ __global__ void __launch_bounds__(1024) k_channel_mean(const double* __restrict_
     mx = max(mx, (uint32_t)kexp[2 * o]);
     mn = min(mn, (uint32_t)kexp[2 * o + 1]);
   }
-  rs[gi][threadIdx.x % CG] = s;
-  re[gi][threadIdx.x % CG] = (mx << 8) | mn;
+  rs[gi][cc] = s;
+  re[gi][cc] = (mx << 8) | mn;
   __syncthreads();
-  if (gi != 0) return;
-  s = 0.0;
-  mx = 0u;
-  mn = 255u;
-  for (int q = 0; q < G; ++q) {
-    s += rs[q][threadIdx.x];
-    mx = max(mx, re[q][threadIdx.x] >> 8);
-    mn = min(mn, re[q][threadIdx.x] & 0xFFu);
-  }
-  int lgN = 0;
-  while ((1LL << lgN) < (long long)N) ++lgN;
-  if (mx >= mn && int(mx) - int(mn) + 8 + lgN + 1 > 53) raise_error(DEV_ERR_INEXACT);
-  // Correct rounding of s / N to float32: the float64 quotient q is within
-  // half a float64 ulp of s/N, so it rounds to the same float32 unless q is a
-  // float32 midpoint; then the sign of the exact remainder s - q*N decides.
-  const double dn = (double)N;
-  const double q = s / dn;
-  float f = __double2float_rn(q);
-  const double fd = (double)f;
-  if (fd != q) {
-    // neighbouring float32 on the other side of q
-    const float g2 = (q > fd) ? nextafterf(f, INFINITY) : nextafterf(f, -INFINITY);
-    const double mid = 0.5 * (fd + (double)g2);
-    if (mid == q) {
-      const double rem = fma(-q, dn, s);  // exact: s - q*N
-      if (rem == 0.0) {
-        f = (__float_as_uint(f) & 1u) ? g2 : f;   // exact tie: even mantissa
-      } else {
-        const bool above = rem > 0.0;             // s/N > q
-        const float lo = fminf(f, g2), hi = fmaxf(f, g2);
-        f = above ? hi : lo;
+  if (gi == 0) {
+    s = 0.0;
+    mx = 0u;
+    mn = 255u;
+    for (int q = 0; q < G; ++q) {
+      s += rs[q][cc];
+      mx = max(mx, re[q][cc] >> 8);
+      mn = min(mn, re[q][cc] & 0xFFu);
+    }
+    int lgN = 0;
+    while ((1LL << lgN) < (long long)N) ++lgN;
+    const bool wide = mx >= mn && int(mx) - int(mn) + 8 + lgN + 1 > 53;
+    need_exact[cc] = wide ? 1 : 0;
+    if (!wide) {
+      // Correct rounding of s / N to float32: the float64 quotient q is within
+      // half a float64 ulp of s/N, so it rounds to the same float32 unless q is
+      // a float32 midpoint; then the sign of the exact remainder s - q*N decides.
+      const double dn = (double)N;
+      const double q = s / dn;
+      float f = __double2float_rn(q);
+      const double fd = (double)f;
+      if (fd != q) {
+        // neighbouring float32 on the other side of q
+        const float g2 = (q > fd) ? nextafterf(f, INFINITY) : nextafterf(f, -INFINITY);
+        const double mid = 0.5 * (fd + (double)g2);
+        if (mid == q) {
+          const double rem = fma(-q, dn, s);  // exact: s - q*N
+          if (rem == 0.0) {
+            f = (__float_as_uint(f) & 1u) ? g2 : f;   // exact tie: even mantissa
+          } else {
+            const bool above = rem > 0.0;             // s/N > q
+            const float lo = fminf(f, g2), hi = fmaxf(f, g2);
+            f = above ? hi : lo;
+          }
+        }
       }
+      mu[bh * D + c] = f;
     }
   }
-  mu[bh * D + c] = f;
+  __syncthreads();
+  int any = 0;
+#pragma unroll
+  for (int q = 0; q < CG; ++q) any |= need_exact[q];
+  if (!any) return;   // uniform
+
+  // exact path: thread (gi, cc) takes rows gi, gi + G, ... of channel c
+  Wide320 pos, neg;
+  wide_zero(pos);
+  wide_zero(neg);
+  if (need_exact[cc]) {
+    const uint16_t* kc = reinterpret_cast<const uint16_t*>(K) + bh * (long long)N * D + c;
+    for (int n = gi; n < N; n += G) wide_add_bf16(pos, neg, __ldg(kc + (long long)n * D));
+  }
+  // lanes l, l ^ 8, l ^ 16, l ^ 24 hold the same channel
+#pragma unroll
+  for (int o = CG; o < 32; o <<= 1) {
+    Wide320 a, b;
+#pragma unroll
+    for (int i = 0; i < kWideLimbs; ++i) {
+      a.w[i] = __shfl_xor_sync(0xffffffffu, pos.w[i], o);
+      b.w[i] = __shfl_xor_sync(0xffffffffu, neg.w[i], o);
+    }
+    wide_add(pos, a);
+    wide_add(neg, b);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane < CG) {
+    wpart[warp][lane][0] = pos;
+    wpart[warp][lane][1] = neg;
+  }
+  __syncthreads();
+  if (gi == 0 && need_exact[cc]) {
+    wide_zero(pos);
+    wide_zero(neg);
+    for (int w = 0; w < 32; ++w) {
+      wide_add(pos, wpart[w][cc][0]);
+      wide_add(neg, wpart[w][cc][1]);
+    }
+    mu[bh * D + c] = wide_mean_to_f32(pos, neg, (uint32_t)N);
+  }
 }
 
 }  // namespace sla

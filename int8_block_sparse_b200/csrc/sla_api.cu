@@ -4,9 +4,8 @@
 //      k_channel_mean  mu                                   (k_stats.cuh)
 //   K2 k_quant         smoothing + INT8 codes + Q block sums (k_quant.cuh)
 //   K3 k_mask          pooled scores + top-k                 (k_mask.cuh)
-//   K5a k_lingemm      sums of the non-selected states       (k_linear.cuh)
-//   K4 k_attn          critical-block attention              (k_attn.cuh)
-//   K5b k_linout       linear branch, projection, add        (k_linear.cuh)
+//   K5 k_lingemm       sums of the non-selected states       (k_linear.cuh)
+//   K4 k_attn          critical-block attention + linear part (k_attn.cuh)
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -230,7 +229,7 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
   k_kstats<D, BLK><<<g1, StatsCfg<D, BLK>::THREADS, sm1, st>>>(mv, mw, k, w.ksum, w.kbar, w.kexp, states ? w.hstate : nullptr, s.N,
                                          (int)s.NB, w.hpitch); }
   { ProfScope ps(SLA_K_MEAN, st);
-  k_channel_mean<D><<<dim3((unsigned)s.BH, D / kMeanCG), 1024, 0, st>>>(w.ksum, w.kexp, w.mu, (int)s.NB, s.N); }
+  k_channel_mean<D><<<dim3((unsigned)s.BH, D / kMeanCG), 1024, 0, st>>>(w.ksum, w.kexp, k, w.mu, (int)s.NB, s.N); }
   CUtensorMap mq, mk;
   {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
@@ -282,41 +281,57 @@ int num_sms() {
   return n;
 }
 
+// k_attn in one of its modes: sparse (the selected blocks), lin (the linear
+// part), out as float32 or bf16.
 template <int D, int BLK>
-int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* v, float* o, cudaStream_t st) {
+int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __nv_bfloat16* v, void* out,
+                bool out_f32, bool sparse, bool lin, cudaStream_t st) {
   using C = AttnCfg<D, BLK>;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mg;
+  std::memset(&mq, 0, sizeof(mq));
+  std::memset(&mk, 0, sizeof(mk));
+  std::memset(&mv, 0, sizeof(mv));
+  std::memset(&mg, 0, sizeof(mg));
   const CUtensorMapSwizzle ksw = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  {
+  if (sparse) {
     cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(s.BH * s.NP)};
     cuuint64_t str[1] = {(cuuint64_t)D};
     cuuint32_t boxq[2] = {(cuuint32_t)D, 128u};
     cuuint32_t boxk[2] = {(cuuint32_t)D, (cuuint32_t)BLK};
     if (!make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w.qi8, dims, str, boxq, ksw)) return SLA_ERR_CUDA;
     if (!make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w.ki8, dims, str, boxk, ksw)) return SLA_ERR_CUDA;
+    cuuint64_t vd[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
+    cuuint64_t vs[2] = {(cuuint64_t)D * 2, (cuuint64_t)s.N * D * 2};
+    cuuint32_t vb[3] = {64u, (cuuint32_t)BLK, 1u};
+    if (!make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, vd, vs, vb, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
   }
-  {
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
-    cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)s.N * D * 2};
-    cuuint32_t box[3] = {64u, (cuuint32_t)BLK, 1u};
-    if (!make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (lin) {
+    cuuint64_t gd[2] = {(cuuint64_t)D, (cuuint64_t)(s.BH * s.NB * D)};
+    cuuint64_t gs[1] = {(cuuint64_t)D * 2};
+    cuuint32_t gb[2] = {64u, (cuuint32_t)C::LROWS};
+    if (!make_map(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.grest, gd, gs, gb, CU_TENSOR_MAP_SWIZZLE_128B))
       return SLA_ERR_CUDA;
   }
   AttnParams p;
-  p.idx = w.idx; p.sq = w.sq; p.sk = w.sk; p.o = o;
+  p.idx = w.idx; p.sq = w.sq; p.sk = w.sk; p.q = q; p.zrest = w.zrest; p.out = out;
   p.N = s.N; p.NB = (int)s.NB; p.NP = (int)s.NP; p.kc = (int)s.kc; p.items = (int)(s.BH * s.NB);
+  p.sparse = sparse ? 1 : 0;
+  p.lin = lin ? 1 : 0;
+  p.out_f32 = out_f32 ? 1 : 0;
   p.qk_scale = (float)(1.4426950408889634 / std::sqrt((double)D));
   cudaFuncSetAttribute(k_attn<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int ctas = (int)std::min<long long>(num_sms(), (p.items + 1) / 2);
   ProfScope ps(SLA_K_ATTN, st);
-  k_attn<D, BLK><<<ctas, 384, C::SMEM, st>>>(mq, mk, mv, p);
+  k_attn<D, BLK><<<ctas, 384, C::SMEM, st>>>(mq, mk, mv, mg, p);
   return cuda_status(cudaGetLastError());
 }
 
+// G'_i and g_i, the sums of the linear states over the blocks query block i
+// did not select (k_lingemm), for k_attn's linear part.
 template <int D>
-int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const float* osparse, float* out,
-                  cudaStream_t st) {
-  CUtensorMap ma, mb, mg;
+int launch_lingemm(const Shape& s, Workspace& w, cudaStream_t st) {
+  CUtensorMap ma, mb;
   {
     cuuint64_t dims[3] = {(cuuint64_t)w.ncpitch, (cuuint64_t)s.NB, (cuuint64_t)s.BH};
     cuuint64_t str[2] = {(cuuint64_t)w.ncpitch * 2, (cuuint64_t)(w.ncpitch * s.NB * 2)};
@@ -331,68 +346,34 @@ int launch_linear(const Shape& s, Workspace& w, const __nv_bfloat16* q, const fl
     if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w.hstate, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return SLA_ERR_CUDA;
   }
-  {
-    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(s.BH * s.NB * D)};
-    cuuint64_t str[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)D};
-    if (!make_map(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w.grest, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return SLA_ERR_CUDA;
-  }
   LinGemmParams gp;
   gp.grest = w.grest; gp.zrest = w.zrest; gp.NB = (int)s.NB; gp.D = D; gp.E = D * D + D;
   gp.nkt = (int)((s.NB + 63) / 64);
   cudaFuncSetAttribute(k_lingemm, cudaFuncAttributeMaxDynamicSharedMemorySize, LG_SMEM);
   dim3 g1((unsigned)((gp.E + 255) / 256), (unsigned)((s.NB + 127) / 128), (unsigned)s.BH);
-  { ProfScope ps(SLA_K_LINGEMM, st);
-  k_lingemm<<<g1, 128, LG_SMEM, st>>>(ma, mb, gp); }
-  // out = O_sparse + y: out must hold O_sparse before the TMA adds y to it
-  if (osparse != out &&
-      cudaMemcpyAsync(out, osparse, (size_t)s.BH * s.N * D * sizeof(float), cudaMemcpyDeviceToDevice, st) !=
-          cudaSuccess)
-    return SLA_ERR_CUDA;
-  CUtensorMap mo, mq;
-  {
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
-    cuuint64_t str[2] = {(cuuint64_t)D * 2, (cuuint64_t)s.N * D * 2};
-    cuuint32_t box[3] = {64u, 128u, 1u};
-    if (!make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return SLA_ERR_CUDA;
-  }
-  {
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
-    cuuint64_t str[2] = {(cuuint64_t)D * 4, (cuuint64_t)s.N * D * 4};
-    cuuint32_t box[3] = {32u, (cuuint32_t)s.block, 1u};
-    if (!make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return SLA_ERR_CUDA;
-  }
-  LinOutParams op;
-  op.q = q; op.zrest = w.zrest;
-  op.N = s.N; op.NB = (int)s.NB; op.BLK = s.block;
-  cudaFuncSetAttribute(k_linout<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinOutCfg<D>::SMEM);
-  dim3 g2((unsigned)s.NB, (unsigned)s.BH);
-  { ProfScope ps(SLA_K_LINOUT, st);
-  k_linout<D><<<g2, 128, LinOutCfg<D>::SMEM, st>>>(mq, mg, mo, op); }
+  ProfScope ps(SLA_K_LINGEMM, st);
+  k_lingemm<<<g1, 128, LG_SMEM, st>>>(ma, mb, gp);
   return cuda_status(cudaGetLastError());
 }
 
 // ------------------------------------------------------------------ dispatch
 template <int D, int BLK>
 int run_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-             const __nv_bfloat16* proj, float* out, float* o_sparse, Workspace& w, cudaStream_t st) {
+             const __nv_bfloat16* proj, void* out, bool out_f32, float* o_sparse, float* o_lin, Workspace& w,
+             cudaStream_t st) {
   const bool linear = s.kc < s.NB;
   int rc = launch_stats_quant<D, BLK>(s, q, k, v, proj, w, linear, true, w.qi8, w.ki8, w.sq, w.sk, st);
   if (rc) return rc;
   rc = launch_mask<D>(s, w, w.idx, nullptr, linear ? w.notcrit : nullptr, st);
   if (rc) return rc;
-  // O_sparse goes to o_sparse when the caller wants it, else straight into
-  // out, which the linear branch then updates in place.
-  float* osp = (linear && o_sparse != nullptr) ? o_sparse : out;
-  rc = launch_attn<D, BLK>(s, w, v, osp, st);
-  if (rc) return rc;
-  if (linear) return launch_linear<D>(s, w, q, osp, out, st);
-  if (o_sparse != nullptr)
-    return cuda_status(cudaMemcpyAsync(o_sparse, out, (size_t)s.BH * s.N * D * sizeof(float),
-                                       cudaMemcpyDeviceToDevice, st));
+  if (linear && (rc = launch_lingemm<D>(s, w, st))) return rc;
+  if ((rc = launch_attn<D, BLK>(s, w, q, v, out, out_f32, true, linear, st))) return rc;
+  // the two parts on their own, in float32 (inspection and tests)
+  if (o_sparse != nullptr && (rc = launch_attn<D, BLK>(s, w, q, v, o_sparse, true, true, false, st))) return rc;
+  if (o_lin != nullptr) {
+    if (linear) return launch_attn<D, BLK>(s, w, q, v, o_lin, true, false, true, st);
+    return cuda_status(cudaMemsetAsync(o_lin, 0, (size_t)s.BH * s.N * D * sizeof(float), st));
+  }
   return SLA_OK;
 }
 
@@ -440,8 +421,37 @@ __global__ void k_selftest_wait_timeout() {
 // Host code must not use this name as an address; see noalloc_scratch().
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SLA_NOALLOC_SCRATCH_BYTES];
 
+// Loads every kernel sla_mask_noalloc can launch onto the current device, so
+// that no later call does so (with lazy module loading, a kernel's first use
+// would otherwise load its code then, which may allocate device memory).
+bool noalloc_load_kernels() {
+  cudaFuncAttributes a;
+  bool ok = true;
+  auto load = [&](const void* f) { ok = ok && cudaFuncGetAttributes(&a, f) == cudaSuccess; };
+  load((const void*)k_kstats<64, 64>);
+  load((const void*)k_kstats<64, 128>);
+  load((const void*)k_kstats<128, 64>);
+  load((const void*)k_kstats<128, 128>);
+  load((const void*)k_channel_mean<64>);
+  load((const void*)k_channel_mean<128>);
+  load((const void*)k_quant<64, 64>);
+  load((const void*)k_quant<64, 128>);
+  load((const void*)k_quant<128, 64>);
+  load((const void*)k_quant<128, 128>);
+  load((const void*)k_mask<64, 1>);
+  load((const void*)k_mask<64, 2>);
+  load((const void*)k_mask<64, 4>);
+  load((const void*)k_mask<64, 8>);
+  load((const void*)k_mask<128, 1>);
+  load((const void*)k_mask<128, 2>);
+  load((const void*)k_mask<128, 4>);
+  load((const void*)k_mask<128, 8>);
+  return ok;
+}
+
 // Device address of g_noalloc_scratch on the current device, looked up once per
-// device (cudaGetSymbolAddress, checked); nullptr if the lookup failed.
+// device (cudaGetSymbolAddress, checked) together with the loading of the
+// entry point's kernels; nullptr if either failed.
 void* noalloc_scratch() {
   static std::mutex mu;
   static void* addr[64] = {};
@@ -451,6 +461,7 @@ void* noalloc_scratch() {
   if (addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    if (!noalloc_load_kernels()) return nullptr;
     addr[dev] = p;
   }
   return addr[dev];
@@ -475,7 +486,6 @@ const char* sla_status_string(int status) {
     case SLA_ERR_CUDA: return "CUDA error";
     case SLA_ERR_OOM: return "out of device memory";
     case SLA_ERR_TIMEOUT: return "a kernel wait timed out";
-    case SLA_ERR_INEXACT_MEAN: return "K channel mean not proven exact";
     case SLA_ERR_SCRATCH_LIMIT: return "problem larger than the fixed no-allocation scratch buffer";
     case SLA_ERR_SMEM_LAYOUT: return "a kernel could not place its shared-memory tiles";
     default: return "unknown status";
@@ -547,11 +557,13 @@ int sla_mask_noalloc(const void* q, const void* k, int32_t* blk_idx, uint8_t* bi
   });
 }
 
-int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, void* out, float* o_sparse,
-                int B, int H, int N, int d, int block, float topk_frac, void* stream) {
+int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, void* out, int out_dtype,
+                float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, float topk_frac,
+                void* stream) {
   if (!q || !k || !v || !proj || !out) return SLA_ERR_INVALID_ARG;
+  if (out_dtype != SLA_OUT_BF16 && out_dtype != SLA_OUT_F32) return SLA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj) || !aligned16(out) ||
-      !aligned16(o_sparse))
+      !aligned16(o_sparse) || !aligned16(o_lin))
     return SLA_ERR_INVALID_ARG;
   if (!frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
   Shape s;
@@ -567,14 +579,14 @@ int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, v
   return with_dims(d, block, [&](auto D_, auto B_) {
     constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
     return run_attn<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                            static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(proj),
-                            static_cast<float*>(out), o_sparse, w, st);
+                            static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(proj), out,
+                            out_dtype == SLA_OUT_F32, o_sparse, o_lin, w, st);
   });
 }
 
 int sla_attn(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N, int d,
              int block, float topk_frac, void* stream) {
-  return sla_attn_ex(q, k, v, proj, out, nullptr, B, H, N, d, block, topk_frac, stream);
+  return sla_attn_ex(q, k, v, proj, out, SLA_OUT_BF16, nullptr, nullptr, B, H, N, d, block, topk_frac, stream);
 }
 
 int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N,
@@ -584,7 +596,7 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
   Shape s;
   int rc = check_shape(B, H, N, d, block, &s);
   if (rc) return rc;
-  const size_t tb = (size_t)s.BH * N * d * 2, ob = (size_t)s.BH * N * d * 4, pb = (size_t)d * d * 2;
+  const size_t tb = (size_t)s.BH * N * d * 2, ob = tb, pb = (size_t)d * d * 2;
   cudaStream_t st = nullptr;
   if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return SLA_ERR_CUDA;
   char* buf = nullptr;
@@ -655,7 +667,6 @@ int sla_get_error(void* stream) {
   if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return SLA_ERR_CUDA;
   if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SLA_ERR_CUDA;
   if (word & DEV_ERR_TIMEOUT) return SLA_ERR_TIMEOUT;
-  if (word & DEV_ERR_INEXACT) return SLA_ERR_INEXACT_MEAN;
   if (word & DEV_ERR_LAYOUT) return SLA_ERR_SMEM_LAYOUT;
   return SLA_OK;
 }

@@ -42,6 +42,12 @@ def mask_mismatch(gpu_idx: np.ndarray, ref_idx: np.ndarray, near_tie: np.ndarray
     return diff, bad
 
 
+def mask_record(case: str, near_tie: np.ndarray, diff: np.ndarray, bad: np.ndarray) -> dict:
+    """Structured count of the mask comparison of one case."""
+    return {"case": case, "rows": int(near_tie.size), "near_tie_rows": int(near_tie.sum()),
+            "differing_rows": int(diff.sum()), "differing_off_near_tie": int(bad.sum())}
+
+
 def sample_items(B, H, nblk, per_head=4, seed=0):
     """Query blocks to check at full size: first, last and a few seeded ones per head."""
     rng = np.random.default_rng(seed)

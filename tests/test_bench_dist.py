@@ -53,7 +53,23 @@ def test_single_process_helpers():
     assert bench.reduce_max(3.5, None) == 3.5
     assert bench.weak_scaling_value(1e12, 1, 0.5) == 2.0
     assert bench.dense_equivalent_ops(1, 12, 32768, 128) == 4.0 * 12 * 32768 ** 2 * 128
-    qk, pv = bench.critical_ops(1, 12, 32768, 128, 128, 26)
+    import numpy as np
+
+    # every block full: 2 * block^2 * d per kept pair, for QK^T and for PV
+    idx = np.tile(np.arange(26, dtype=np.int32), (1, 12, 256, 1))
+    qk, pv = bench.critical_ops(idx, 32768, 128, 128)
     assert qk == pv == 12 * 256 * 26 * 2.0 * 128 * 128 * 128
     peak, _ = bench.attn_roofline(qk, pv, {"bf16_tflops": 1000.0})
     assert peak == pytest.approx(2 / (1 / 2000.0 + 1 / 1000.0))
+    # a partial last block (N = 300, block 128: sizes 128, 128, 44) counts its valid rows and keys
+    idx = np.array([[[[0, 2], [1, 2], [0, 1]]]], dtype=np.int32)
+    qk, _ = bench.critical_ops(idx, 300, 64, 128)
+    assert qk == 2.0 * 64 * (128 * (128 + 44) + 128 * (128 + 44) + 44 * (128 + 128))
+    # the whole-call roofline takes the slower of the tensor and HBM bounds
+    r = bench.call_roofline(2e12, 1e12, 6.5e9, 2.0, {"bf16_tflops": 1000.0, "hbm_gbs": 6500.0})
+    assert r["bound"] == "tensor" and r["t_roof_ms"] == pytest.approx(2.0) and r["frac"] == pytest.approx(1.0)
+    r = bench.call_roofline(2e9, 1e9, 6.5e9, 2.0, {"bf16_tflops": 1000.0, "hbm_gbs": 6500.0})
+    assert r["bound"] == "hbm" and r["t_roof_ms"] == pytest.approx(1.0) and r["frac"] == pytest.approx(0.5)
+    assert bench.algorithmic_bytes(1, 12, 32768, 128, 256, 26) == (
+        12 * 32768 * 128 * 12 + 2 * 12 * 256 * (128 * 128 + 128) * 4)
+    assert bench.algorithmic_bytes(1, 12, 32768, 128, 256, 256) == 12 * 32768 * 128 * 12

@@ -1,5 +1,9 @@
 """CUDA path vs the CPU oracle, element by element, through the C interface.
 
+The oracle here is the plain C++ one (oracle/sla_oracle.cpp, through
+oracle/cpp_oracle.py), pinned by tests/test_oracle_pins.py together with the
+numpy statement it restates.
+
 Integer work (INT8 codes, scales, the channel mean, the block lists) must be
 bit-exact; a block list may differ only on a row the oracle marks as a near
 tie, and then the oracle is re-run with the GPU's list for that row.  The
@@ -7,13 +11,16 @@ float32 output must be within max-abs 2e-2, mean-abs 2e-3 and cosine 0.9999
 of the oracle's float64 output.
 """
 
+import json
+
 import numpy as np
 import pytest
 
-import oracle as O
+from oracle import cpp_oracle as O
+from oracle import sla_oracle as NP
 from synth import CONFIGS, make_inputs, make_workload
-from tests.parity import (assert_out_ok, compare_out, mask_mismatch, sample_items,
-                          to_dev)
+from tests.parity import (MAX_ABS, MEAN_ABS, MIN_COS, assert_out_ok, compare_out, mask_mismatch,
+                          mask_record, sample_items, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -47,41 +54,95 @@ def check_quant(got, ref):
 
 
 def run_attn(S, x, block, frac):
+    """The operator through the C interface: float32 out with both parts
+    (sla_attn_ex), the default bf16 out (sla_attn) and the block lists."""
     import torch
 
     q, k, v, w = (to_dev(x[t]) for t in ("q", "k", "v", "proj"))
     B, H, N, d = x["q"].shape
-    osp = torch.empty((B, H, N, d), dtype=torch.float32, device="cuda")
-    out = S.sla_attn(q, k, v, w, block=block, topk_frac=frac, o_sparse=osp)
+
+    def f32():
+        return torch.full((B, H, N, d), float("nan"), dtype=torch.float32, device="cuda")
+
+    out, osp, olin = f32(), f32(), f32()
+    S.sla_attn(q, k, v, w, block=block, topk_frac=frac, out=out, o_sparse=osp, o_lin=olin)
+    ob = S.sla_attn(q, k, v, w, block=block, topk_frac=frac)
+    assert ob.dtype == torch.bfloat16
     idx = S.sla_mask(q, k, block, frac)
     assert S.get_error() == 0
-    return out.cpu().numpy().astype(np.float64), osp.cpu().numpy().astype(np.float64), idx.cpu().numpy()
+    got = {"out": out, "o_sparse": osp, "o_lin": olin, "out_bf16": ob.float()}
+    return {key: t.cpu().numpy().astype(np.float64) for key, t in got.items()}, idx.cpu().numpy()
 
 
-def check_attn(x, block, frac, items=None):
-    """Full comparison (items None) or on sampled query blocks."""
+def check_attn(x, block, frac, items=None, case="?"):
+    """Full comparison (items None) or on sampled query blocks.
+
+    Returns (out stats, o_sparse stats, mask record).  The mask record counts
+    the query rows the oracle marks as near ties and the rows whose GPU list
+    differs from the oracle's; every differing row must be a near tie, and
+    near ties must stay rare (at most 1% of the rows), else the bit-exact
+    mask comparison would mean little.  The float32 output and its two parts
+    (O_sparse; O_lin . W_proj) are held to the output tolerance against the
+    oracle's float64 values; the bf16 output must be the float32 output rounded
+    to bf16, and within the tolerance of the oracle's rounded output (see
+    check_bf16)."""
     import int8_block_sparse_b200 as S
 
-    out, osp, gidx = run_attn(S, x, block, frac)
+    got, gidx = run_attn(S, x, block, frac)
     B, H, N, d = x["q"].shape
     ref_mask = O.block_mask(x["q"], x["k"], block, frac)
     diff, bad = mask_mismatch(gidx, ref_mask["idx"], ref_mask["near_tie"])
+    rec = mask_record(case, ref_mask["near_tie"], diff, bad)
+    print(json.dumps(rec))
     assert not bad.any(), f"{int(bad.sum())} block lists differ off near ties"
+    assert rec["near_tie_rows"] <= 0.01 * rec["rows"], rec
     override = {tuple(int(t) for t in ix): gidx[tuple(ix)] for ix in np.argwhere(diff)}
     res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, frac, items=items,
                           idx_override=override or None)
-    got, ref, gs, rs = [], [], [], []
+    w64 = O.bf16_to_f64(x["proj"])
+    parts = {"out": [], "o_sparse": [], "o_lin": [], "out_bf16": []}
+    refs = {"out": [], "o_sparse": [], "o_lin": []}
     for (b, h, i), o in res["out"].items():
         lo, hi = i * block, min(N, (i + 1) * block)
-        got.append(out[b, h, lo:hi])
-        ref.append(o)
-        gs.append(osp[b, h, lo:hi])
-        rs.append(res["o_sparse"][(b, h, i)])
-    st = compare_out(np.concatenate(got), np.concatenate(ref))
-    st_sp = compare_out(np.concatenate(gs), np.concatenate(rs))
+        for key in parts:
+            parts[key].append(got[key][b, h, lo:hi])
+        refs["out"].append(o)
+        refs["o_sparse"].append(res["o_sparse"][(b, h, i)])
+        refs["o_lin"].append(res["o_lin"][(b, h, i)] @ w64)
+    cat = {key: np.concatenate(v) for key, v in parts.items()}
+    ref = {key: np.concatenate(v) for key, v in refs.items()}
+    st = compare_out(cat["out"], ref["out"])
+    st_sp = compare_out(cat["o_sparse"], ref["o_sparse"])
+    st_lin = compare_out(cat["o_lin"], ref["o_lin"]) if np.any(ref["o_lin"]) else None
     assert_out_ok(st_sp, "o_sparse")
+    if st_lin is not None:
+        assert_out_ok(st_lin, "o_lin")
+    else:
+        assert not np.any(cat["o_lin"]), "no linear part, yet o_lin is not zero"
     assert_out_ok(st, "out")
-    return st, st_sp, int(diff.sum())
+    st_b = check_bf16(cat["out_bf16"], cat["out"], ref["out"])
+    print(json.dumps({"case": case, "out": st, "o_sparse": st_sp, "o_lin": st_lin, "out_bf16": st_b}))
+    return st, st_sp, rec
+
+
+def check_bf16(got_b, got_f32, ref):
+    """The bf16 output: exactly the float32 result of the same operator rounded
+    to bf16 (round to nearest even; both outputs come from the same kernel,
+    which differs only in the store), and close to the oracle's float64 output
+    rounded to bf16 the same way: mean-abs and cosine within the output
+    tolerance, and per element within the max-abs tolerance or one bf16 step
+    of the rounded value, whichever is larger (where the float32 error
+    straddles a rounding boundary the two roundings land one step apart, and a
+    step is 2^-5 already at |out| >= 4)."""
+    assert np.array_equal(got_b, O.round_bf16(got_f32)), "bf16 out is not the rounded float32 out"
+    ref_b = O.round_bf16(ref)
+    st = compare_out(got_b, ref_b)
+    assert st["mean_abs"] <= MEAN_ABS and st["cos"] >= MIN_COS, ("out_bf16", st)
+    mag = np.maximum(np.abs(ref_b), 2.0 ** -126)
+    step = np.exp2(np.floor(np.log2(mag)) - 7)
+    assert np.all(np.abs(got_b - ref_b) <= np.maximum(MAX_ABS, step)), ("out_bf16", st)
+    st["equal_to_rounded_oracle"] = float(np.mean(got_b == ref_b))
+    return st
 
 
 # ---------------------------------------------------------------- small cases
@@ -111,7 +172,7 @@ def test_quant_bitexact_small(S, B, H, N, d, block, frac, dist, seed):
 def test_attention_small(S, B, H, N, d, block, frac, dist, seed):
     grid = (4, 32, 32) if dist == "field" else None
     x = make_inputs(B, H, N, d, seed, dist, grid)
-    check_attn(x, block, frac)
+    check_attn(x, block, frac, case=f"small-{seed}")
 
 
 def test_mask_bitmap_and_list_agree(S):
@@ -153,7 +214,7 @@ def test_host_buffers_match_device_path(S):
     dev = [to_dev(x[t]) for t in ("q", "k", "v", "proj")]
     out_dev = S.sla_attn(*dev, block=128, topk_frac=0.25)
     host = [t.cpu().pin_memory() for t in dev]
-    out_host = torch.empty(host[0].shape, dtype=torch.float32).pin_memory()
+    out_host = torch.empty(host[0].shape, dtype=torch.bfloat16).pin_memory()
     S.sla_attn_host(*host, out_host, block=128, topk_frac=0.25)
     assert torch.equal(out_host, out_dev.cpu())
 
@@ -175,8 +236,8 @@ def _full_case(S, name, per_head):
     x = make_workload(w)
     check_quant(run_quant(S, x, w.block), O.quantize(x["q"], x["k"], w.block))
     items = sample_items(w.B, w.H, w.nblk, per_head=per_head, seed=w.seed)
-    st, st_sp, ndiff = check_attn(x, w.block, w.topk_frac, items=items)
-    print(f"{name}: out {st} o_sparse {st_sp} near-tie rows with other lists: {ndiff}")
+    st, st_sp, rec = check_attn(x, w.block, w.topk_frac, items=items, case=name)
+    print(json.dumps({"case": name, "out": st, "o_sparse": st_sp}))
 
 
 def test_full_tiny(S):
@@ -200,6 +261,42 @@ def test_full_720p(S):
     _full_case(S, "720p", per_head=2)
 
 
+def _wide_exponent_inputs(N, d, seed):
+    """K whose channels span more exponents than a float64 sum holds exactly:
+    the channel mean must still be the exact mean rounded once to float32."""
+    from synth.workloads import f32_to_bf16_bits
+
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    k = rng.standard_normal((1, 1, N, d)).astype(np.float32) + 3.0
+    # channel 0: 2^100, 1, -2^100 among zeros (exact sum 1)
+    k[..., :, 0] = 0.0
+    k[..., 5, 0], k[..., N // 2, 0], k[..., N - 1, 0] = 2.0 ** 100, 1.0, -(2.0 ** 100)
+    # channel 1: magnitudes near 8 and near 2^-30, random signs
+    mag = np.where(rng.random(N) < 0.5, 8.0, 2.0 ** -30) * rng.uniform(1.0, 2.0, N)
+    k[0, 0, :, 1] = mag * rng.choice([-1.0, 1.0], N)
+    # channel 2: near the largest bf16 value, alternating signs, and tiny values
+    k[0, 0, :, 2] = np.where(np.arange(N) % 3 == 0, 1e-30, 3.0e38) * np.where(np.arange(N) % 2, -1.0, 1.0)
+    kb = f32_to_bf16_bits(k)
+    # channel 3: bf16 subnormals (raw patterns) with a few values of 1
+    sub = rng.integers(1, 128, N).astype(np.uint16) | (rng.integers(0, 2, N).astype(np.uint16) << 15)
+    sub[:: max(1, N // 7)] = 0x3F80
+    kb[0, 0, :, 3] = sub
+    # channel 4: every value is -0.0
+    kb[0, 0, :, 4] = 0x8000
+    return f32_to_bf16_bits(q), kb
+
+
+@pytest.mark.parametrize("N,d,block", [(32768, 128, 128), (1000, 64, 64), (777, 128, 128)])
+def test_channel_mean_exact_for_wide_exponent_spans(S, N, d, block):
+    qb, kb = _wide_exponent_inputs(N, d, seed=N)
+    got = run_quant(S, {"q": qb, "k": kb}, block)
+    ref = O.quantize(qb, kb, block)
+    check_quant(got, ref)
+    # channel 0 sums to exactly 1, so its mean is 1/N rounded once
+    assert got["mu"][0, 0, 0] == np.float32(NP.round_rational_to_f32(1, N))
+
+
 def test_bounded_wait_reports_timeout_and_context_survives(S):
     """A kernel whose barrier is never completed gives up after its bounded wait,
     records SLA_ERR_TIMEOUT and returns; the context stays usable."""
@@ -212,4 +309,4 @@ def test_bounded_wait_reports_timeout_and_context_survives(S):
     assert S.get_error() == 5
     assert S.get_error() == 0            # the error word was cleared
     x = make_inputs(1, 1, 256, 128, 6)
-    check_attn(x, 128, 0.5)              # the device still computes correctly
+    check_attn(x, 128, 0.5, case="after-timeout")   # the device still computes correctly

@@ -66,6 +66,34 @@ def test_noalloc_mask_matches_sla_mask_on_two_calls():
         assert np.array_equal(got_bm, ref_bm.cpu().numpy())
 
 
+def test_noalloc_mask_leaves_device_memory_untouched():
+    """After the first call on the device (its set-up), a call with another
+    shape changes neither the device's free memory nor the library's pool."""
+    import torch
+
+    import int8_block_sparse_b200 as S
+    from int8_block_sparse_b200.build import build
+
+    build()
+    x1 = make_inputs(1, 2, 1500, 128, 8)
+    x2 = make_inputs(2, 2, 700, 64, 9)
+    q1, k1 = _dev(x1["q"]), _dev(x1["k"])
+    q2, k2 = _dev(x2["q"]), _dev(x2["k"])
+    _noalloc(S, q1, k1, 128, 0.2)                     # set-up call
+    idx = torch.empty((2, 2, 11, S.topk_count(700, 64, 0.3)), dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    rc = S.lib().sla_mask_noalloc(ctypes.c_void_p(q2.data_ptr()), ctypes.c_void_p(k2.data_ptr()),
+                                  ctypes.c_void_p(idx.data_ptr()), None, 2, 2, 700, 64, 64, ctypes.c_float(0.3),
+                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert S.get_error() == 0
+    ref = S.sla_mask(q2, k2, 64, 0.3).cpu().numpy()
+    assert np.array_equal(idx.cpu().numpy(), ref)
+
+
 def test_noalloc_mask_refuses_problems_beyond_its_buffer():
     import int8_block_sparse_b200 as S
 
