@@ -116,7 +116,8 @@ int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, in
  * mask needs live in one file-scope device buffer of
  * SLA_NOALLOC_SCRATCH_BYTES (16 MiB) in this library, which every GPU that
  * loads the library holds until the process exits.  A problem must fit in
- * it: 26 * B*H*nblk*d + 4 * B*H*d bytes, each part rounded up to 256 bytes
+ * it: 26 * B*H*nblk*d + 4 * B*H*d bytes (nblk rounded up to an even count in
+ * 8 * B*H*nblk*d of them), each part rounded up to 256 bytes
  * (for example B*H = 12, nblk = 256, d = 128 fits; B*H = 40, nblk = 591
  * does not); larger ones return SLA_ERR_SCRATCH_LIMIT before any work is
  * enqueued.
@@ -158,8 +159,12 @@ int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, v
                 void* stream);
 
 /* sla_attn on HOST buffers (pageable or pinned): copies q, k, v, proj to the
- * device, runs the operator on an internal stream of the current device,
- * copies out (bf16) back and returns when it is in host memory. */
+ * device, runs the operator and copies out (bf16) back, and returns when the
+ * result is in host memory.  The (batch, head) pairs are processed in up to
+ * six chunks spread over three streams of the current device (created at the
+ * first call on that device and kept), so that with pinned host buffers one
+ * chunk's copies overlap another chunk's operator; the result is the same as
+ * sla_attn's.  Calls on the same device are serialised. */
 int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
                   int N, int d, int block, float topk_frac);
 

@@ -26,8 +26,14 @@
 //                one more block; a K stage is released when its block's QK^T
 //                products finish, a V stage when its PV products finish)
 //   warp 1 / 3   tcgen05.mma issuer of tile 0 / 1
-//   warps 4-7    softmax + epilogue of tile 0 (thread = query row = TMEM lane)
-//   warps 8-11   softmax + epilogue of tile 1
+//   warps 4-7    softmax of tile 0 (thread = query row = TMEM lane)
+//   warps 8-11   softmax of tile 1
+//   warps 12-15  output warpgroup of both tiles (thread = query row): den and
+//                A of the linear part, then the epilogue O / l -> out
+// The softmax warpgroups hand each row's l over through shared memory, so
+// they go on to the next item while the output warpgroup finishes this one.
+// Registers are split with setmaxnreg: 80 per thread for warps 0-3, 144 for
+// the other three warpgroups (512 threads x 128 at launch = 65536).
 // A tile walks its key blocks in halves of 64 keys.  TMEM (512 columns): tile
 // u owns columns [256u, 256u+256): two S buffers of 64 columns (S for half h
 // goes to buffer h % 2; P, bf16, is written over the first 32 columns of its
@@ -67,8 +73,9 @@ struct AttnCfg {
   static constexpr int V_BYTES = BLK * D * 2;    // bf16
   static constexpr int STAGES = 2;
   static constexpr int TILE_BYTES = Q_BYTES + STAGES * (K_BYTES + V_BYTES);
-  static constexpr int BAR_BYTES = 2 * 20 * 8 + 16;         // two TileBars, TMEM slot, abort flag
-  static constexpr int SMEM_USED = 2 * TILE_BYTES + BAR_BYTES;
+  static constexpr int BAR_BYTES = 2 * 22 * 8 + 16;         // two TileBars, TMEM slot, abort flag
+  static constexpr int L_BYTES = 2 * 128 * 4;               // l of every row of both tiles
+  static constexpr int SMEM_USED = 2 * TILE_BYTES + BAR_BYTES + L_BYTES;
   static constexpr int SMEM_LIMIT = 232448;                  // 227 KB per CTA
   static_assert(SMEM_USED <= SMEM_LIMIT, "tile rings do not fit in shared memory");
   // room to round the base up to 1024 bytes where the limit allows (checked at
@@ -94,7 +101,14 @@ struct TileBars {
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   uint64_t mma_drain;   // end of the MMA issuer: every MMA it issued has finished
   uint64_t a_full;      // A of the linear part is in TMEM
+  uint64_t l_full;      // the softmax has finished the item: l is in shared memory
+  uint64_t pad;
 };
+
+constexpr int kAttnThreads = 512;
+constexpr uint32_t kRegsLoad = 80;    // warps 0-3: TMA producers, MMA issuers
+constexpr uint32_t kRegsMath = 144;   // warps 4-15: softmax, output
+static_assert(128 * (kRegsLoad + 3 * kRegsMath) <= 65536, "register split within the launch's registers");
 
 // The running row maximum is raised (and O, l rescaled) only when a new
 // maximum exceeds it by more than this many powers of two; until then P may
@@ -137,7 +151,7 @@ __device__ __forceinline__ float linear_den(const __nv_bfloat16* qrow, const flo
 }
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant__ CUtensorMap tm_q,
                                                  const __grid_constant__ CUtensorMap tm_k,
                                                  const __grid_constant__ CUtensorMap tm_v,
                                                  const __grid_constant__ CUtensorMap tm_g, const AttnParams p) {
@@ -146,7 +160,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  static_assert(sizeof(TileBars) == 20 * 8, "barrier block size");
+  static_assert(sizeof(TileBars) == 22 * 8, "barrier block size");
   if (uint32_t(base - smem_raw) + C::SMEM_USED > dynamic_smem_bytes()) {
     if (threadIdx.x == 0) raise_error(DEV_ERR_LAYOUT);
     return;   // uniform: every thread sees the same base
@@ -154,6 +168,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
   TileBars* bars = reinterpret_cast<TileBars*>(base + 2 * C::TILE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* l_buf = reinterpret_cast<float*>(base + 2 * C::TILE_BYTES + C::BAR_BYTES);   // [2][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -166,6 +181,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
       mbar_init(&b.o_free, 128);
       mbar_init(&b.mma_drain, 1);
       mbar_init(&b.a_full, 128);
+      mbar_init(&b.l_full, 128);
       for (int s = 0; s < 2; ++s) {
         mbar_init(&b.s_full[s], 1);
         mbar_init(&b.p_full[s], 128);
@@ -193,6 +209,11 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
   const int tiles_total = 2 * gridDim.x;
   const bool sparse = p.sparse != 0, lin = p.lin != 0;
   const int H = sparse ? kc * NH : 0;   // halves per item
+
+  if (warp < 4)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLoad));
+  else
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsMath));
 
   if (warp < 4) {
     const int u = warp >> 1;
@@ -346,7 +367,7 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
         (void)mbar_wait(&b.mma_drain, 0, nullptr);
       }
     }
-  } else {
+  } else if (warp < 12) {
     // -------------------------------------------------------------- softmax
     const int u = (warp - 4) >> 2;
     TileBars& b = bars[u];
@@ -354,25 +375,15 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem_base + u * 256 + lane_off;
     const uint32_t tO = tS + 128;
-    uint32_t item_it = 0, hg = 0;
+    uint32_t hg = 0;
     bool ok = true;
     const int part_rows = p.N % BLK;                // rows of a partial last block (0: none)
-    for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
+    for (int item = blockIdx.x * 2 + u; sparse && item < p.items && ok; item += tiles_total) {
       const int bh = item / NB, i = item % NB;
-      const long long n = (long long)i * BLK + r;
-      const bool valid = r < BLK && n < p.N;
-      const __nv_bfloat16* qrow = p.q + ((long long)bh * p.N + (valid ? n : 0)) * D;
-      const float* grow = p.zrest + ((long long)bh * NB + i) * D;
-      // running maximum m (log2 domain) and normaliser l of this row
-      float m = -INFINITY, l = sparse ? 0.f : 1.f;
-      float den = 0.f;
-      if (lin) {
-        if (!sparse) den = linear_den<D>(qrow, grow, valid);
-        else if (valid)   // read after the first half
-          for (int c = 0; c < D; c += 64) asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + c));
-      }
-      const float sq_i = sparse ? __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale : 0.f;
+      const float sq_i = __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale;
       const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
+      // running maximum m (log2 domain) and normaliser l of this row
+      float m = -INFINITY, l = 0.f;
       float cl = 0.f;
       int jl = 0;
       for (int x = 0; x < H; ++x) {
@@ -479,40 +490,101 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&b.p_full[g & 1]);
-        // den of the linear part, while the tensor core runs this half's PV
-        if (lin && x == 0) den = linear_den<D>(qrow, grow, valid);
       }
       if (!ok) break;
+      hg += H;
+      // hand l over: the output warpgroup reads it before it releases O
+      // (o_free), which the next item's first PV waits for
+      l_buf[u * 128 + r] = l;
+      mbar_arrive(&b.l_full);
+    }
+  } else {
+    // -------------------------------------------------------------- output
+    // Rounds of items, one of each tile.  Per tile u:
+    //   A(u): once the softmax has finished the item (l_full), A of the
+    //         linear part goes to TMEM (a_full);
+    //   E(u): once O is final (o_full), the epilogue O / l -> out (o_free).
+    // Order: A(0), A(1) if tile 1 is already done, E(0), A(1) otherwise,
+    // E(1), then den of both tiles' next items, which no tile waits for then:
+    // tile 0's next first PV (o_free) never waits for tile 1.
+    const int r = tid - 384;                        // query row inside a tile = TMEM lane
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    uint32_t hgs[2] = {0u, 0u};
+    float den[2] = {0.f, 0.f}, lrow[2] = {1.f, 1.f};
+    bool ok = true;
+    int it = 0;
+    auto row_of = [&](int u, int round, int& bh, int& i, long long& n) {
+      const int item = blockIdx.x * 2 + u + round * tiles_total;
+      bh = item / NB;
+      i = item % NB;
+      n = (long long)i * BLK + r;
+      return r < BLK && n < p.N;                    // a row of the output
+    };
+    auto has = [&](int u, int round) { return blockIdx.x * 2 + u + round * tiles_total < p.items; };
+    auto make_dens = [&](int round) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (has(u, round)) {
+          int bh, i;
+          long long n;
+          const bool valid = row_of(u, round, bh, i, n);
+          den[u] = linear_den<D>(p.q + ((long long)bh * p.N + (valid ? n : 0)) * D,
+                                 p.zrest + ((long long)bh * NB + i) * D, valid);
+        }
+    };
+    // A of tile u (after its softmax); false if a wait gave up
+    auto do_a = [&](int u) -> bool {
+      TileBars& b = bars[u];
+      if (sparse) {
+        if (!mbar_wait(&b.l_full, it & 1, abort_flag)) return false;
+        lrow[u] = l_buf[u * 128 + r];
+      }
       if (lin) {
-        // A = bf16(phi(q) * l / den) into the S buffer of half hg + H, once the
-        // PV that last read that buffer (half hg + H - 2 of this item) is done;
-        // an earlier reader finished before the previous o_full
-        const float sc = (valid && den > 0.f) ? l / den : 0.f;
+        int bh, i;
+        long long n;
+        const bool valid = row_of(u, it, bh, i, n);
+        // A = bf16(phi(q) * l / den) into the S buffer of half hg + H, once
+        // the PV that last read that buffer (half hg + H - 2 of this item) is
+        // done; an earlier reader finished before the previous o_full
+        const float sc = (valid && den[u] > 0.f) ? lrow[u] / den[u] : 0.f;
+        const uint4* qr = reinterpret_cast<const uint4*>(p.q + ((long long)bh * p.N + (valid ? n : 0)) * D);
         uint32_t a[D / 2];
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) {
-          const uint4 raw = valid ? __ldg(reinterpret_cast<const uint4*>(qrow) + c8) : make_uint4(0, 0, 0, 0);
-          a[4 * c8 + 0] = pack_bf16x2(phi_bf16(uint16_t(raw.x)) * sc, phi_bf16(uint16_t(raw.x >> 16)) * sc);
-          a[4 * c8 + 1] = pack_bf16x2(phi_bf16(uint16_t(raw.y)) * sc, phi_bf16(uint16_t(raw.y >> 16)) * sc);
-          a[4 * c8 + 2] = pack_bf16x2(phi_bf16(uint16_t(raw.z)) * sc, phi_bf16(uint16_t(raw.z >> 16)) * sc);
-          a[4 * c8 + 3] = pack_bf16x2(phi_bf16(uint16_t(raw.w)) * sc, phi_bf16(uint16_t(raw.w >> 16)) * sc);
+          const uint4 raw = valid ? __ldg(qr + c8) : make_uint4(0, 0, 0, 0);
+          a[4 * c8] = raw.x;
+          a[4 * c8 + 1] = raw.y;
+          a[4 * c8 + 2] = raw.z;
+          a[4 * c8 + 3] = raw.w;
         }
+#pragma unroll
+        for (int c = 0; c < D / 2; ++c)
+          a[c] = pack_bf16x2(phi_bf16(uint16_t(a[c])) * sc, phi_bf16(uint16_t(a[c] >> 16)) * sc);
         if (H >= 2) {
-          const uint32_t gp = hg + H - 2;
-          if (!(ok = mbar_wait(&b.pv_done[gp & 1], (gp >> 1) & 1, abort_flag))) break;
+          const uint32_t gp = hgs[u] + H - 2;
+          if (!mbar_wait(&b.pv_done[gp & 1], (gp >> 1) & 1, abort_flag)) return false;
         }
         tc_fence_after();
-        const uint32_t abuf = tS + ((hg + H) & 1) * 64;
+        const uint32_t abuf = tmem_base + u * 256 + lane_off + ((hgs[u] + H) & 1) * 64;
 #pragma unroll
         for (int c = 0; c < D / 2; c += 16) SLA_TMEM_ST16(abuf + c, (a + c));
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&b.a_full);
       }
-      hg += H;
-      if (!(ok = mbar_wait(&b.o_full, item_it & 1, abort_flag))) break;
+      hgs[u] += H;
+      return true;
+    };
+    // epilogue of tile u; false if the wait gave up
+    auto do_e = [&](int u) -> bool {
+      TileBars& b = bars[u];
+      if (!mbar_wait(&b.o_full, it & 1, abort_flag)) return false;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      int bh, i;
+      long long n;
+      const bool valid = row_of(u, it, bh, i, n);
+      const uint32_t tO = tmem_base + u * 256 + lane_off + 128;
+      const float inv_l = 1.f / lrow[u];
       const long long obase = ((long long)bh * p.N + n) * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
@@ -530,15 +602,31 @@ __global__ void __launch_bounds__(384, 1) k_attn(const __grid_constant__ CUtenso
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + obase + ch * 32);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(pack_bf16x2(__uint_as_float(w[8 * q]) * inv_l, __uint_as_float(w[8 * q + 1]) * inv_l),
-                                  pack_bf16x2(__uint_as_float(w[8 * q + 2]) * inv_l, __uint_as_float(w[8 * q + 3]) * inv_l),
-                                  pack_bf16x2(__uint_as_float(w[8 * q + 4]) * inv_l, __uint_as_float(w[8 * q + 5]) * inv_l),
-                                  pack_bf16x2(__uint_as_float(w[8 * q + 6]) * inv_l, __uint_as_float(w[8 * q + 7]) * inv_l));
+              dst[q] = make_uint4(
+                  pack_bf16x2(__uint_as_float(w[8 * q]) * inv_l, __uint_as_float(w[8 * q + 1]) * inv_l),
+                  pack_bf16x2(__uint_as_float(w[8 * q + 2]) * inv_l, __uint_as_float(w[8 * q + 3]) * inv_l),
+                  pack_bf16x2(__uint_as_float(w[8 * q + 4]) * inv_l, __uint_as_float(w[8 * q + 5]) * inv_l),
+                  pack_bf16x2(__uint_as_float(w[8 * q + 6]) * inv_l, __uint_as_float(w[8 * q + 7]) * inv_l));
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&b.o_free);
+      return true;
+    };
+    if (lin) make_dens(0);
+    for (; ok && has(0, it); ++it) {
+      const bool t1 = has(1, it);
+      ok = do_a(0);
+      bool a1 = false;
+      if (ok && t1 && (!sparse || __all_sync(0xffffffffu, mbar_test_wait(&bars[1].l_full, it & 1)))) {
+        ok = do_a(1);
+        a1 = true;
+      }
+      ok = ok && do_e(0);
+      if (ok && t1 && !a1) ok = do_a(1);
+      if (ok && t1) ok = do_e(1);
+      if (ok && lin) make_dens(it + 1);
     }
   }
 

@@ -10,15 +10,19 @@
 //
 // One CTA handles R query blocks of one head (R <= 8: a warp per row in the
 // selection; R = 8 unless the scores of a long sequence need a smaller R to fit
-// in shared memory).  Scores: thread t takes key blocks t, t + 256, ... and computes
-// the R dot products of its key block with the R pooled query blocks (staged
-// in shared memory, read as broadcasts), each as four interleaved partial sums
-// over the channels (c mod 4) added as (a0 + a1) + (a2 + a3); its pooled key
-// block is read once, straight from global memory.  Selection: each warp turns
-// its row into order-preserving 64-bit keys and finds the kc-th largest by a
-// bitwise search over the high 32 bits (warp reductions with redux.sync), then
-// over the low 32 bits of the keys tied at that high half, if they are not all
-// kept.
+// in shared memory).  Scores: for each group of 256 key blocks, thread t takes
+// key block 256 * group + t and computes the R dot products of it with the R
+// pooled query blocks (staged in shared memory, read as broadcasts), each as
+// four interleaved partial sums over the channels (c mod 4) added as
+// (a0 + a1) + (a2 + a3).  The pooled key blocks are stored channel-major
+// (kbar[bh][c][j]); slabs of 16 channels x 256 key blocks come into a
+// double-buffered shared ring by TMA, the next slab landing while the
+// current one is used.  Selection: each warp turns its
+// row into order-preserving 64-bit keys in place (their halves also held in
+// registers when the row has at most 256 key blocks) and finds the kc-th
+// largest by a bitwise search over the high 32 bits (warp reductions with
+// redux.sync), then over the low 32 bits of the keys tied at that high half,
+// if they are not all kept.
 #pragma once
 #include "sm100.cuh"
 
@@ -29,49 +33,115 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
   return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
+// Number of the warp's keys (KPL per lane, or all NB from shared memory when
+// KPL == 0; w32[2j] low, w32[2j + 1] high half of key j) whose high half is
+// >= cand (tied: high half == th and low half >= cand).
+template <int KPL>
+__device__ __forceinline__ uint32_t count_ge(const uint32_t* hi_r, const uint32_t* lo_r, const uint32_t* w32,
+                                             int NB, int lane, bool tied, uint32_t th, uint32_t cand) {
+  uint32_t cnt = 0u;
+  if (KPL > 0) {
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      const bool in = lane + 32 * e < NB;
+      cnt += (in && (tied ? (hi_r[e] == th && lo_r[e] >= cand) : hi_r[e] >= cand)) ? 1u : 0u;
+    }
+  } else {
+    for (int j = lane; j < NB; j += 32)
+      cnt += (tied ? (w32[2 * j + 1] == th && w32[2 * j] >= cand) : w32[2 * j + 1] >= cand) ? 1u : 0u;
+  }
+  return __reduce_add_sync(0xffffffffu, cnt);
+}
+
+constexpr int kMaskSlabCh = 16;                               // channels per slab
+constexpr int kMaskSlabBytes = kMaskSlabCh * 256 * 8;          // 32 KB
+
 template <int D, int R>
-__global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, const double* __restrict__ kbar,
-                                             int NB, int kc, int32_t* __restrict__ idx, uint8_t* __restrict__ bitmap,
+__global__ void __launch_bounds__(256) k_mask(const __grid_constant__ CUtensorMap tm_kbar,
+                                             const double* __restrict__ qbar, int NB, int kc,
+                                             int32_t* __restrict__ idx, uint8_t* __restrict__ bitmap,
                                              __nv_bfloat16* __restrict__ notcrit, int ncpitch) {
   static_assert(R >= 1 && R <= 8, "one warp per row in the selection");
+  static_assert(D % kMaskSlabCh == 0, "whole slabs");
+  constexpr int SLABS = D / kMaskSlabCh;                      // slabs per group of key blocks
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  double* qb = reinterpret_cast<double*>(smem_raw);   // [R][D]
-  double* sc = qb + R * D;                            // [R][NB]
+  double* kbuf = reinterpret_cast<double*>(smem_raw);          // [2][16][256]
+  double* qb = kbuf + 2 * kMaskSlabCh * 256;                   // [R][D]
+  double* sc = qb + R * D;                                     // [R][NB] scores, then their order keys
+  uint64_t* full = reinterpret_cast<uint64_t*>(sc + R * NB);   // [2]
 
   const long long bh = blockIdx.y;
   const int i0 = blockIdx.x * R;
   const int nrows = min(R, NB - i0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const double sqd = sqrt((double)D);
+  const int groups = (NB + 255) / 256;
+  const int total = groups * SLABS;
 
+  auto issue = [&](int n) {   // slab n: group n / SLABS, channels 16 * (n % SLABS) ..
+    const int b = n & 1;
+    mbar_expect_tx(&full[b], kMaskSlabBytes);
+    tma_load_2d(kbuf + b * kMaskSlabCh * 256, &tm_kbar, &full[b], (n / SLABS) * 256,
+                int(bh * D + (n % SLABS) * kMaskSlabCh));
+  };
+  int issued = 0;   // slabs requested (thread 0)
+  if (tid == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_kbar);
+    issue(0);
+    issued = 1;
+    if (total > 1) issue(issued++);
+  }
   for (int e = tid; e < R * D; e += 256) {
     const int r = e / D;
     qb[e] = (r < nrows) ? qbar[(bh * NB + i0) * (long long)D + e] : 0.0;
   }
   __syncthreads();
-  for (int j = tid; j < NB; j += 256) {
-    const double2* kr = reinterpret_cast<const double2*>(kbar + (bh * NB + j) * (long long)D);
-    double a[R][4];
+  double a[R][4];
+  bool ok = true;
+  for (int n = 0; n < total; ++n) {
+    const int grp = n / SLABS, slab = n % SLABS;
+    if (slab == 0) {
 #pragma unroll
-    for (int r = 0; r < R; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0.0;
-#pragma unroll 2
-    for (int c = 0; c < D; c += 4) {
-      const double2 k01 = __ldg(kr + c / 2), k23 = __ldg(kr + c / 2 + 1);
+      for (int r = 0; r < R; ++r) a[r][0] = a[r][1] = a[r][2] = a[r][3] = 0.0;
+    }
+    ok = __syncthreads_and(mbar_wait(&full[n & 1], (n >> 1) & 1, nullptr)) && ok;
+    const double* kb = kbuf + (n & 1) * kMaskSlabCh * 256;
+    if (ok) {
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const double2 q01 = *reinterpret_cast<const double2*>(qb + r * D + c);
-        const double2 q23 = *reinterpret_cast<const double2*>(qb + r * D + c + 2);
-        a[r][0] = fma(q01.x, k01.x, a[r][0]);
-        a[r][1] = fma(q01.y, k01.y, a[r][1]);
-        a[r][2] = fma(q23.x, k23.x, a[r][2]);
-        a[r][3] = fma(q23.y, k23.y, a[r][3]);
+      for (int cc = 0; cc < kMaskSlabCh; cc += 4) {
+        const int c = slab * kMaskSlabCh + cc;
+        const double k0 = kb[cc * 256 + tid], k1 = kb[(cc + 1) * 256 + tid];
+        const double k2 = kb[(cc + 2) * 256 + tid], k3 = kb[(cc + 3) * 256 + tid];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const double2 q01 = *reinterpret_cast<const double2*>(qb + r * D + c);
+          const double2 q23 = *reinterpret_cast<const double2*>(qb + r * D + c + 2);
+          a[r][0] = fma(q01.x, k0, a[r][0]);
+          a[r][1] = fma(q01.y, k1, a[r][1]);
+          a[r][2] = fma(q23.x, k2, a[r][2]);
+          a[r][3] = fma(q23.y, k3, a[r][3]);
+        }
       }
     }
+    const int j = grp * 256 + tid;
+    if (slab == SLABS - 1 && j < NB) {
 #pragma unroll
-    for (int r = 0; r < R; ++r)
-      if (r < nrows) sc[r * NB + j] = ((a[r][0] + a[r][1]) + (a[r][2] + a[r][3])) / sqd;
+      for (int r = 0; r < R; ++r)
+        if (r < nrows) sc[r * NB + j] = ((a[r][0] + a[r][1]) + (a[r][2] + a[r][3])) / sqd;
+    }
+    __syncthreads();   // the buffer of slab n is free again
+    if (!ok) break;    // uniform: a slab did not land in time (recorded as a timeout)
+    if (tid == 0 && n + 2 < total) issue(issued++);
   }
-  __syncthreads();
+  if (!ok) {
+    // slabs still in flight land before the CTA's shared memory is handed on
+    if (tid == 0)
+      for (int q = issued > 2 ? issued - 2 : 0; q < issued; ++q) (void)mbar_wait(&full[q & 1], (q >> 1) & 1, nullptr);
+    return;
+  }
 
   for (int r = warp; r < nrows; r += 8) {
     const int i = i0 + r;
@@ -80,14 +150,23 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, c
     for (int j = lane; j < NB; j += 32) rk[j] = order_key(sc[r * NB + j]);
     __syncwarp();
     const uint32_t* w32 = reinterpret_cast<const uint32_t*>(rk);   // word 2j: low half, 2j+1: high half
+    constexpr int KPL = 8;                       // register keys per lane when NB <= 256
+    const bool regs = NB <= 32 * KPL;
+    uint32_t hi_r[KPL], lo_r[KPL];
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+      const int j = lane + 32 * e;
+      hi_r[e] = (regs && j < NB) ? w32[2 * j + 1] : 0u;
+      lo_r[e] = (regs && j < NB) ? w32[2 * j] : 0u;
+    }
     // T = the kc-th largest key: first the kc-th largest high half Th, then,
     // among the keys whose high half is Th, the (kc - #above)-th largest low half
     uint32_t Th = 0u;
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = Th | (1u << bit);
-      uint32_t cnt = 0u;
-      for (int j = lane; j < NB; j += 32) cnt += (w32[2 * j + 1] >= cand) ? 1u : 0u;
-      if (__reduce_add_sync(0xffffffffu, cnt) >= (uint32_t)kc) Th = cand;
+      const uint32_t cnt = regs ? count_ge<KPL>(hi_r, lo_r, w32, NB, lane, false, 0u, cand)
+                                : count_ge<0>(hi_r, lo_r, w32, NB, lane, false, 0u, cand);
+      if (cnt >= (uint32_t)kc) Th = cand;
     }
     uint32_t above = 0u, tied = 0u, tied_min = 0xFFFFFFFFu;
     for (int j = lane; j < NB; j += 32) {
@@ -107,13 +186,13 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, c
       Tl = 0u;
       for (int bit = 31; bit >= 0; --bit) {
         const uint32_t cand = Tl | (1u << bit);
-        uint32_t cnt = 0u;
-        for (int j = lane; j < NB; j += 32) cnt += (w32[2 * j + 1] == Th && w32[2 * j] >= cand) ? 1u : 0u;
-        if (__reduce_add_sync(0xffffffffu, cnt) >= need) Tl = cand;
+        const uint32_t cnt = regs ? count_ge<KPL>(hi_r, lo_r, w32, NB, lane, true, Th, cand)
+                                  : count_ge<0>(hi_r, lo_r, w32, NB, lane, true, Th, cand);
+        if (cnt >= need) Tl = cand;
       }
     }
-    const unsigned long long T = ((unsigned long long)Th << 32) | Tl;
     int gt = 0;
+    const unsigned long long T = ((unsigned long long)Th << 32) | Tl;
     for (int j = lane; j < NB; j += 32) gt += (rk[j] > T) ? 1 : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
@@ -122,12 +201,13 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, c
     int32_t* dst = idx + (bh * NB + i) * (long long)kc;
     for (int j0 = 0; j0 < NB; j0 += 32) {
       const int j = j0 + lane;
-      const unsigned long long key = (j < NB) ? rk[j] : 0ull;
       const bool inb = j < NB;
+      const unsigned long long key = inb ? rk[j] : 0ull;
       const bool eq = inb && key == T;
+      const bool great = inb && key > T;
       const unsigned eqmask = __ballot_sync(0xffffffffu, eq);
       const int eq_before = eq_seen + __popc(eqmask & ((1u << lane) - 1u));
-      const bool sel = inb && (key > T || (eq && eq_before < need_eq));
+      const bool sel = great || (eq && eq_before < need_eq);
       const unsigned selmask = __ballot_sync(0xffffffffu, sel);
       if (sel) dst[out_pos + __popc(selmask & ((1u << lane) - 1u))] = j;
       if (bitmap != nullptr && inb) bitmap[(bh * NB + i) * (long long)NB + j] = sel ? 1 : 0;
@@ -146,7 +226,7 @@ __global__ void __launch_bounds__(256) k_mask(const double* __restrict__ qbar, c
 
 template <int D>
 size_t mask_smem(int rows, int NB) {
-  return (size_t(rows) * D + size_t(rows) * NB) * sizeof(double);
+  return size_t(2) * kMaskSlabBytes + (size_t(rows) * D + size_t(rows) * NB) * sizeof(double) + 2 * 8;
 }
 
 }  // namespace sla

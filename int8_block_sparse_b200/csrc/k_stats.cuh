@@ -4,7 +4,9 @@
 // writes
 //   ksum[bh][j][c]   float64 sum of the raw K values of channel c (for the
 //                    channel mean);
-//   kbar[bh][j][c]   float64 mean of those values (the pooled block of the mask);
+//   kbar[bh][c][j]   float64 mean of those values (the pooled block of the mask),
+//                    channel-major so that the mask reads contiguous channel slabs
+//                    (row pitch kbar_pitch(NB), a multiple of 16 bytes);
 //   kexp[bh][j][c]   largest and smallest bf16 exponent field among the nonzero
 //                    K values of the channel (checks that the float64 sums are
 //                    exact);
@@ -31,6 +33,10 @@ namespace sla {
 
 // phi = elu + 1: x + 1 for x > 0, exp(x) otherwise.
 __device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+// Row pitch (in doubles) of the channel-major pooled K blocks: NB rounded up
+// to an even count, so that rows start on 16-byte boundaries (TMA strides).
+__host__ __device__ __forceinline__ long long kbar_pitch(int NB) { return (NB + 1) & ~1; }
 
 // bf16 exponent field of a raw 16-bit pattern.
 __device__ __forceinline__ uint32_t bf16_exp_field(uint16_t b) { return (b >> 7) & 0xFFu; }
@@ -186,7 +192,7 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
     }
     const long long o = (bh * NB + j) * (long long)D + tid;
     ksum[o] = s;
-    kbar[o] = s / (double)rows;
+    kbar[(bh * (long long)D + tid) * kbar_pitch(NB) + j] = s / (double)rows;
     kexp[2 * o] = (uint8_t)mx;
     kexp[2 * o + 1] = (uint8_t)mn;
     if (states) hstate[(bh * (long long)NB + j) * hpitch + D * D + tid] = __float2bfloat16_rn(z);

@@ -132,7 +132,8 @@ struct Workspace {
 size_t workspace_bytes(const Shape& s, int what) {
   const size_t BH = s.BH, NB = s.NB, NP = s.NP, d = s.d, kc = s.kc;
   const size_t ncpitch = (NB + 63) / 64 * 64, hpitch = d * d + d;
-  size_t b = rounded<double>(BH * NB * d) * 3 + rounded<uint8_t>(BH * NB * d * 2) + rounded<float>(BH * d);
+  size_t b = rounded<double>(BH * NB * d) * 2 + rounded<double>(BH * d * (size_t)kbar_pitch((int)NB)) +
+             rounded<uint8_t>(BH * NB * d * 2) + rounded<float>(BH * d);
   if (what & 1) b += rounded<int8_t>(BH * NP * d) * 2 + rounded<float>(BH * NB) * 2;
   if (what & 2) b += rounded<int32_t>(BH * NB * kc);
   if (what & 8)
@@ -149,7 +150,7 @@ Workspace carve(const Shape& s, int what, char* base) {
   w.ncpitch = (NB + 63) / 64 * 64;
   w.hpitch = d * d + d;
   w.ksum = a.take<double>(BH * NB * d);
-  w.kbar = a.take<double>(BH * NB * d);
+  w.kbar = a.take<double>(BH * d * (size_t)kbar_pitch((int)NB));
   w.qbar = a.take<double>(BH * NB * d);
   w.kexp = a.take<uint8_t>(BH * NB * d * 2);
   w.mu = a.take<float>(BH * d);
@@ -203,6 +204,17 @@ struct ProfScope {
 };
 
 // ------------------------------------------------------------------ launch helpers
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <int D, int BLK>
 int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                        const __nv_bfloat16* proj, Workspace& w, bool states, bool kcodes, int8_t* qi8,
@@ -251,11 +263,20 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
 template <int D, int R>
 int launch_mask_rows(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __nv_bfloat16* notcrit,
                      cudaStream_t st) {
+  // kbar as a 2-D float64 tensor [BH * D rows][NB key blocks]; slabs of 16 rows x 256
+  CUtensorMap mkb;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)s.NB, (cuuint64_t)(s.BH * D)};
+    cuuint64_t str[1] = {(cuuint64_t)kbar_pitch((int)s.NB) * 8};
+    cuuint32_t box[2] = {256u, (cuuint32_t)kMaskSlabCh};
+    if (!make_map(&mkb, CU_TENSOR_MAP_DATA_TYPE_FLOAT64, 2, w.kbar, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return SLA_ERR_CUDA;
+  }
   const size_t sm = mask_smem<D>(R, (int)s.NB);
   cudaFuncSetAttribute(k_mask<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   dim3 g((unsigned)((s.NB + R - 1) / R), (unsigned)s.BH);
   ProfScope ps(SLA_K_MASK, st);
-  k_mask<D, R><<<g, 256, sm, st>>>(w.qbar, w.kbar, (int)s.NB, (int)s.kc, idx, bitmap, notcrit, (int)w.ncpitch);
+  k_mask<D, R><<<g, 256, sm, st>>>(mkb, w.qbar, (int)s.NB, (int)s.kc, idx, bitmap, notcrit, (int)w.ncpitch);
   return cuda_status(cudaGetLastError());
 }
 
@@ -270,16 +291,6 @@ int launch_mask(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __n
   return launch_mask_rows<D, 1>(s, w, idx, bitmap, notcrit, st);
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 // k_attn in one of its modes: sparse (the selected blocks), lin (the linear
 // part), out as float32 or bf16.
@@ -323,7 +334,7 @@ int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __nv
   cudaFuncSetAttribute(k_attn<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int ctas = (int)std::min<long long>(num_sms(), (p.items + 1) / 2);
   ProfScope ps(SLA_K_ATTN, st);
-  k_attn<D, BLK><<<ctas, 384, C::SMEM, st>>>(mq, mk, mv, mg, p);
+  k_attn<D, BLK><<<ctas, kAttnThreads, C::SMEM, st>>>(mq, mk, mv, mg, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -349,10 +360,13 @@ int launch_lingemm(const Shape& s, Workspace& w, cudaStream_t st) {
   LinGemmParams gp;
   gp.grest = w.grest; gp.zrest = w.zrest; gp.NB = (int)s.NB; gp.D = D; gp.E = D * D + D;
   gp.nkt = (int)((s.NB + 63) / 64);
+  gp.mgroups = (int)((s.NB + 255) / 256);
+  gp.ntiles = (gp.E + 127) / 128;
+  gp.units = (int)(s.BH * gp.mgroups * gp.ntiles);
   cudaFuncSetAttribute(k_lingemm, cudaFuncAttributeMaxDynamicSharedMemorySize, LG_SMEM);
-  dim3 g1((unsigned)((gp.E + 255) / 256), (unsigned)((s.NB + 127) / 128), (unsigned)s.BH);
+  const int ctas = std::min(num_sms(), gp.units);
   ProfScope ps(SLA_K_LINGEMM, st);
-  k_lingemm<<<g1, 128, LG_SMEM, st>>>(ma, mb, gp);
+  k_lingemm<<<ctas, LG_THREADS, LG_SMEM, st>>>(ma, mb, gp);
   return cuda_status(cudaGetLastError());
 }
 
@@ -465,6 +479,35 @@ void* noalloc_scratch() {
     addr[dev] = p;
   }
   return addr[dev];
+}
+
+// ------------------------------------------------------------------ host-buffer entry point
+// Streams and events of sla_attn_host, created once per device and kept (a
+// call holds the device's set for its duration).
+constexpr int kHostStreams = 3;
+constexpr long long kHostChunks = 6;
+
+struct HostStreams {
+  std::mutex mu;
+  cudaStream_t st[kHostStreams] = {};
+  cudaEvent_t ev[kHostStreams] = {};
+};
+
+HostStreams* host_streams() {
+  static std::mutex mu;
+  static HostStreams* sets[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (sets[dev] == nullptr) {
+    HostStreams* h = new HostStreams();
+    for (int i = 0; i < kHostStreams; ++i)
+      if (cudaStreamCreateWithFlags(&h->st[i], cudaStreamNonBlocking) != cudaSuccess ||
+          cudaEventCreateWithFlags(&h->ev[i], cudaEventDisableTiming) != cudaSuccess)
+        return nullptr;
+    sets[dev] = h;
+  }
+  return sets[dev];
 }
 
 }  // namespace
@@ -596,31 +639,51 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
   Shape s;
   int rc = check_shape(B, H, N, d, block, &s);
   if (rc) return rc;
-  const size_t tb = (size_t)s.BH * N * d * 2, ob = tb, pb = (size_t)d * d * 2;
-  cudaStream_t st = nullptr;
-  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return SLA_ERR_CUDA;
+  HostStreams* hs = host_streams();
+  if (hs == nullptr) return SLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(hs->mu);
+  cudaStream_t* st = hs->st;
+  const size_t head = (size_t)N * d * 2;                    // bytes of one head of q, k, v or out
+  const size_t tb = (size_t)s.BH * head, pb = (size_t)d * d * 2;
+  const size_t off = (tb + 255) & ~size_t(255), poff = (pb + 255) & ~size_t(255);
   char* buf = nullptr;
-  const size_t off = (tb + 255) & ~size_t(255), ooff = (ob + 255) & ~size_t(255), poff = (pb + 255) & ~size_t(255);
   cudaMemPool_t pool = pool_for_current_device();
-  cudaError_t e = pool ? cudaMallocFromPoolAsync(reinterpret_cast<void**>(&buf), 3 * off + ooff + poff, pool, st)
+  cudaError_t e = pool ? cudaMallocFromPoolAsync(reinterpret_cast<void**>(&buf), 4 * off + poff, pool, st[0])
                        : cudaErrorInitializationError;
-  if (e != cudaSuccess) {
-    cudaStreamDestroy(st);
-    return cuda_status(e);
-  }
-  char *dq = buf, *dk = buf + off, *dv = buf + 2 * off, *dout = buf + 3 * off, *dp = buf + 3 * off + ooff;
+  if (e != cudaSuccess) return cuda_status(e);
+  char *dq = buf, *dk = buf + off, *dv = buf + 2 * off, *dout = buf + 3 * off, *dp = buf + 4 * off;
   rc = SLA_OK;
-  if (cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(dp, proj, pb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  if (cudaMemcpyAsync(dp, proj, pb, cudaMemcpyHostToDevice, st[0]) != cudaSuccess ||
+      cudaEventRecord(hs->ev[0], st[0]) != cudaSuccess)
     rc = SLA_ERR_CUDA;
-  if (rc == SLA_OK) rc = sla_attn(dq, dk, dv, dp, dout, B, H, N, d, block, topk_frac, st);
-  if (rc == SLA_OK && cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, st) != cudaSuccess) rc = SLA_ERR_CUDA;
-  cudaFreeAsync(buf, st);
-  const cudaError_t se = cudaStreamSynchronize(st);
+  // heads in chunks over the streams: a chunk's copies in, operator and copy
+  // out are ordered on its stream; chunks on different streams overlap
+  const long long chunks = std::min<long long>(s.BH, kHostChunks);
+  const long long per = (s.BH + chunks - 1) / chunks;
+  for (long long c = 0; c < chunks && rc == SLA_OK; ++c) {
+    const long long h0 = c * per, nh = std::min<long long>(per, s.BH - h0);
+    if (nh <= 0) break;
+    cudaStream_t sc = st[c % kHostStreams];
+    const size_t o = (size_t)h0 * head, nb = (size_t)nh * head;
+    if ((c % kHostStreams != 0 && cudaStreamWaitEvent(sc, hs->ev[0], 0) != cudaSuccess) ||
+        cudaMemcpyAsync(dq + o, static_cast<const char*>(q) + o, nb, cudaMemcpyHostToDevice, sc) != cudaSuccess ||
+        cudaMemcpyAsync(dk + o, static_cast<const char*>(k) + o, nb, cudaMemcpyHostToDevice, sc) != cudaSuccess ||
+        cudaMemcpyAsync(dv + o, static_cast<const char*>(v) + o, nb, cudaMemcpyHostToDevice, sc) != cudaSuccess) {
+      rc = SLA_ERR_CUDA;
+      break;
+    }
+    rc = sla_attn(dq + o, dk + o, dv + o, dp, dout + o, 1, (int)nh, N, d, block, topk_frac, sc);
+    if (rc == SLA_OK &&
+        cudaMemcpyAsync(static_cast<char*>(out) + o, dout + o, nb, cudaMemcpyDeviceToHost, sc) != cudaSuccess)
+      rc = SLA_ERR_CUDA;
+  }
+  // join the streams, release the buffers, wait for the results
+  for (int i = 1; i < kHostStreams; ++i)
+    if (cudaEventRecord(hs->ev[i], st[i]) != cudaSuccess || cudaStreamWaitEvent(st[0], hs->ev[i], 0) != cudaSuccess)
+      if (rc == SLA_OK) rc = SLA_ERR_CUDA;
+  cudaFreeAsync(buf, st[0]);
+  const cudaError_t se = cudaStreamSynchronize(st[0]);
   if (rc == SLA_OK && se != cudaSuccess) rc = SLA_ERR_CUDA;
-  cudaStreamDestroy(st);
   return rc;
 }
 
