@@ -31,15 +31,22 @@
 
 namespace sla {
 
-// phi = elu + 1: x + 1 for x > 0, exp(x) otherwise.
-__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+// phi = elu + 1: x + 1 for x > 0, exp(x) otherwise (the fast exponential: phi
+// enters h' as bf16 and z as a float32 sum).
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+// A normal or zero bf16 value (raw bits) as a float64, built from its fields
+// (exact; subnormal bf16 values are converted by the caller instead).
+__device__ __forceinline__ double bf16_normal_to_f64(uint32_t h) {
+  const uint64_t sgn = uint64_t(h & 0x8000u) << 48;
+  const uint32_t e = (h >> 7) & 0xFFu;
+  const uint64_t bits = e ? (sgn | (uint64_t(e + 896u) << 52) | (uint64_t(h & 0x7Fu) << 45)) : sgn;
+  return __longlong_as_double((long long)bits);
+}
 
 // Row pitch (in doubles) of the channel-major pooled K blocks: NB rounded up
 // to an even count, so that rows start on 16-byte boundaries (TMA strides).
 __host__ __device__ __forceinline__ long long kbar_pitch(int NB) { return (NB + 1) & ~1; }
-
-// bf16 exponent field of a raw 16-bit pattern.
-__device__ __forceinline__ uint32_t bf16_exp_field(uint16_t b) { return (b >> 7) & 0xFFu; }
 
 template <int D, int BLK>
 struct StatsCfg {
@@ -93,7 +100,7 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
     fence_mbar_init();
   }
   if (states && warp == 0) {
-    tmem_alloc(tmem_slot, 2 * D);
+    tmem_alloc(tmem_slot, D);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -123,23 +130,37 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
   }
   double part[8];
   float zp[8];
-  uint32_t emax[8], emin[8];
+  // magnitudes (sign cleared) of channel pairs, packed 16-bit: largest, and
+  // smallest nonzero (0x7FFF = none); their exponent fields bound the channel's
+  uint32_t mxp[4], mnp[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) { part[e] = 0.0; zp[e] = 0.f; emax[e] = 0u; emin[e] = 255u; }
+  for (int e = 0; e < 8; ++e) { part[e] = 0.0; zp[e] = 0.f; }
+#pragma unroll
+  for (int w = 0; w < 4; ++w) { mxp[w] = 0u; mnp[w] = 0x7FFF7FFFu; }
 #pragma unroll
   for (int t = 0; t < NR; ++t) {
     const int r = rg + t * RG;
-    const uint16_t* kh = reinterpret_cast<const uint16_t*>(&kr[t]);
+    const uint32_t wv[4] = {kr[t].x, kr[t].y, kr[t].z, kr[t].w};
+    bool sub = false;   // a subnormal bf16 among the eight values
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t m = wv[w] & 0x7FFF7FFFu;
+      mxp[w] = __vmaxu2(mxp[w], m);
+      mnp[w] = __vminu2(mnp[w], m | (__vcmpeq2(m, 0u) & 0x7FFF7FFFu));
+      const uint32_t ez = __vcmpeq2(m & 0x7F807F80u, 0u) & ~__vcmpeq2(m, 0u);
+      sub = sub || ez != 0u;
+    }
     uint32_t pk[4];
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
-      const float k0 = __uint_as_float(uint32_t(kh[e]) << 16), k1 = __uint_as_float(uint32_t(kh[e + 1]) << 16);
-      part[e] += (double)k0;
-      part[e + 1] += (double)k1;
-      if ((kh[e] & 0x7FFFu) != 0u) { emax[e] = max(emax[e], bf16_exp_field(kh[e])); emin[e] = min(emin[e], bf16_exp_field(kh[e])); }
-      if ((kh[e + 1] & 0x7FFFu) != 0u) {
-        emax[e + 1] = max(emax[e + 1], bf16_exp_field(kh[e + 1]));
-        emin[e + 1] = min(emin[e + 1], bf16_exp_field(kh[e + 1]));
+      const uint32_t h0 = wv[e >> 1] & 0xFFFFu, h1 = wv[e >> 1] >> 16;
+      const float k0 = __uint_as_float(h0 << 16), k1 = __uint_as_float(h1 << 16);
+      if (!sub) {
+        part[e] += bf16_normal_to_f64(h0);
+        part[e + 1] += bf16_normal_to_f64(h1);
+      } else {
+        part[e] += (double)k0;
+        part[e + 1] += (double)k1;
       }
       const float p0 = (r < rows) ? phi_elu1(k0) : 0.f, p1 = (r < rows) ? phi_elu1(k1) : 0.f;
       zp[e] += p0;
@@ -165,8 +186,11 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
     for (int e = 0; e < 8; ++e) {
       part[e] += __shfl_xor_sync(0xffffffffu, part[e], o);
       zp[e] += __shfl_xor_sync(0xffffffffu, zp[e], o);
-      emax[e] = max(emax[e], __shfl_xor_sync(0xffffffffu, emax[e], o));
-      emin[e] = min(emin[e], __shfl_xor_sync(0xffffffffu, emin[e], o));
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      mxp[w] = __vmaxu2(mxp[w], __shfl_xor_sync(0xffffffffu, mxp[w], o));
+      mnp[w] = __vminu2(mnp[w], __shfl_xor_sync(0xffffffffu, mnp[w], o));
     }
   }
   if ((tid & 31) < GROUPS) {
@@ -174,7 +198,9 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
     for (int e = 0; e < 8; ++e) {
       red[warp * D + g * 8 + e] = part[e];
       redz[warp * D + g * 8 + e] = zp[e];
-      rede[warp * D + g * 8 + e] = uint16_t((emax[e] << 8) | emin[e]);
+      const uint32_t emx = ((e & 1) ? (mxp[e >> 1] >> 16) : (mxp[e >> 1] & 0xFFFFu)) >> 7;
+      const uint32_t emn = ((e & 1) ? (mnp[e >> 1] >> 16) : (mnp[e >> 1] & 0xFFFFu)) >> 7;
+      rede[warp * D + g * 8 + e] = uint16_t((emx << 8) | emn);
     }
   }
   fence_async_shared();
@@ -253,7 +279,7 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
       for (int kk = 0; kk < BLK / 16; ++kk) {
         const uint64_t da = smem_desc(smem_u32(sP) + kk * 2048, BLK * 128, 1024, 2);
         const uint64_t db = smem_desc(smem_u32(sV) + kk * 2048, BLK * 128, 1024, 2);
-        mma_bf16_ss(tmem + D, da, db, id1, kk > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem, da, db, id1, kk > 0 ? 1u : 0u);
       }
     }
     tc_commit(&bars[2]);
@@ -262,7 +288,7 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
   ok = mbar_wait(&bars[2], 0, abort_flag) && ok;
   tc_fence_after();
   {
-    const uint32_t trow = tmem + D + (uint32_t((warp & 3) * 32) << 16);
+    const uint32_t trow = tmem + (uint32_t((warp & 3) * 32) << 16);
     __nv_bfloat16* hs = hstate + (bh * (long long)NB + j) * hpitch + (long long)lrow * D;
 #pragma unroll
     for (int cq = 0; cq < D / 32; ++cq) {
@@ -283,7 +309,7 @@ __global__ void __launch_bounds__(256, 2) k_kstats(const __grid_constant__ CUten
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 2 * D);
+  if (warp == 0) tmem_dealloc(tmem, D);
 }
 
 // mu[bh][c] = float32 nearest to (sum of the N values of K[bh][:][c]) / N.
