@@ -43,7 +43,10 @@ def lib() -> ctypes.CDLL:
         L.ora_select_topk.argtypes = [vp, ll, i, i, i, vp, vp]
         L.ora_topk_count.argtypes = [i, f]
         L.ora_topk_count.restype = i
-        L.ora_sla_rows.argtypes = [vp] * 4 + [i] * 6 + [vp] * 6 + [i] * 3 + [vp, i, i] + [vp] * 3
+        L.ora_skip_count.argtypes = [i, i, f]
+        L.ora_skip_count.restype = i
+        L.ora_block_classes.argtypes = [vp, ll, i, ll, i, vp, vp, i, vp, vp]
+        L.ora_sla_rows.argtypes = [vp] * 4 + [i] * 5 + [vp] * 6 + [i] * 3 + [vp, i, i] + [vp] * 3
         L.ora_sla_rows.restype = i
         _lib = L
     return _lib
@@ -162,10 +165,59 @@ def bitmap_of(idx: np.ndarray, nblk: int) -> np.ndarray:
     return out
 
 
+# ---------------------------------------------------------------- three classes, per-head counts
+
+CLS_NEGLIGIBLE, CLS_LINEAR, CLS_CRITICAL = 0, 1, 2
+
+
+def skip_count(nblk: int, kc: int, skip_frac: float) -> int:
+    kn = lib().ora_skip_count(int(nblk), int(kc), float(skip_frac))
+    if kn < 0:
+        raise ValueError("skip_frac must be in [0, 1)")
+    return kn
+
+
+def head_counts(nblk: int, H: int, topk_frac, skip_frac=None):
+    tf = np.broadcast_to(np.asarray(topk_frac, dtype=np.float64), (H,))
+    sf = np.broadcast_to(np.asarray(0.0 if skip_frac is None else skip_frac, dtype=np.float64), (H,))
+    kc = np.array([topk_count(nblk, float(t)) for t in tf], dtype=np.int64)
+    kn = np.array([skip_count(nblk, int(c), float(x)) for c, x in zip(kc, sf)], dtype=np.int64)
+    return kc, kn
+
+
+def _classes(p, rows_per_head, kc, kn):
+    pp = _c(p, np.float64)
+    n = pp.shape[-1]
+    rows = pp.size // n
+    cls = np.empty(pp.shape, dtype=np.uint8)
+    tie = np.empty(pp.shape[:-1], dtype=np.uint8)
+    kca = _c(kc, np.int32)
+    kna = _c(kn, np.int32)
+    lib().ora_block_classes(_p(pp), rows, n, rows_per_head, len(kca), _p(kca), _p(kna), threads(), _p(cls), _p(tie))
+    return cls, tie.astype(bool)
+
+
+def block_classes(p: np.ndarray, kc: int, kn: int):
+    n = p.shape[-1]
+    return _classes(p, max(1, np.asarray(p).size // n), [kc], [kn])
+
+
+def block_mask_classes(q_bits, k_bits, block: int, topk_frac, skip_frac=None) -> dict:
+    p = block_probs(block_means(q_bits, block), block_means(k_bits, block))
+    B, H, nblk, _ = p.shape
+    kc, kn = head_counts(nblk, H, topk_frac, skip_frac)
+    cls, tie = _classes(p, nblk, kc, kn)
+    idx = np.full((B, H, nblk, int(kc.max())), -1, dtype=np.int32)
+    for h in range(H):
+        crit = np.nonzero(cls[:, h] == CLS_CRITICAL)   # row-major: ascending j within each (b, i)
+        idx[:, h, :, :kc[h]] = crit[2].reshape(B, nblk, int(kc[h]))
+    return {"cls": cls, "idx": idx, "kc": kc, "kn": kn, "near_tie": tie, "probs": p}
+
+
 # ---------------------------------------------------------------- the whole operator
 
-def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, *,
-                  items=None, quant=True, pcast=True, smooth=True, idx_override=None):
+def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
+                  items=None, quant=True, pcast=True, smooth=True, idx_override=None, skip_frac=None):
     """Same arguments and result as sla_oracle.sla_attention: {"out",
     "o_sparse", "o_lin" (before the projection): {(b, h, i): float64 rows},
     "mask", "quant"}."""
@@ -175,14 +227,21 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
     w = _c(w_bits, np.uint16)
     B, H, N, d = q.shape
     nblk = (N + block - 1) // block
-    mask = block_mask(q, k, block, topk_frac)
+    classes = skip_frac is not None or np.ndim(topk_frac) > 0
+    if classes:
+        mask = block_mask_classes(q, k, block, topk_frac, skip_frac)
+        cls = np.array(mask["cls"], dtype=np.uint8, copy=True)
+        for (b, h, i), row in (idx_override or {}).items():
+            cls[b, h, i] = np.asarray(row, dtype=np.uint8)
+    else:
+        mask = block_mask(q, k, block, topk_frac)
+        cls = np.ones((B, H, nblk, nblk), dtype=np.uint8)
+        np.put_along_axis(cls, mask["idx"].astype(np.int64), CLS_CRITICAL, axis=-1)
+        for (b, h, i), lst in (idx_override or {}).items():
+            cls[b, h, i] = CLS_LINEAR
+            cls[b, h, i, np.asarray(lst, dtype=np.int64)] = CLS_CRITICAL
     qz = quantize(q, k, block) if quant else None
     mu = qz["mu"] if quant else channel_mean(k)
-    kc = mask["kc"]
-    crit = np.array(mask["idx"], dtype=np.int32, copy=True)
-    if idx_override:
-        for (b, h, i), lst in idx_override.items():
-            crit[b, h, i] = np.asarray(lst, dtype=np.int32)
     if items is None:
         items = [(b, h, i) for b in range(B) for h in range(H) for i in range(nblk)]
     items = [tuple(int(t) for t in it) for it in items]
@@ -195,7 +254,7 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
         ptrs = [_p(qz["q_i8"]), _p(qz["k_i8"]), _p(qz["q_scale"]), _p(qz["k_scale"])]
     else:
         ptrs = [None, None, None, None]
-    rc = lib().ora_sla_rows(_p(q), _p(k), _p(v), _p(w), B, H, N, d, block, kc, _p(crit),
+    rc = lib().ora_sla_rows(_p(q), _p(k), _p(v), _p(w), B, H, N, d, block, _p(cls),
                             _p(_c(mu, np.float32)), *ptrs, 1 if quant else 0, 1 if pcast else 0,
                             1 if smooth else 0, _p(it), n, threads(), _p(out), _p(osp), _p(olin))
     if rc != 0:

@@ -15,7 +15,11 @@
 //   linear branch with a linear projection, SageSLA = selection followed by
 //   INT8 computation on the kept blocks);
 //   "TurboDiffusion技术指南：突破视频生成效率瓶颈的实践方案" (blog.gitcode.com),
-//   section "SageSLA" and the T2V parameter list (--sla_topk 0.1 keeps 10%).
+//   section "SageSLA" and the T2V parameter list (--sla_topk 0.1 keeps 10%);
+//   "TurboDiffusion: 即時AI影片生成的重大突破" (bonega.ai), section "SLA:
+//   稀疏線性注意力" (cheaper substitutes where full attention is not needed),
+//   the basis of the optional third block class (left out entirely) and of
+//   per-head fractions, an extension the pages do not spell out.
 // The readings where the pages leave a step open are stated at each function;
 // they are the same readings as oracle/sla_oracle.py (the numpy statement),
 // which this file restates independently.
@@ -374,9 +378,52 @@ int ora_topk_count(int nblk, float topk_frac) {
   return int(std::min(double(nblk), std::max(1.0, kc)));
 }
 
+// Negligible blocks per query block: floor(float(skip_frac) * nblk), at most
+// nblk - kc (the third class of the three-class mask: left out of the linear
+// branch too; none when skip_frac = 0).  -1 if skip_frac is not in [0, 1).
+int ora_skip_count(int nblk, int kc, float skip_frac) {
+  const double f = double(skip_frac);
+  if (!(f >= 0.0 && f < 1.0)) return -1;
+  const double kn = std::floor(f * double(nblk));
+  return int(std::min(kn, double(nblk - kc)));
+}
+
+// Classes of the key blocks in each of `rows` rows of p (length nblk): row r
+// belongs to head (r / rows_per_head) % H and uses kc and kn of that head.
+// Ranking: larger value first, equal values by the lower index first;
+// rank < kc: critical (2); rank >= nblk - kn: negligible (0); otherwise
+// linear (1).  A block's rank is the number of blocks ranked before it,
+// counted directly.  near_tie[r] = 1 when a class boundary separates values
+// within 1e-9 (relative).
+void ora_block_classes(const double* p, long long rows, int nblk, long long rows_per_head, int H, const int* kc,
+                       const int* kn, int threads, uint8_t* cls, uint8_t* near_tie) {
+  parallel_for(rows, threads, [&](long long r) {
+    const int h = int((r / rows_per_head) % H);
+    const int c = kc[h], z = kn[h];
+    const double* row = p + r * nblk;
+    std::vector<int> rank(nblk);
+    for (int j = 0; j < nblk; ++j) {
+      int before = 0;
+      for (int m = 0; m < nblk; ++m) before += (row[m] > row[j] || (row[m] == row[j] && m < j)) ? 1 : 0;
+      rank[j] = before;
+      cls[r * nblk + j] = before < c ? 2 : (before >= nblk - z ? 0 : 1);
+    }
+    std::vector<int> at(nblk);
+    for (int j = 0; j < nblk; ++j) at[rank[j]] = j;
+    uint8_t tie = 0;
+    for (int cut : {c, nblk - z})
+      if (cut > 0 && cut < nblk) {
+        const double a = row[at[cut - 1]], b = row[at[cut]];
+        if ((a - b) <= 1e-9 * a) tie = 1;
+      }
+    near_tie[r] = tie;
+  });
+}
+
 // Output rows of the whole operator for a list of query blocks.
 //   q, k, v: bf16 [B][H][N][d]; w: bf16 [d][d] (W_proj, O_lin . W: row vectors)
-//   crit: int32 [B][H][nblk][kc] the kept key blocks of every query block
+//   cls: uint8 [B][H][nblk][nblk] the class of every (query block, key
+//     block): 2 kept (exact attention), 1 linear branch, 0 left out
 //   mu: float32 [B][H][d] (the K channel mean)
 //   qi8, ki8, sq, sk: the INT8 codes and scales (quant = 1), else unused
 //   items: n_items triples (b, h, i)
@@ -390,10 +437,11 @@ int ora_topk_count(int nblk, float topk_frac) {
 //   unrounded P, P rounded to bf16 when pcast = 1; O_sparse = (P . V) / l.
 //   phi(x) = x + 1 for x > 0, else exp(x); per key block j h_j = sum phi(k)
 //   v^T, z_j = sum phi(k) over its valid rows (raw K); h_rest, z_rest are
-//   summed directly over the blocks NOT kept; O_lin = phi(q) h_rest /
-//   (phi(q) . z_rest), zero when every block is kept; out = O_sparse + O_lin W.
+//   summed directly over the blocks of class 1; O_lin = phi(q) h_rest /
+//   (phi(q) . z_rest), zero when no block is of class 1; out = O_sparse +
+//   O_lin W.
 int ora_sla_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* w, int B, int H, int N,
-                 int d, int block, int kc, const int32_t* crit, const float* mu, const int8_t* qi8,
+                 int d, int block, const uint8_t* cls, const float* mu, const int8_t* qi8,
                  const int8_t* ki8, const float* sq, const float* sk, int quant, int pcast, int smooth,
                  const int32_t* items, int n_items, int threads, double* out, double* o_sparse, double* o_lin) {
   const int nblk = (N + block - 1) / block;
@@ -438,7 +486,11 @@ int ora_sla_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const 
   parallel_for(n_items, threads, [&](long long t) {
     const int b = items[3 * t], hh = items[3 * t + 1], i = items[3 * t + 2];
     const long long bh = (long long)b * H + hh;
-    const int32_t* lst = crit + (bh * nblk + i) * kc;
+    const uint8_t* row_cls = cls + (bh * nblk + i) * nblk;
+    std::vector<int> lst;
+    for (int j = 0; j < nblk; ++j)
+      if (row_cls[j] == 2) lst.push_back(j);
+    const int kc = int(lst.size());
     const int lo = i * block, hi = std::min(N, lo + block);
     const int rows = hi - lo;
     double* po = out + (size_t)t * block * d;
@@ -490,17 +542,15 @@ int ora_sla_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const 
       }
       for (int c = 0; c < d; ++c) ps[(size_t)r * d + c] = acc_c[c] / l;
     }
-    // linear part over the blocks not kept
-    std::vector<char> kept(nblk, 0);
-    for (int u = 0; u < kc; ++u) kept[lst[u]] = 1;
+    // linear part over the blocks of class 1
     bool any_rest = false;
-    for (int j = 0; j < nblk; ++j) any_rest = any_rest || !kept[j];
+    for (int j = 0; j < nblk; ++j) any_rest = any_rest || row_cls[j] == 1;
     if (any_rest) {
       const std::vector<double>& h = hs[head_of[bh]];
       const std::vector<double>& z = zs[head_of[bh]];
       std::vector<double> hr((size_t)d * d, 0.0), zr(d, 0.0);
       for (int j = 0; j < nblk; ++j) {
-        if (kept[j]) continue;
+        if (row_cls[j] != 1) continue;
         for (int a = 0; a < d; ++a) {
           zr[a] += z[(size_t)j * d + a];
           for (int c = 0; c < d; ++c) hr[(size_t)a * d + c] += h[((size_t)j * d + a) * d + c];

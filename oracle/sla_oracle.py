@@ -29,6 +29,10 @@ Notation: inputs are bf16 bit patterns, uint16 arrays Q, K, V [B, H, N, d] and
 W_proj [d, d]; ``block`` tokens per block; nblk = ceil(N / block); block r
 covers rows [r*block, min(N, (r+1)*block)).
 
+The three-class mask (block_classes and its callers) is an extension: the
+pages name two classes (top-K core blocks, the rest linear); a third class,
+left out of both branches, is optional and off by default.
+
 Parity status: every function here is pinned by a test in
 tests/test_oracle_pins.py against a closed form, a library routine, a brute
 force or a hand-derived case, except the choice of raw K (rather than
@@ -288,6 +292,92 @@ def bitmap_of(idx: np.ndarray, nblk: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# three block classes and per-head fractions
+# ---------------------------------------------------------------------------
+# [P1] 三(二) items 1-2 split the key blocks of a query block into the top-K
+# "core" blocks (exact attention) and the rest (the linear branch); [P4]
+# "SLA: 稀疏線性注意力" replaces dense attention by cheaper substitutes where it
+# is not needed.  Extension adopted here (the pages name no third class): the
+# blocks at the bottom of the same ranking may be left out of the linear
+# branch too ("negligible").  With skip_frac = 0 nothing is left out and the
+# operator is exactly the two-class one above.  topk_frac and skip_frac may
+# be given per head (the same value for every batch entry).
+
+CLS_NEGLIGIBLE, CLS_LINEAR, CLS_CRITICAL = 0, 1, 2
+
+
+def skip_count(nblk: int, kc: int, skip_frac: float) -> int:
+    """Number of negligible key blocks per query block: floor(skip_frac * nblk), at most nblk - kc.
+
+    Reading: like topk_frac, the fraction is the float32 value the C interface
+    receives, multiplied by nblk exactly; it is rounded DOWN (a block is left
+    out only when the whole fraction covers it) and capped so that the
+    critical blocks stay.  skip_frac must be in [0, 1).
+    """
+    f = float(np.float32(skip_frac))
+    if not (f >= 0.0 and f < 1.0):
+        raise ValueError("skip_frac must be in [0, 1)")
+    return min(math.floor(f * nblk), nblk - kc)
+
+
+def head_counts(nblk: int, H: int, topk_frac, skip_frac=None) -> tuple[np.ndarray, np.ndarray]:
+    """(kc [H], kn [H]) from a scalar or one fraction per head."""
+    tf = np.broadcast_to(np.asarray(topk_frac, dtype=np.float64), (H,))
+    sf = np.broadcast_to(np.asarray(0.0 if skip_frac is None else skip_frac, dtype=np.float64), (H,))
+    kc = np.array([topk_count(nblk, float(t)) for t in tf], dtype=np.int64)
+    kn = np.array([skip_count(nblk, int(c), float(f)) for c, f in zip(kc, sf)], dtype=np.int64)
+    return kc, kn
+
+
+def block_classes(p: np.ndarray, kc: int, kn: int) -> tuple[np.ndarray, np.ndarray]:
+    """Class of every key block of every row of p: uint8 [..., n] and near_tie bool [...].
+
+    The blocks are ranked by value, larger first, equal values by the lower
+    index first (the same ranking as select_topk).  The first kc are critical
+    (2), the last kn negligible (0), the rest go to the linear branch (1).  A
+    row is a near tie when either boundary separates values that differ by at
+    most 1e-9 of the larger.
+    """
+    shp = p.shape[:-1]
+    n = p.shape[-1]
+    flat = p.reshape(-1, n)
+    cls = np.full(flat.shape, CLS_LINEAR, dtype=np.uint8)
+    tie = np.zeros(flat.shape[0], dtype=bool)
+    pos = np.arange(n)
+    for r in range(flat.shape[0]):
+        row = flat[r]
+        order = np.lexsort((pos, -row))
+        cls[r, order[:kc]] = CLS_CRITICAL
+        if kn > 0:
+            cls[r, order[n - kn:]] = CLS_NEGLIGIBLE
+        for cut in (kc, n - kn):
+            if 0 < cut < n:
+                a, b = row[order[cut - 1]], row[order[cut]]
+                tie[r] = tie[r] or bool((a - b) <= NEAR_TIE_REL * a)
+    return cls.reshape(shp + (n,)), tie.reshape(shp)
+
+
+def block_mask_classes(q_bits: np.ndarray, k_bits: np.ndarray, block: int, topk_frac, skip_frac=None) -> dict:
+    """Three-class mask with per-head counts: {"cls" uint8 [B, H, nblk, nblk],
+    "idx" int32 [B, H, nblk, max kc] (critical blocks ascending, then -1),
+    "kc" [H], "kn" [H], "near_tie", "probs"}."""
+    qbar = block_means(q_bits, block)
+    kbar = block_means(k_bits, block)
+    p = block_probs(qbar, kbar)
+    B, H, nblk, _ = p.shape
+    kc, kn = head_counts(nblk, H, topk_frac, skip_frac)
+    cls = np.empty(p.shape, dtype=np.uint8)
+    tie = np.empty(p.shape[:-1], dtype=bool)
+    idx = np.full((B, H, nblk, int(kc.max())), -1, dtype=np.int32)
+    for h in range(H):
+        cls[:, h], tie[:, h] = block_classes(p[:, h], int(kc[h]), int(kn[h]))
+        for b in range(B):
+            for i in range(nblk):
+                idx[b, h, i, :kc[h]] = np.flatnonzero(cls[b, h, i] == CLS_CRITICAL)
+    return {"cls": cls, "idx": idx, "kc": kc, "kn": kn, "near_tie": tie, "probs": p}
+
+
+# ---------------------------------------------------------------------------
 # critical blocks: INT8 QK^T, softmax, bf16 P, PV  ([P1] 三(一) item 3, 三(二) item 3)
 # ---------------------------------------------------------------------------
 
@@ -361,17 +451,21 @@ def linear_states(k64: np.ndarray, v64: np.ndarray, block: int) -> tuple[np.ndar
     return h, z
 
 
-def linear_rows(q64_blk: np.ndarray, h: np.ndarray, z: np.ndarray, crit) -> np.ndarray:
+def linear_rows(q64_blk: np.ndarray, h: np.ndarray, z: np.ndarray, crit, lin=None) -> np.ndarray:
     """O_lin for the rows of one query block: phi(q) h_rest / (phi(q) . z_rest).
 
     h_rest and z_rest are summed directly over the key blocks NOT in ``crit``
     (the plain definition: every non-critical block goes through the linear
-    branch).  When every block is critical there is no linear part and
-    O_lin = 0.
+    branch), or, when ``lin`` (bool [nblk]) is given, over the blocks it
+    marks (the linear class of the three-class mask).  With no block in the
+    linear branch there is no linear part and O_lin = 0.
     """
     nblk, d, _ = h.shape
-    keep = np.ones(nblk, dtype=bool)
-    keep[np.asarray(crit, dtype=np.int64)] = False
+    if lin is not None:
+        keep = np.asarray(lin, dtype=bool).copy()
+    else:
+        keep = np.ones(nblk, dtype=bool)
+        keep[np.asarray(crit, dtype=np.int64)] = False
     if not keep.any():
         return np.zeros((q64_blk.shape[0], d))
     h_rest = h[keep].sum(axis=0)
@@ -384,8 +478,8 @@ def linear_rows(q64_blk: np.ndarray, h: np.ndarray, z: np.ndarray, crit) -> np.n
 # the whole operator
 # ---------------------------------------------------------------------------
 
-def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, *,
-                  items=None, quant=True, pcast=True, smooth=True, idx_override=None):
+def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
+                  items=None, quant=True, pcast=True, smooth=True, idx_override=None, skip_frac=None):
     """SageSLA attention: out = O_sparse + O_lin . W_proj.
 
     [P1] 三(二) item 3 (SLA selection, then INT8 computation on the selected
@@ -398,7 +492,12 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
     quant/pcast/smooth: False switches off INT8 quantisation (float64 scores),
     the bf16 cast of P, or the K smoothing; all True is the operator itself.
     idx_override: optional {(b, h, i): key-block list} replacing the mask's
-    choice for those rows (used where the mask is a near tie).
+    choice for those rows (used where the mask is a near tie); with the
+    three-class mask, {(b, h, i): class row uint8 [nblk]}.
+    topk_frac may be one fraction per head, and skip_frac (scalar or per
+    head) leaves the lowest-ranked blocks out of the linear branch; either
+    one selects the three-class mask (block_mask_classes), whose "mask"
+    entry is then that function's result.
 
     Returns {"out": {(b,h,i): float64 [rows, d]}, "o_sparse", "o_lin",
     "mask": block_mask(...), "quant": quantize(...)}.
@@ -406,7 +505,11 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
     q_bits = np.asarray(q_bits, dtype=np.uint16)
     B, H, N, d = q_bits.shape
     nblk = (N + block - 1) // block
-    mask = block_mask(q_bits, k_bits, block, topk_frac)
+    classes = skip_frac is not None or np.ndim(topk_frac) > 0
+    if classes:
+        mask = block_mask_classes(q_bits, k_bits, block, topk_frac, skip_frac)
+    else:
+        mask = block_mask(q_bits, k_bits, block, topk_frac)
     qz = quantize(q_bits, k_bits, block) if quant else None
     mu = qz["mu"] if quant else channel_mean(k_bits)
     w64 = bf16_to_f64(w_bits)
@@ -423,9 +526,17 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
         hst, zst = linear_states(k64, v64, block)
         ks64 = k64 - mu[b, h].astype(np.float64)[None, :] if smooth else k64
         for i in rows:
-            crit = mask["idx"][b, h, i]
-            if idx_override is not None and (b, h, i) in idx_override:
-                crit = np.asarray(idx_override[(b, h, i)], dtype=np.int32)
+            lin = None
+            if classes:
+                row_cls = mask["cls"][b, h, i]
+                if idx_override is not None and (b, h, i) in idx_override:
+                    row_cls = np.asarray(idx_override[(b, h, i)], dtype=np.uint8)
+                crit = np.flatnonzero(row_cls == CLS_CRITICAL).astype(np.int32)
+                lin = row_cls == CLS_LINEAR
+            else:
+                crit = mask["idx"][b, h, i]
+                if idx_override is not None and (b, h, i) in idx_override:
+                    crit = np.asarray(idx_override[(b, h, i)], dtype=np.int32)
             lo, hi = i * block, min(N, (i + 1) * block)
             if quant:
                 qi8_blk = qz["q_i8"][b, h, i * block:(i + 1) * block]
@@ -437,7 +548,7 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac: float, 
                 os_ = critical_rows(None, None, None, None, v64, crit, N, block, pcast=pcast,
                                     q64_blk=qb, ks64=ks64)
             os_ = os_[:hi - lo]
-            ol = linear_rows(q64[lo:hi], hst, zst, crit)
+            ol = linear_rows(q64[lo:hi], hst, zst, crit, lin)
             out = os_ + np.matmul(ol, w64)
             res["o_sparse"][(b, h, i)] = os_
             res["o_lin"][(b, h, i)] = ol

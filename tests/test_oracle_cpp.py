@@ -55,3 +55,23 @@ def test_cpp_oracle_modes_agree_with_numpy_oracle():
         b = C.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.4, **kw)
         for key in a["out"]:
             assert np.max(np.abs(a["out"][key] - b["out"][key])) <= 1e-12, kw
+
+
+@pytest.mark.parametrize("N,d,block,fr,sk,seed", [
+    (1000, 64, 64, [0.1, 0.3, 0.5], [0.5, 0.2, 0.0], 21),
+    (777, 128, 128, [0.25, 1.0, 0.05], [0.7, 0.0, 0.9], 22),
+])
+def test_cpp_oracle_three_classes_agree_with_numpy_oracle(N, d, block, fr, sk, seed):
+    x = make_inputs(2, 3, N, d, seed, "iid", None)
+    a = NP.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, fr, skip_frac=sk)
+    b = C.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, fr, skip_frac=sk)
+    assert np.array_equal(a["mask"]["kc"], b["mask"]["kc"]) and np.array_equal(a["mask"]["kn"], b["mask"]["kn"])
+    assert np.array_equal(a["mask"]["near_tie"], b["mask"]["near_tie"])
+    diff = np.any(a["mask"]["cls"] != b["mask"]["cls"], axis=-1)
+    assert not np.any(diff & ~a["mask"]["near_tie"])
+    assert np.array_equal(a["mask"]["idx"][~diff], b["mask"]["idx"][~diff])
+    for part in ("out", "o_sparse", "o_lin"):
+        for key in a[part]:
+            if diff[key]:
+                continue
+            assert np.max(np.abs(a[part][key] - b[part][key])) <= 1e-12, (part, key)

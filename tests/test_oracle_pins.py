@@ -387,3 +387,103 @@ def test_linear_hand_case_through_the_whole_operator(impl):
     expect = np.array([[eval(s, {"e": e}) for s in row] for row in g["o_lin_expr"]])
     got = np.concatenate([res["o_lin"][(0, 0, i)] for i in range(2)])
     assert np.allclose(got, expect, rtol=1e-14, atol=0)
+
+
+# ---------------------------------------------------------------- three classes, per-head fractions
+
+def test_skip_counts_golden(impl):
+    g = golden("skip_counts.json")
+    for c in g["cases"]:
+        assert impl.skip_count(c["nblk"], c["kc"], c["frac"]) == c["kn"], c
+    with pytest.raises(ValueError):
+        impl.skip_count(10, 1, 1.0)
+    with pytest.raises(ValueError):
+        impl.skip_count(10, 1, -0.1)
+
+
+def test_block_classes_are_two_nested_top_k_selections(impl):
+    """The ranking is a total order, so the critical blocks are the top kc and
+    the blocks that are not negligible are the top nblk - kn; select_topk (pinned
+    by brute force over all subsets above) gives both.  Rows with exact ties."""
+    rng = np.random.default_rng(31)
+    for n in (1, 2, 5, 9, 16):
+        p = rng.integers(0, 4, size=(6, n)).astype(np.float64)   # many exact ties
+        for kc in range(1, n + 1):
+            for kn in range(0, n - kc + 1):
+                cls, _ = impl.block_classes(p, kc, kn)
+                for r in range(p.shape[0]):
+                    top, _ = O.select_topk(p[r][None], kc)
+                    keep, _ = O.select_topk(p[r][None], n - kn) if kn < n else (np.zeros((1, 0), int), None)
+                    want = np.zeros(n, dtype=np.uint8)
+                    want[keep[0]] = 1
+                    want[top[0]] = 2
+                    assert np.array_equal(cls[r], want), (n, kc, kn, r)
+
+
+def test_block_classes_near_tie_at_either_boundary(impl):
+    p = np.array([[0.5, 0.3, 0.2, 0.2 * (1 + 1e-12)],    # tie between ranks 2 and 3 only
+                  [0.5, 0.5 * (1 - 1e-12), 0.1, 0.05]])   # tie between ranks 0 and 1 only
+    _, t = impl.block_classes(p, 1, 1)     # boundaries after rank 0 and after rank 2
+    assert t.tolist() == [True, True]
+    _, t = impl.block_classes(p, 2, 0)     # boundary after rank 1 only
+    assert t.tolist() == [False, False]
+
+
+def test_three_classes_with_no_skip_equal_the_two_class_operator(impl):
+    x = make_inputs(1, 2, 300, 16, seed=41)
+    a = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 32, 0.3)
+    b = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 32, [0.3, 0.3], skip_frac=0.0)
+    assert np.array_equal(b["mask"]["idx"], a["mask"]["idx"])
+    for key in a["out"]:
+        assert np.array_equal(a["out"][key], b["out"][key])
+
+
+def test_per_head_fractions_are_the_scalar_operator_head_by_head(impl):
+    x = make_inputs(1, 3, 256, 16, seed=42)
+    fr = [0.1, 0.25, 0.6]
+    res = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 32, fr, skip_frac=[0.0, 0.0, 0.0])
+    for h, f in enumerate(fr):
+        one = impl.sla_attention(x["q"][:, h:h + 1], x["k"][:, h:h + 1], x["v"][:, h:h + 1], x["proj"], 32, f)
+        kc = impl.topk_count(8, f)
+        assert res["mask"]["kc"][h] == kc
+        assert np.array_equal(res["mask"]["idx"][0, h, :, :kc], one["mask"]["idx"][0, 0])
+        assert (res["mask"]["idx"][0, h, :, kc:] == -1).all()
+        for i in range(8):
+            assert np.array_equal(res["out"][(0, h, i)], one["out"][(0, 0, i)])
+
+
+def test_three_classes_closed_form_q_k_zero(impl):
+    """Q = K = 0: every score ties, so the ranking is the block index: blocks
+    [0, kc) critical, the last kn negligible, the rest linear; P = 1 on every
+    kept key and phi = 1: out = mean(V over the critical keys) + mean(V over the
+    linear keys) . W, per head with its own fractions."""
+    rng = np.random.default_rng(43)
+    B, H, N, d, block = 1, 3, 200, 8, 32                  # nblk 7, the last block 8 rows
+    fr, sk = [0.3, 0.15, 0.5], [0.3, 0.6, 0.5]
+    v = rng.standard_normal((B, H, N, d)).astype(np.float32)
+    w = rng.standard_normal((d, d)).astype(np.float32) / 4
+    vb, wb = f32_to_bf16_bits(v), f32_to_bf16_bits(w)
+    z = np.zeros((B, H, N, d), dtype=np.uint16)
+    res = impl.sla_attention(z, z, vb, wb, block, fr, skip_frac=sk)
+    V, W = O.bf16_to_f64(vb), O.bf16_to_f64(wb)
+    for h in range(H):
+        kc = impl.topk_count(7, fr[h])
+        kn = impl.skip_count(7, kc, sk[h])
+        assert (kc, kn) == [(3, 2), (2, 4), (4, 3)][h]
+        want = np.array([2] * kc + [1] * (7 - kc - kn) + [0] * kn, dtype=np.uint8)
+        assert (res["mask"]["cls"][0, h] == want).all()
+        lin_keys = V[0, h, kc * block:min(N, (7 - kn) * block)]
+        expect = V[0, h, :kc * block].mean(0) + (lin_keys.mean(0) @ W if len(lin_keys) else 0.0)
+        for i in range(7):
+            rows = res["out"][(0, h, i)]
+            assert np.allclose(rows, np.broadcast_to(expect, rows.shape), rtol=0, atol=1e-12)
+
+
+def test_no_linear_class_means_no_linear_part(impl):
+    """kc + kn = nblk leaves no block for the linear branch: O_lin = 0, out = O_sparse."""
+    x = make_inputs(1, 1, 256, 16, seed=44)
+    res = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 32, 0.25, skip_frac=0.75)
+    assert not (res["mask"]["cls"] == 1).any()
+    for key in res["out"]:
+        assert not res["o_lin"][key].any()
+        assert np.array_equal(res["out"][key], res["o_sparse"][key])
