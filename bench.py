@@ -4,10 +4,12 @@ and ms per call at the 480P video-DiT shape (B=1, H=12, N=32768, d=128,
 block=128, top-10%), one call of the whole operator per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 480p|720p|dense|sweep0.05|sweep0.10|sweep0.20|sweep0.40|tiny]
+                    [--workload 480p|720p|dense|sweep0.05|sweep0.10|sweep0.20|sweep0.40|tiny|480p_classes]
 
 --workload picks another of the seeded synthetic workloads (default: the
 480P headline); the JSON line's metric string names the workload's shape.
+480p_classes runs the three-class operator (per-head fractions, the lowest
+half of every ranking left out of the linear branch) on the 480P shape.
 
 One process per GPU (torchrun for N > 1).  Every (batch, head) problem is
 independent, so each rank runs its own full-size problem with no collective
@@ -53,6 +55,9 @@ def metric_for(w) -> str:
     if w.name == WORKLOAD:
         return METRIC
     pct = f"{w.topk_frac * 100:g}%"
+    if w.classes:
+        fr = sorted(set(w.head_fracs)) if w.head_fracs else [w.topk_frac]
+        pct = f"{fr[0] * 100:g}..{fr[-1] * 100:g}% per head, skip {(w.skip_frac or 0) * 100:g}%"
     return (f"effective sparse-attn TOPS & ms/call, B={w.B} N={w.N} H={w.H} d={w.d} top-{pct}, 1 B200 "
             f"({w.name} workload)")
 
@@ -66,22 +71,24 @@ def critical_ops(idx, N, d, block):
     """Ops of the critical-block work counted from the block lists idx
     [B, H, nblk, kc]: int8 QK^T and bf16 PV, 2 * rows_i * keys_j * d each for
     every kept (query block i, key block j), with the valid rows and keys of
-    a partial last block."""
+    a partial last block.  Entries -1 (lists shorter than the pitch) count
+    nothing."""
     import numpy as np
 
     nblk = idx.shape[-2]
     sizes = np.minimum(block, N - np.arange(nblk) * block).astype(np.float64)
-    keys = sizes[idx.astype(np.int64)].sum(axis=-1)          # [B, H, nblk]
+    ix = idx.astype(np.int64)
+    keys = np.where(ix >= 0, sizes[np.maximum(ix, 0)], 0.0).sum(axis=-1)   # [B, H, nblk]
     ops = float((2.0 * d * sizes[None, None, :] * keys).sum())
     return ops, ops
 
 
-def algorithmic_bytes(B, H, N, d, nblk, kc):
+def algorithmic_bytes(B, H, N, d, nblk, kc, linear=None):
     """Bytes a call must move at least: q, k, v in (bf16), out (bf16), the
     INT8 codes written and read once, and the float32 linear states written
-    and read once (none when every block is kept)."""
+    and read once (none when every block is kept, or `linear` is False)."""
     b = B * H * N * d * (3 * 2 + 2 + 2 * 1 * 2)
-    if kc < nblk:
+    if (kc < nblk) if linear is None else linear:
         b += 2 * B * H * nblk * (d * d + d) * 4
     return float(b)
 
@@ -255,6 +262,43 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
+# ---------------------------------------------------------------- one operator, two mask kinds
+
+def op_attn(S, t, w, out):
+    """The device operator on the workload (three-class entry point where the workload asks for it)."""
+    if w.classes:
+        S.sla_attn_classes(t["q"], t["k"], t["v"], t["proj"], block=w.block, topk_frac=w.fracs,
+                           skip_frac=w.skip_frac, out=out)
+    else:
+        S.sla_attn(t["q"], t["k"], t["v"], t["proj"], block=w.block, topk_frac=w.topk_frac, out=out)
+
+
+def op_host(S, host, hout, w):
+    if w.classes:
+        S.sla_attn_classes_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block,
+                                topk_frac=w.fracs, skip_frac=w.skip_frac)
+    else:
+        S.sla_attn_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block, topk_frac=w.topk_frac)
+
+
+def op_mask(S, t, w):
+    """(block lists [B, H, nblk, pitch], class map or None, kc per head, linear branch used)."""
+    if w.classes:
+        idx, cls = S.sla_mask_classes(t["q"], t["k"], w.block, w.fracs, w.skip_frac, classes=True)
+        kc, kn, _ = S.head_counts(w.N, w.block, w.H, w.fracs, w.skip_frac)
+        return idx.cpu().numpy(), cls.cpu().numpy(), kc, any(c + n < w.nblk for c, n in zip(kc, kn))
+    kc = S.topk_count(w.N, w.block, w.topk_frac)
+    return S.sla_mask(t["q"], t["k"], w.block, w.topk_frac).cpu().numpy(), None, [kc] * w.H, kc < w.nblk
+
+
+def oracle_head(O, w, xs, h):
+    """The CPU oracle on head h of the workload (xs: that head's inputs)."""
+    if w.classes:
+        fr = w.fracs[h] if isinstance(w.fracs, list) else w.fracs
+        return O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, [fr], skip_frac=w.skip_frac)
+    return O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, w.topk_frac)
+
+
 # ---------------------------------------------------------------- CPU oracle sample
 
 def oracle_sample(w, x, max_heads: int, budget_s: float):
@@ -267,7 +311,7 @@ def oracle_sample(w, x, max_heads: int, budget_s: float):
     for h in range(min(max_heads, w.H)):
         xs = {k: (v[:1, h:h + 1] if v.ndim == 4 else v) for k, v in x.items()}
         t0 = time.perf_counter()
-        O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, w.topk_frac)
+        oracle_head(O, w, xs, h)
         dt += time.perf_counter() - t0
         nh += 1
         if dt >= budget_s:
@@ -278,16 +322,21 @@ def oracle_sample(w, x, max_heads: int, budget_s: float):
                      f"value = dense-equivalent ops of those heads / wall time")
 
 
-def mask_parity(w, x, gidx):
-    """The GPU's block lists against the oracle's over the whole workload:
-    rows, rows the oracle marks as near ties, rows whose lists differ, and
-    rows that differ without being near ties (must be 0)."""
+def mask_parity(w, x, gidx, gcls=None):
+    """The GPU's block lists (class maps, for the three-class mask) against
+    the oracle's over the whole workload: rows, rows the oracle marks as near
+    ties, rows that differ, and rows that differ without being near ties
+    (must be 0)."""
     import numpy as np
 
     from oracle import cpp_oracle as O
 
-    ref = O.block_mask(x["q"], x["k"], w.block, w.topk_frac)
-    diff = np.any(gidx != ref["idx"], axis=-1)
+    if w.classes:
+        ref = O.block_mask_classes(x["q"], x["k"], w.block, w.fracs, w.skip_frac)
+        diff = np.any(gcls != ref["cls"], axis=-1)
+    else:
+        ref = O.block_mask(x["q"], x["k"], w.block, w.topk_frac)
+        diff = np.any(gidx != ref["idx"], axis=-1)
     return {"rows": int(diff.size), "near_tie_rows": int(ref["near_tie"].sum()),
             "differing_rows": int(diff.sum()), "differing_off_near_tie": int((diff & ~ref["near_tie"]).sum())}
 
@@ -317,7 +366,8 @@ def run_ours(args, dist):
     if args.heads:
         import dataclasses
 
-        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}-first{args.heads}heads")
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}-first{args.heads}heads",
+                                head_fracs=w.head_fracs[:args.heads] if w.head_fracs else None)
         x = make_workload(CONFIGS[args.workload], heads=list(range(args.heads)))
     else:
         x = make_workload(w)
@@ -326,7 +376,7 @@ def run_ours(args, dist):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        S.sla_attn(t["q"], t["k"], t["v"], t["proj"], block=w.block, topk_frac=w.topk_frac, out=out)
+        op_attn(S, t, w, out)
 
     for _ in range(args.warmup):
         step()
@@ -359,8 +409,8 @@ def run_ours(args, dist):
 
     ops = dense_equivalent_ops(w.B, w.H, w.N, w.d)
     value = weak_scaling_value(ops, dist.world, ms / 1e3)
-    kc = S.topk_count(w.N, w.block, w.topk_frac)
-    gidx = S.sla_mask(t["q"], t["k"], w.block, w.topk_frac).cpu().numpy()
+    gidx, gcls, kcs, linear = op_mask(S, t, w)
+    kc = kcs[0] if len(set(kcs)) == 1 else kcs
     qk, pv = critical_ops(gidx, w.N, w.d, w.block)
     peaks = load_peaks()
     peak, peak_src = attn_roofline(qk, pv, peaks)
@@ -386,9 +436,12 @@ def run_ours(args, dist):
         "data": "synthetic (seeded field-plus-noise, see synth/workloads.py)",
         "config": {"workload": w.describe(), "kc": kc,
                    "parallelism": f"replicas x{dist.world} (independent problems per rank)",
-                   "l2": "inputs larger than L2 (q, k, v: 302 MB; ~1 GB moved per call), no flush"},
+                   "l2": (f"inputs larger than L2 (q, k, v: {3 * w.B * w.H * w.N * w.d * 2 / 1e6:.0f} MB), "
+                          "no flush") if 3 * w.B * w.H * w.N * w.d * 2 > 126e6 else
+                         "inputs smaller than L2 (launch-bound case), no flush"},
         "roofline": roof,
-        "roofline_call": call_roofline(qk, pv, algorithmic_bytes(w.B, w.H, w.N, w.d, w.nblk, kc), ms, peaks),
+        "roofline_call": call_roofline(qk, pv, algorithmic_bytes(w.B, w.H, w.N, w.d, w.nblk, max(kcs), linear),
+                                       ms, peaks),
         "kernels": kernels, "gpu_launches": launches, "clocks": clocks, "e2e": e2e,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
@@ -396,7 +449,7 @@ def run_ours(args, dist):
         line["cpu_baseline"] = {"value": round(cops / dt / 1e12, 6), "unit": UNIT, "cores": oracle_threads(),
                                 "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
         # near ties of the block mask (CPU oracle leg): every differing row must be one
-        line["mask_parity"] = mask_parity(w, x, gidx)
+        line["mask_parity"] = mask_parity(w, x, gidx, gcls)
         line["near_tie_rows"] = line["mask_parity"]["near_tie_rows"]
     return line
 
@@ -409,20 +462,20 @@ def run_e2e(S, t, w, args, dist):
 
     host = {k: v.cpu().pin_memory() for k, v in t.items()}
     hout = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16).pin_memory()
-    S.sla_attn_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block, topk_frac=w.topk_frac)
+    op_host(S, host, hout, w)
     n = max(1, min(args.steps, args.e2e_steps))
     dist.barrier()
     t0 = time.perf_counter()
     for _ in range(n):
-        S.sla_attn_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block,
-                        topk_frac=w.topk_frac)
+        op_host(S, host, hout, w)
     dt = dist.max((time.perf_counter() - t0) / n)
     ops = dense_equivalent_ops(w.B, w.H, w.N, w.d)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = hout.numel() * hout.element_size()
     return {"value": round(weak_scaling_value(ops, dist.world, dt), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(dt * 1e3, 3),
-            "steps": n, "timer": "host wall clock around sla_attn_host (synchronous)"}
+            "steps": n, "timer": "host wall clock around the synchronous host-buffer call "
+                                 f"({'sla_attn_classes_host' if w.classes else 'sla_attn_host'})"}
 
 
 def run_reference(args, dist):
@@ -444,7 +497,7 @@ def run_reference(args, dist):
     def step(s):
         h = pos[s % w.H]
         xs = {k: (v[:1, h:h + 1] if v.ndim == 4 else v) for k, v in x.items()}
-        O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, w.topk_frac)
+        oracle_head(O, w, xs, s % w.H)
 
     for s_ in range(args.warmup):
         step(s_)
@@ -476,7 +529,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=["tiny", "480p", "720p", "dense", "sweep0.05", "sweep0.10", "sweep0.20", "sweep0.40"])
+                    choices=["tiny", "480p", "720p", "dense", "sweep0.05", "sweep0.10", "sweep0.20", "sweep0.40",
+                             "480p_classes"])
     ap.add_argument("--cpu-heads", type=int, default=6,
                     help="most heads of the workload the CPU oracle baseline runs in full")
     ap.add_argument("--cpu-budget", type=float, default=15.0,

@@ -9,7 +9,9 @@
  *        items 1-3;
  *   [P3] "TurboDiffusion技术指南：突破视频生成效率瓶颈的实践方案"
  *        (blog.gitcode.com), section "SageSLA" and the T2V parameter list
- *        (--attention_type sagesla, --sla_topk 0.1 = keep 10%).
+ *        (--attention_type sagesla, --sla_topk 0.1 = keep 10%);
+ *   [P4] "TurboDiffusion: 即時AI影片生成的重大突破" (bonega.ai), section
+ *        "SLA: 稀疏線性注意力".
  * The pages give no formulas; the exact semantics implemented here are:
  *   1. mu = per-channel mean of K over the N tokens (exact sum, rounded once to
  *      float32, for every finite input); K_s = float32(K) - mu.  ([P1] 三(一) item 1, "outlier smoothing")
@@ -158,6 +160,44 @@ int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, v
                 float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, float topk_frac,
                 void* stream);
 
+/* Three block classes and per-head fractions (an extension: the pages name
+ * two classes, the top-K "core" blocks of [P1] 三(二) 1 and the rest through
+ * the linear branch of [P1] 三(二) 2; [P4] "SLA: 稀疏線性注意力" replaces dense
+ * attention by cheaper substitutes where it is not needed).  Head h (the same
+ * h for every batch entry) uses topk_frac[h] and skip_frac[h]:
+ *   kc_h = clamp(ceil(float(topk_frac[h]) * nblk), 1, nblk) blocks are kept
+ *          (exact attention), as in sla_topk_count;
+ *   kn_h = min(floor(float(skip_frac[h]) * nblk), nblk - kc_h) blocks, those
+ *          ranked last, are left out of both branches;
+ *   the other nblk - kc_h - kn_h blocks go through the linear branch.
+ * Ranking: larger pooled score first, equal scores lower block index first
+ * (the order sla_mask keeps by).  skip_frac may be NULL (all 0): then every
+ * head is the two-class operator with its own fraction.  A query block with
+ * no block in the linear branch has no linear part.
+ *   topk_frac : in, HOST float [H], each in (0, 1]
+ *   skip_frac : in, HOST float [H], each in [0, 1), or NULL
+ * H <= 512, else SLA_ERR_UNSUPPORTED. */
+
+/* Host only: kc_h and kn_h for every head (kc, kn: HOST int [H], either may
+ * be NULL).  Returns the largest kc_h (the pitch of sla_mask_classes'
+ * blk_idx), or minus an error code. */
+int sla_head_counts(int N, int block, int H, const float* topk_frac, const float* skip_frac, int* kc, int* kn);
+
+/* Step 3 with per-head counts and three classes.
+ *   blk_idx : out, int32 [B,H,nblk,kcp] (kcp = sla_head_counts' result): the
+ *             kc_h kept key blocks of each query block, ascending, then -1
+ *   classes : out, uint8 [B,H,nblk,nblk]: 2 kept, 1 linear branch, 0 left
+ *             out; or NULL */
+int sla_mask_classes(const void* q, const void* k, int32_t* blk_idx, uint8_t* classes, int B, int H, int N, int d,
+                     int block, const float* topk_frac, const float* skip_frac, void* stream);
+
+/* sla_attn_ex with per-head counts and three classes: the linear branch sums
+ * the states of the blocks of class 1 only.  Arguments as sla_attn_ex, with
+ * topk_frac and skip_frac as above. */
+int sla_attn_classes(const void* q, const void* k, const void* v, const void* proj, void* out, int out_dtype,
+                     float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, const float* topk_frac,
+                     const float* skip_frac, void* stream);
+
 /* sla_attn on HOST buffers (pageable or pinned): copies q, k, v, proj to the
  * device, runs the operator and copies out (bf16) back, and returns when the
  * result is in host memory.  The (batch, head) pairs are processed in up to
@@ -167,6 +207,10 @@ int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, v
  * sla_attn's.  Calls on the same device are serialised. */
 int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
                   int N, int d, int block, float topk_frac);
+
+/* sla_attn_classes on HOST buffers, as sla_attn_host (output bf16). */
+int sla_attn_classes_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
+                          int N, int d, int block, const float* topk_frac, const float* skip_frac);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  The word is shared by every stream of the device: a code

@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
 
 EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
            "sla_get_error", "sla_status_string", "sla_profile_enable", "sla_profile_read",
-           "sla_mask_noalloc", "sla_selftest_wait_timeout")
+           "sla_mask_noalloc", "sla_selftest_wait_timeout", "sla_head_counts", "sla_mask_classes",
+           "sla_attn_classes", "sla_attn_classes_host")
 
 KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm")
 
@@ -54,6 +55,10 @@ def lib() -> ctypes.CDLL:
         L.sla_attn.argtypes = [vp] * 5 + [i] * 5 + [f, vp]
         L.sla_attn_ex.argtypes = [vp] * 5 + [i] + [vp] * 2 + [i] * 5 + [f, vp]
         L.sla_attn_host.argtypes = [vp] * 5 + [i] * 5 + [f]
+        L.sla_head_counts.argtypes = [i, i, i, vp, vp, vp, vp]
+        L.sla_mask_classes.argtypes = [vp] * 4 + [i] * 5 + [vp, vp, vp]
+        L.sla_attn_classes.argtypes = [vp] * 5 + [i] + [vp] * 2 + [i] * 5 + [vp, vp, vp]
+        L.sla_attn_classes_host.argtypes = [vp] * 5 + [i] * 5 + [vp, vp]
         L.sla_get_error.argtypes = [vp]
         L.sla_status_string.argtypes = [i]
         L.sla_status_string.restype = ctypes.c_char_p
@@ -170,11 +175,90 @@ def sla_attn(q, k, v, proj, block: int = 128, topk_frac: float = 0.1, out=None, 
     return out
 
 
+def _head_fracs(H: int, topk_frac, skip_frac):
+    """HOST float32 arrays of one topk_frac and one skip_frac (or None) per head."""
+    tf = (ctypes.c_float * H)(*[float(x) for x in _per_head(topk_frac, H)])
+    sf = None if skip_frac is None else (ctypes.c_float * H)(*[float(x) for x in _per_head(skip_frac, H)])
+    return tf, sf
+
+
+def _per_head(x, H: int):
+    try:
+        vals = [float(t) for t in x]
+    except TypeError:
+        vals = [float(x)] * H
+    if len(vals) != H:
+        raise ValueError(f"expected one fraction per head ({H})")
+    return vals
+
+
+def _cptr(arr):
+    return None if arr is None else ctypes.cast(arr, ctypes.c_void_p)
+
+
+def head_counts(N: int, block: int, H: int, topk_frac, skip_frac=None):
+    """(kc per head, kn per head, list pitch) of the three-class mask."""
+    tf, sf = _head_fracs(H, topk_frac, skip_frac)
+    kc = (ctypes.c_int * H)()
+    kn = (ctypes.c_int * H)()
+    kcp = lib().sla_head_counts(int(N), int(block), int(H), _cptr(tf), _cptr(sf), _cptr(kc), _cptr(kn))
+    if kcp < 0:
+        raise SlaError(-kcp, "sla_head_counts")
+    return list(kc), list(kn), kcp
+
+
+def sla_mask_classes(q, k, block: int, topk_frac, skip_frac=None, classes: bool = False, stream=None,
+                     check: bool = False):
+    """Three-class block mask with per-head fractions.  Returns idx [B,H,nblk,kcp]
+    int32 (kept blocks ascending, then -1) and, with classes=True, the uint8
+    class map [B,H,nblk,nblk] (2 kept, 1 linear branch, 0 left out)."""
+    import torch
+
+    B, H, N, d = _shape(q)
+    nb = nblk(N, block)
+    tf, sf = _head_fracs(H, topk_frac, skip_frac)
+    _, _, kcp = head_counts(N, block, H, topk_frac, skip_frac)
+    idx = torch.empty((B, H, nb, kcp), dtype=torch.int32, device=q.device)
+    cm = torch.empty((B, H, nb, nb), dtype=torch.uint8, device=q.device) if classes else None
+    _check(lib().sla_mask_classes(_ptr(q), _ptr(k), _ptr(idx), _ptr(cm), B, H, N, d, block, _cptr(tf), _cptr(sf),
+                                  _stream(stream)), "sla_mask_classes")
+    _after(check, stream, "sla_mask_classes")
+    return (idx, cm) if classes else idx
+
+
+def sla_attn_classes(q, k, v, proj, block: int = 128, topk_frac=0.1, skip_frac=None, out=None, out_dtype=None,
+                     o_sparse=None, o_lin=None, stream=None, check: bool = False):
+    """SageSLA attention with per-head fractions and an optional third block
+    class left out of the linear branch (skip_frac per head or scalar)."""
+    import torch
+
+    B, H, N, d = _shape(q)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=out_dtype or torch.bfloat16, device=q.device)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bf16 or float32")
+    tf, sf = _head_fracs(H, topk_frac, skip_frac)
+    kind = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _check(lib().sla_attn_classes(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), kind, _ptr(o_sparse),
+                                  _ptr(o_lin), B, H, N, d, block, _cptr(tf), _cptr(sf), _stream(stream)),
+           "sla_attn_classes")
+    _after(check, stream, "sla_attn_classes")
+    return out
+
+
 def sla_attn_host(q, k, v, proj, out, block: int = 128, topk_frac: float = 0.1) -> None:
     """SageSLA attention on host (CPU) tensors (out: bf16); copies in and out inside the call."""
     B, H, N, d = _shape(q)
     _check(lib().sla_attn_host(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
                                float(topk_frac)), "sla_attn_host")
+
+
+def sla_attn_classes_host(q, k, v, proj, out, block: int = 128, topk_frac=0.1, skip_frac=None) -> None:
+    """sla_attn_classes on host (CPU) tensors (out: bf16); copies in and out inside the call."""
+    B, H, N, d = _shape(q)
+    tf, sf = _head_fracs(H, topk_frac, skip_frac)
+    _check(lib().sla_attn_classes_host(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
+                                       _cptr(tf), _cptr(sf)), "sla_attn_classes_host")
 
 
 def profile_enable(on: bool = True) -> None:

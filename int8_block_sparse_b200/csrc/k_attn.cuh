@@ -50,13 +50,14 @@
 namespace sla {
 
 struct AttnParams {
-  const int32_t* idx;          // [BH][NB][kc]
+  const int32_t* idx;          // [BH][NB][kcp] kept blocks, ascending
+  const int* kc_bh;            // [BH] list length per head, or nullptr: kc for every head
   const float* sq;             // [BH][NB]
   const float* sk;             // [BH][NB]
   const __nv_bfloat16* q;      // [BH][N][D] raw queries (phi(q) of the linear part)
   const float* zrest;          // [BH][NB][D] g_i: z sums over the non-selected blocks
   void* out;                   // [BH][N][D], bf16 or float32
-  int N, NB, NP, kc, items;
+  int N, NB, NP, kc, kcp, items;
   int sparse;                  // the selected blocks (softmax attention) take part
   int lin;                     // the linear part is added
   int out_f32;                 // float32 output (else bf16)
@@ -204,11 +205,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int kc = p.kc;
   const int NB = p.NB;
   const int tiles_total = 2 * gridDim.x;
   const bool sparse = p.sparse != 0, lin = p.lin != 0;
-  const int H = sparse ? kc * NH : 0;   // halves per item
+  // kept blocks of the items of head bh, and the halves (64 keys) they make
+  auto kc_of = [&](int bh) { return p.kc_bh != nullptr ? __ldg(p.kc_bh + bh) : p.kc; };
+  auto halves_of = [&](int bh) { return sparse ? kc_of(bh) * NH : 0; };
 
   if (warp < 4)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLoad));
@@ -238,13 +240,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
         for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
           const int bh = item / NB, i = item % NB;
           if (sparse) {
+            const int kc = kc_of(bh);
             if (lane == 0) {
               if (!(ok = mbar_wait(&b.q_empty, (item_it & 1) ^ 1, abort_flag))) break;
               mbar_expect_tx(&b.q_full, C::Q_BYTES);
               tma_load_2d(tq, &tm_q, &b.q_full, 0, bh * p.NP + i * BLK);
               ++nq;
             }
-            const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
+            const int32_t* lst = p.idx + ((long long)bh * NB + i) * p.kcp;
             int jn = __ldg(lst);
             for (int t = 0; t < kc; ++t) {
               const int j = jn;
@@ -295,6 +298,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
         uint32_t kit = 0, vit = 0, item_it = 0, hg = 0;   // hg: halves of the items before this one
         bool ok = true;
         for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
+          const int H = halves_of(item / NB);
           if (sparse) {
             if (!(ok = mbar_wait(&b.q_full, item_it & 1, abort_flag))) break;
             // S(y) = Q K_half(y)^T into buffer (hg + y) % 2; at the first half of a
@@ -337,8 +341,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
               if (x + 2 < H) ok = issue_qk(x + 2);
             }
             if (!ok) break;
-            kit += kc;
-            vit += kc;
+            kit += H / NH;
+            vit += H / NH;
           }
           if (lin) {
             // O += A . G'_i, A (bf16, D/2 columns) in the S buffer of half hg + H
@@ -380,8 +384,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
     const int part_rows = p.N % BLK;                // rows of a partial last block (0: none)
     for (int item = blockIdx.x * 2 + u; sparse && item < p.items && ok; item += tiles_total) {
       const int bh = item / NB, i = item % NB;
+      const int kc = kc_of(bh), H = kc * NH;
       const float sq_i = __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale;
-      const int32_t* lst = p.idx + ((long long)bh * NB + i) * kc;
+      const int32_t* lst = p.idx + ((long long)bh * NB + i) * p.kcp;
       // running maximum m (log2 domain) and normaliser l of this row
       float m = -INFINITY, l = 0.f;
       float cl = 0.f;
@@ -535,6 +540,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
     // A of tile u (after its softmax); false if a wait gave up
     auto do_a = [&](int u) -> bool {
       TileBars& b = bars[u];
+      const int H = halves_of((blockIdx.x * 2 + u + it * tiles_total) / NB);
       if (sparse) {
         if (!mbar_wait(&b.l_full, it & 1, abort_flag)) return false;
         lrow[u] = l_buf[u * 128 + r];

@@ -23,6 +23,14 @@
 // largest by a bitwise search over the high 32 bits (warp reductions with
 // redux.sync), then over the low 32 bits of the keys tied at that high half,
 // if they are not all kept.
+//
+// Per-head counts and a third class (an extension: the pages name two
+// classes): head h keeps kc_h blocks and may leave its kn_h lowest-ranked
+// blocks out of the linear branch as well (ranking: larger score first, equal
+// scores lower index first).  The blocks that are not negligible are then the
+// top nblk - kn_h, found by the same search.  The linear indicator row
+// (notcrit) marks the blocks of the linear class; the optional byte map holds
+// 1 for kept blocks or, in class mode, the class (2 kept, 1 linear, 0 left out).
 #pragma once
 #include "sm100.cuh"
 
@@ -55,10 +63,20 @@ __device__ __forceinline__ uint32_t count_ge(const uint32_t* hi_r, const uint32_
 
 constexpr int kMaskSlabCh = 16;                               // channels per slab
 constexpr int kMaskSlabBytes = kMaskSlabCh * 256 * 8;          // 32 KB
+constexpr int kMaxHeadCounts = 512;
+
+// Block counts per head, passed by value: head bh % H keeps kc[.] blocks and
+// leaves kn[.] out; kcp is the pitch of the block lists (the largest kc).
+struct HeadCounts {
+  int H, kcp, classes;            // classes: the byte map holds classes, not 0/1
+  uint16_t kc[kMaxHeadCounts];
+  uint16_t kn[kMaxHeadCounts];
+};
 
 template <int D, int R>
 __global__ void __launch_bounds__(256) k_mask(const __grid_constant__ CUtensorMap tm_kbar,
-                                             const double* __restrict__ qbar, int NB, int kc,
+                                             const double* __restrict__ qbar, int NB,
+                                             const __grid_constant__ HeadCounts hc, int* __restrict__ kc_bh,
                                              int32_t* __restrict__ idx, uint8_t* __restrict__ bitmap,
                                              __nv_bfloat16* __restrict__ notcrit, int ncpitch) {
   static_assert(R >= 1 && R <= 8, "one warp per row in the selection");
@@ -71,6 +89,7 @@ __global__ void __launch_bounds__(256) k_mask(const __grid_constant__ CUtensorMa
   uint64_t* full = reinterpret_cast<uint64_t*>(sc + R * NB);   // [2]
 
   const long long bh = blockIdx.y;
+  const int kc = hc.kc[bh % hc.H], kn = hc.kn[bh % hc.H];
   const int i0 = blockIdx.x * R;
   const int nrows = min(R, NB - i0);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -85,6 +104,7 @@ __global__ void __launch_bounds__(256) k_mask(const __grid_constant__ CUtensorMa
                 int(bh * D + (n % SLABS) * kMaskSlabCh));
   };
   int issued = 0;   // slabs requested (thread 0)
+  if (kc_bh != nullptr && blockIdx.x == 0 && tid == 0) kc_bh[bh] = kc;
   if (tid == 0) {
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
@@ -159,63 +179,79 @@ __global__ void __launch_bounds__(256) k_mask(const __grid_constant__ CUtensorMa
       hi_r[e] = (regs && j < NB) ? w32[2 * j + 1] : 0u;
       lo_r[e] = (regs && j < NB) ? w32[2 * j] : 0u;
     }
-    // T = the kc-th largest key: first the kc-th largest high half Th, then,
-    // among the keys whose high half is Th, the (kc - #above)-th largest low half
-    uint32_t Th = 0u;
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = Th | (1u << bit);
-      const uint32_t cnt = regs ? count_ge<KPL>(hi_r, lo_r, w32, NB, lane, false, 0u, cand)
-                                : count_ge<0>(hi_r, lo_r, w32, NB, lane, false, 0u, cand);
-      if (cnt >= (uint32_t)kc) Th = cand;
-    }
-    uint32_t above = 0u, tied = 0u, tied_min = 0xFFFFFFFFu;
-    for (int j = lane; j < NB; j += 32) {
-      const uint32_t h = w32[2 * j + 1];
-      above += (h > Th) ? 1u : 0u;
-      if (h == Th) {
-        ++tied;
-        tied_min = min(tied_min, w32[2 * j]);
-      }
-    }
-    above = __reduce_add_sync(0xffffffffu, above);
-    tied = __reduce_add_sync(0xffffffffu, tied);
-    tied_min = __reduce_min_sync(0xffffffffu, tied_min);
-    const uint32_t need = (uint32_t)kc - above;   // >= 1: at least kc high halves are >= Th
-    uint32_t Tl = tied_min;                       // all tied keys are kept
-    if (tied != need) {
-      Tl = 0u;
+    // The k-th largest key T and how many keys equal to T rank before the
+    // cut (need_eq): first the k-th largest high half Th by a bitwise search,
+    // then, among the keys whose high half is Th, the (k - #above)-th largest
+    // low half.
+    auto kth = [&](int k, unsigned long long& T, int& need_eq) {
+      uint32_t Th = 0u;
       for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t cand = Tl | (1u << bit);
-        const uint32_t cnt = regs ? count_ge<KPL>(hi_r, lo_r, w32, NB, lane, true, Th, cand)
-                                  : count_ge<0>(hi_r, lo_r, w32, NB, lane, true, Th, cand);
-        if (cnt >= need) Tl = cand;
+        const uint32_t cand = Th | (1u << bit);
+        const uint32_t cnt = regs ? count_ge<KPL>(hi_r, lo_r, w32, NB, lane, false, 0u, cand)
+                                  : count_ge<0>(hi_r, lo_r, w32, NB, lane, false, 0u, cand);
+        if (cnt >= (uint32_t)k) Th = cand;
       }
-    }
-    int gt = 0;
-    const unsigned long long T = ((unsigned long long)Th << 32) | Tl;
-    for (int j = lane; j < NB; j += 32) gt += (rk[j] > T) ? 1 : 0;
+      uint32_t above = 0u, tied = 0u, tied_min = 0xFFFFFFFFu;
+      for (int j = lane; j < NB; j += 32) {
+        const uint32_t h = w32[2 * j + 1];
+        above += (h > Th) ? 1u : 0u;
+        if (h == Th) {
+          ++tied;
+          tied_min = min(tied_min, w32[2 * j]);
+        }
+      }
+      above = __reduce_add_sync(0xffffffffu, above);
+      tied = __reduce_add_sync(0xffffffffu, tied);
+      tied_min = __reduce_min_sync(0xffffffffu, tied_min);
+      const uint32_t need = (uint32_t)k - above;   // >= 1: at least k high halves are >= Th
+      uint32_t Tl = tied_min;                      // all tied keys are kept
+      if (tied != need) {
+        Tl = 0u;
+        for (int bit = 31; bit >= 0; --bit) {
+          const uint32_t cand = Tl | (1u << bit);
+          const uint32_t cnt = regs ? count_ge<KPL>(hi_r, lo_r, w32, NB, lane, true, Th, cand)
+                                    : count_ge<0>(hi_r, lo_r, w32, NB, lane, true, Th, cand);
+          if (cnt >= need) Tl = cand;
+        }
+      }
+      int gt = 0;
+      T = ((unsigned long long)Th << 32) | Tl;
+      for (int j = lane; j < NB; j += 32) gt += (rk[j] > T) ? 1 : 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
-    const int need_eq = kc - gt;
-    int eq_seen = 0, out_pos = 0;
-    int32_t* dst = idx + (bh * NB + i) * (long long)kc;
+      for (int o = 16; o > 0; o >>= 1) gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      need_eq = k - gt;
+    };
+    unsigned long long Tc, Tn = 0ull;
+    int need_c, need_n = 0;
+    kth(kc, Tc, need_c);
+    if (kn > 0) kth(NB - kn, Tn, need_n);   // the blocks ranked before NB - kn are not negligible
+    int eqc_seen = 0, eqn_seen = 0, out_pos = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    int32_t* dst = idx + (bh * NB + i) * (long long)hc.kcp;
     for (int j0 = 0; j0 < NB; j0 += 32) {
       const int j = j0 + lane;
       const bool inb = j < NB;
       const unsigned long long key = inb ? rk[j] : 0ull;
-      const bool eq = inb && key == T;
-      const bool great = inb && key > T;
-      const unsigned eqmask = __ballot_sync(0xffffffffu, eq);
-      const int eq_before = eq_seen + __popc(eqmask & ((1u << lane) - 1u));
-      const bool sel = great || (eq && eq_before < need_eq);
+      const bool eqc = inb && key == Tc;
+      const unsigned eqcmask = __ballot_sync(0xffffffffu, eqc);
+      const bool sel = (inb && key > Tc) || (eqc && eqc_seen + __popc(eqcmask & lt) < need_c);
+      bool keep = inb;                        // not negligible
+      if (kn > 0) {
+        const bool eqn = inb && key == Tn;
+        const unsigned eqnmask = __ballot_sync(0xffffffffu, eqn);
+        keep = (inb && key > Tn) || (eqn && eqn_seen + __popc(eqnmask & lt) < need_n);
+        eqn_seen += __popc(eqnmask);
+      }
       const unsigned selmask = __ballot_sync(0xffffffffu, sel);
-      if (sel) dst[out_pos + __popc(selmask & ((1u << lane) - 1u))] = j;
-      if (bitmap != nullptr && inb) bitmap[(bh * NB + i) * (long long)NB + j] = sel ? 1 : 0;
+      if (sel) dst[out_pos + __popc(selmask & lt)] = j;
+      if (bitmap != nullptr && inb)
+        bitmap[(bh * NB + i) * (long long)NB + j] = hc.classes ? (sel ? 2 : (keep ? 1 : 0)) : (sel ? 1 : 0);
       if (notcrit != nullptr && j < ncpitch)
-        notcrit[(bh * NB + i) * (long long)ncpitch + j] = __float2bfloat16_rn((inb && !sel) ? 1.f : 0.f);
-      eq_seen += __popc(eqmask);
+        notcrit[(bh * NB + i) * (long long)ncpitch + j] = __float2bfloat16_rn((keep && !sel) ? 1.f : 0.f);
+      eqc_seen += __popc(eqcmask);
       out_pos += __popc(selmask);
     }
+    for (int t = kc + lane; t < hc.kcp; t += 32) dst[t] = -1;   // lists shorter than the pitch
     if (notcrit != nullptr) {
       const int jstart = ((NB + 31) / 32) * 32;
       for (int j = jstart + lane; j < ncpitch; j += 32)

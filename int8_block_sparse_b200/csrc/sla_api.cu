@@ -54,6 +54,45 @@ long long topk_count_ll(long long nblk, float frac) {
 }
 
 bool frac_ok(float f) { return f > 0.f && f <= 1.f; }
+bool skip_ok(float f) { return f >= 0.f && f < 1.f; }
+
+long long skip_count_ll(long long nblk, long long kc, float frac) {
+  const double kn = std::floor((double)frac * (double)nblk);
+  return std::min<long long>((long long)kn, nblk - kc);
+}
+
+// Counts of the two-class mask: every head keeps kc blocks.
+HeadCounts uniform_counts(long long kc) {
+  HeadCounts hc;
+  std::memset(&hc, 0, sizeof(hc));
+  hc.H = 1;
+  hc.kcp = (int)kc;
+  hc.kc[0] = (uint16_t)kc;
+  return hc;
+}
+
+// Per-head counts (topk_frac[h], skip_frac[h] or 0); SLA_OK or an error code.
+int head_counts(long long nblk, int H, const float* topk_frac, const float* skip_frac, HeadCounts* hc,
+                bool* linear) {
+  if (topk_frac == nullptr) return SLA_ERR_INVALID_ARG;
+  if (H > kMaxHeadCounts) return SLA_ERR_UNSUPPORTED;
+  std::memset(hc, 0, sizeof(*hc));
+  hc->H = H;
+  hc->classes = 1;
+  *linear = false;
+  for (int h = 0; h < H; ++h) {
+    if (!frac_ok(topk_frac[h])) return SLA_ERR_INVALID_ARG;
+    const float sf = skip_frac != nullptr ? skip_frac[h] : 0.f;
+    if (!skip_ok(sf)) return SLA_ERR_INVALID_ARG;
+    const long long kc = topk_count_ll(nblk, topk_frac[h]);
+    const long long kn = skip_count_ll(nblk, kc, sf);
+    hc->kc[h] = (uint16_t)kc;
+    hc->kn[h] = (uint16_t)kn;
+    hc->kcp = std::max(hc->kcp, (int)kc);
+    *linear = *linear || kc + kn < nblk;
+  }
+  return SLA_OK;
+}
 
 // ------------------------------------------------------------------ TMA descriptors
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -123,7 +162,7 @@ size_t rounded(size_t count) { return (count * sizeof(T) + 255) & ~size_t(255); 
 
 struct Workspace {
   double* ksum; double* kbar; uint8_t* kexp; float* mu; double* qbar;
-  int8_t* qi8; int8_t* ki8; float* sq; float* sk; int32_t* idx;
+  int8_t* qi8; int8_t* ki8; float* sq; float* sk; int32_t* idx; int* kc_bh;
   __nv_bfloat16* notcrit; __nv_bfloat16* hstate; __nv_bfloat16* grest; float* zrest;
   long long ncpitch, hpitch;
 };
@@ -135,7 +174,7 @@ size_t workspace_bytes(const Shape& s, int what) {
   size_t b = rounded<double>(BH * NB * d) * 2 + rounded<double>(BH * d * (size_t)kbar_pitch((int)NB)) +
              rounded<uint8_t>(BH * NB * d * 2) + rounded<float>(BH * d);
   if (what & 1) b += rounded<int8_t>(BH * NP * d) * 2 + rounded<float>(BH * NB) * 2;
-  if (what & 2) b += rounded<int32_t>(BH * NB * kc);
+  if (what & 2) b += rounded<int32_t>(BH * NB * kc) + rounded<int>(BH);
   if (what & 8)
     b += rounded<__nv_bfloat16>(BH * NB * ncpitch) + rounded<__nv_bfloat16>(BH * NB * hpitch) +
          rounded<__nv_bfloat16>(BH * NB * d * d) + rounded<float>(BH * NB * d);
@@ -160,7 +199,10 @@ Workspace carve(const Shape& s, int what, char* base) {
     w.sq = a.take<float>(BH * NB);
     w.sk = a.take<float>(BH * NB);
   }
-  if (what & 2) w.idx = a.take<int32_t>(BH * NB * kc);
+  if (what & 2) {
+    w.idx = a.take<int32_t>(BH * NB * kc);
+    w.kc_bh = a.take<int>(BH);
+  }
   if (what & 8) {
     w.notcrit = a.take<__nv_bfloat16>(BH * NB * w.ncpitch);
     w.hstate = a.take<__nv_bfloat16>(BH * NB * w.hpitch);
@@ -261,8 +303,8 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
 }
 
 template <int D, int R>
-int launch_mask_rows(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __nv_bfloat16* notcrit,
-                     cudaStream_t st) {
+int launch_mask_rows(const Shape& s, Workspace& w, const HeadCounts& hc, int* kc_bh, int32_t* idx, uint8_t* bitmap,
+                     __nv_bfloat16* notcrit, cudaStream_t st) {
   // kbar as a 2-D float64 tensor [BH * D rows][NB key blocks]; slabs of 16 rows x 256
   CUtensorMap mkb;
   {
@@ -276,27 +318,27 @@ int launch_mask_rows(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap
   cudaFuncSetAttribute(k_mask<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   dim3 g((unsigned)((s.NB + R - 1) / R), (unsigned)s.BH);
   ProfScope ps(SLA_K_MASK, st);
-  k_mask<D, R><<<g, 256, sm, st>>>(mkb, w.qbar, (int)s.NB, (int)s.kc, idx, bitmap, notcrit, (int)w.ncpitch);
+  k_mask<D, R><<<g, 256, sm, st>>>(mkb, w.qbar, (int)s.NB, hc, kc_bh, idx, bitmap, notcrit, (int)w.ncpitch);
   return cuda_status(cudaGetLastError());
 }
 
 template <int D>
-int launch_mask(const Shape& s, Workspace& w, int32_t* idx, uint8_t* bitmap, __nv_bfloat16* notcrit,
-                cudaStream_t st) {
+int launch_mask(const Shape& s, Workspace& w, const HeadCounts& hc, int* kc_bh, int32_t* idx, uint8_t* bitmap,
+                __nv_bfloat16* notcrit, cudaStream_t st) {
   // rows per CTA: 8 unless the R x NB float64 scores would not fit
   const size_t lim = 200 * 1024;
-  if (mask_smem<D>(8, (int)s.NB) <= lim) return launch_mask_rows<D, 8>(s, w, idx, bitmap, notcrit, st);
-  if (mask_smem<D>(4, (int)s.NB) <= lim) return launch_mask_rows<D, 4>(s, w, idx, bitmap, notcrit, st);
-  if (mask_smem<D>(2, (int)s.NB) <= lim) return launch_mask_rows<D, 2>(s, w, idx, bitmap, notcrit, st);
-  return launch_mask_rows<D, 1>(s, w, idx, bitmap, notcrit, st);
+  if (mask_smem<D>(8, (int)s.NB) <= lim) return launch_mask_rows<D, 8>(s, w, hc, kc_bh, idx, bitmap, notcrit, st);
+  if (mask_smem<D>(4, (int)s.NB) <= lim) return launch_mask_rows<D, 4>(s, w, hc, kc_bh, idx, bitmap, notcrit, st);
+  if (mask_smem<D>(2, (int)s.NB) <= lim) return launch_mask_rows<D, 2>(s, w, hc, kc_bh, idx, bitmap, notcrit, st);
+  return launch_mask_rows<D, 1>(s, w, hc, kc_bh, idx, bitmap, notcrit, st);
 }
 
 
 // k_attn in one of its modes: sparse (the selected blocks), lin (the linear
 // part), out as float32 or bf16.
 template <int D, int BLK>
-int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __nv_bfloat16* v, void* out,
-                bool out_f32, bool sparse, bool lin, cudaStream_t st) {
+int launch_attn(const Shape& s, Workspace& w, const int* kc_bh, const __nv_bfloat16* q, const __nv_bfloat16* v,
+                void* out, bool out_f32, bool sparse, bool lin, cudaStream_t st) {
   using C = AttnCfg<D, BLK>;
   CUtensorMap mq, mk, mv, mg;
   std::memset(&mq, 0, sizeof(mq));
@@ -326,7 +368,8 @@ int launch_attn(const Shape& s, Workspace& w, const __nv_bfloat16* q, const __nv
   }
   AttnParams p;
   p.idx = w.idx; p.sq = w.sq; p.sk = w.sk; p.q = q; p.zrest = w.zrest; p.out = out;
-  p.N = s.N; p.NB = (int)s.NB; p.NP = (int)s.NP; p.kc = (int)s.kc; p.items = (int)(s.BH * s.NB);
+  p.kc_bh = kc_bh;
+  p.N = s.N; p.NB = (int)s.NB; p.NP = (int)s.NP; p.kc = (int)s.kc; p.kcp = (int)s.kc; p.items = (int)(s.BH * s.NB);
   p.sparse = sparse ? 1 : 0;
   p.lin = lin ? 1 : 0;
   p.out_f32 = out_f32 ? 1 : 0;
@@ -371,21 +414,24 @@ int launch_lingemm(const Shape& s, Workspace& w, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------------ dispatch
+// s.kc is the pitch of the block lists (the largest count of hc); `linear`:
+// some query block has blocks in the linear branch.
 template <int D, int BLK>
-int run_attn(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-             const __nv_bfloat16* proj, void* out, bool out_f32, float* o_sparse, float* o_lin, Workspace& w,
-             cudaStream_t st) {
-  const bool linear = s.kc < s.NB;
+int run_attn(const Shape& s, const HeadCounts& hc, bool linear, const __nv_bfloat16* q, const __nv_bfloat16* k,
+             const __nv_bfloat16* v, const __nv_bfloat16* proj, void* out, bool out_f32, float* o_sparse,
+             float* o_lin, Workspace& w, cudaStream_t st) {
+  int* kc_bh = hc.H > 1 || hc.kc[0] != s.kc ? w.kc_bh : nullptr;   // per-head list lengths
   int rc = launch_stats_quant<D, BLK>(s, q, k, v, proj, w, linear, true, w.qi8, w.ki8, w.sq, w.sk, st);
   if (rc) return rc;
-  rc = launch_mask<D>(s, w, w.idx, nullptr, linear ? w.notcrit : nullptr, st);
+  rc = launch_mask<D>(s, w, hc, kc_bh, w.idx, nullptr, linear ? w.notcrit : nullptr, st);
   if (rc) return rc;
   if (linear && (rc = launch_lingemm<D>(s, w, st))) return rc;
-  if ((rc = launch_attn<D, BLK>(s, w, q, v, out, out_f32, true, linear, st))) return rc;
+  if ((rc = launch_attn<D, BLK>(s, w, kc_bh, q, v, out, out_f32, true, linear, st))) return rc;
   // the two parts on their own, in float32 (inspection and tests)
-  if (o_sparse != nullptr && (rc = launch_attn<D, BLK>(s, w, q, v, o_sparse, true, true, false, st))) return rc;
+  if (o_sparse != nullptr && (rc = launch_attn<D, BLK>(s, w, kc_bh, q, v, o_sparse, true, true, false, st)))
+    return rc;
   if (o_lin != nullptr) {
-    if (linear) return launch_attn<D, BLK>(s, w, q, v, o_lin, true, false, true, st);
+    if (linear) return launch_attn<D, BLK>(s, w, kc_bh, q, v, o_lin, true, false, true, st);
     return cuda_status(cudaMemsetAsync(o_lin, 0, (size_t)s.BH * s.N * D * sizeof(float), st));
   }
   return SLA_OK;
@@ -573,7 +619,7 @@ int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, in
     int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                        nullptr, nullptr, w, false, false, nullptr, nullptr, nullptr, nullptr, st);
     if (r) return r;
-    return launch_mask<D>(s, w, blk_idx, bitmap, nullptr, st);
+    return launch_mask<D>(s, w, uniform_counts(s.kc), nullptr, blk_idx, bitmap, nullptr, st);
   });
 }
 
@@ -596,7 +642,7 @@ int sla_mask_noalloc(const void* q, const void* k, int32_t* blk_idx, uint8_t* bi
     int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                        nullptr, nullptr, w, false, false, nullptr, nullptr, nullptr, nullptr, st);
     if (r) return r;
-    return launch_mask<D>(s, w, blk_idx, bitmap, nullptr, st);
+    return launch_mask<D>(s, w, uniform_counts(s.kc), nullptr, blk_idx, bitmap, nullptr, st);
   });
 }
 
@@ -621,10 +667,77 @@ int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, v
   Workspace w = carve(s, what, static_cast<char*>(sc.ptr));
   return with_dims(d, block, [&](auto D_, auto B_) {
     constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
-    return run_attn<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+    return run_attn<D, BLK>(s, uniform_counts(s.kc), linear, static_cast<const __nv_bfloat16*>(q),
+                            static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                            static_cast<const __nv_bfloat16*>(proj), out, out_dtype == SLA_OUT_F32, o_sparse, o_lin,
+                            w, st);
+  });
+}
+
+int sla_attn_classes(const void* q, const void* k, const void* v, const void* proj, void* out, int out_dtype,
+                     float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, const float* topk_frac,
+                     const float* skip_frac, void* stream) {
+  if (!q || !k || !v || !proj || !out) return SLA_ERR_INVALID_ARG;
+  if (out_dtype != SLA_OUT_BF16 && out_dtype != SLA_OUT_F32) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj) || !aligned16(out) ||
+      !aligned16(o_sparse) || !aligned16(o_lin))
+    return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  HeadCounts hc;
+  bool linear = false;
+  if ((rc = head_counts(s.NB, H, topk_frac, skip_frac, &hc, &linear))) return rc;
+  s.kc = hc.kcp;
+  const int what = 1 | 2 | 4 | (linear ? 8 : 0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch sc;
+  if ((rc = sc.get(workspace_bytes(s, what), st))) return rc;
+  Workspace w = carve(s, what, static_cast<char*>(sc.ptr));
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    return run_attn<D, BLK>(s, hc, linear, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                             static_cast<const __nv_bfloat16*>(v), static_cast<const __nv_bfloat16*>(proj), out,
                             out_dtype == SLA_OUT_F32, o_sparse, o_lin, w, st);
   });
+}
+
+int sla_mask_classes(const void* q, const void* k, int32_t* blk_idx, uint8_t* classes, int B, int H, int N, int d,
+                     int block, const float* topk_frac, const float* skip_frac, void* stream) {
+  if (!q || !k || !blk_idx) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  HeadCounts hc;
+  bool linear = false;
+  if ((rc = head_counts(s.NB, H, topk_frac, skip_frac, &hc, &linear))) return rc;
+  s.kc = hc.kcp;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch sc;
+  if ((rc = sc.get(workspace_bytes(s, 0), st))) return rc;
+  Workspace w = carve(s, 0, static_cast<char*>(sc.ptr));
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    int r = launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                       nullptr, nullptr, w, false, false, nullptr, nullptr, nullptr, nullptr, st);
+    if (r) return r;
+    return launch_mask<D>(s, w, hc, nullptr, blk_idx, classes, nullptr, st);
+  });
+}
+
+int sla_head_counts(int N, int block, int H, const float* topk_frac, const float* skip_frac, int* kc, int* kn) {
+  if (N < 1 || block < 1 || H < 1) return -SLA_ERR_INVALID_ARG;
+  HeadCounts hc;
+  bool linear = false;
+  const long long nb = ((long long)N + block - 1) / block;
+  const int rc = head_counts(nb, H, topk_frac, skip_frac, &hc, &linear);
+  if (rc) return -rc;
+  for (int h = 0; h < H; ++h) {
+    if (kc) kc[h] = hc.kc[h];
+    if (kn) kn[h] = hc.kn[h];
+  }
+  return hc.kcp;
 }
 
 int sla_attn(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N, int d,
@@ -632,13 +745,24 @@ int sla_attn(const void* q, const void* k, const void* v, const void* proj, void
   return sla_attn_ex(q, k, v, proj, out, SLA_OUT_BF16, nullptr, nullptr, B, H, N, d, block, topk_frac, stream);
 }
 
-int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N,
-                  int d, int block, float topk_frac) {
+}  // extern "C"
+
+namespace {
+
+// sla_attn_host and sla_attn_classes_host: one fraction for every head, or
+// (tf != nullptr) the three-class operator with per-head fractions.
+int attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N, int d,
+              int block, float topk_frac, const float* tf, const float* sf) {
   if (!q || !k || !v || !proj || !out) return SLA_ERR_INVALID_ARG;
-  if (!frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
   Shape s;
   int rc = check_shape(B, H, N, d, block, &s);
   if (rc) return rc;
+  if (tf == nullptr && !frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
+  if (tf != nullptr) {   // the whole argument check before any copy
+    HeadCounts hc;
+    bool linear = false;
+    if ((rc = head_counts(s.NB, H, tf, sf, &hc, &linear))) return rc;
+  }
   HostStreams* hs = host_streams();
   if (hs == nullptr) return SLA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(hs->mu);
@@ -658,7 +782,9 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
     rc = SLA_ERR_CUDA;
   // heads in chunks over the streams: a chunk's copies in, operator and copy
   // out are ordered on its stream; chunks on different streams overlap
-  const long long chunks = std::min<long long>(s.BH, kHostChunks);
+  long long chunks = std::min<long long>(s.BH, kHostChunks);
+  if (tf != nullptr)   // a chunk's per-head counts must fit the kernels' table
+    chunks = std::max<long long>(chunks, (s.BH + kMaxHeadCounts - 1) / kMaxHeadCounts);
   const long long per = (s.BH + chunks - 1) / chunks;
   for (long long c = 0; c < chunks && rc == SLA_OK; ++c) {
     const long long h0 = c * per, nh = std::min<long long>(per, s.BH - h0);
@@ -672,7 +798,17 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
       rc = SLA_ERR_CUDA;
       break;
     }
-    rc = sla_attn(dq + o, dk + o, dv + o, dp, dout + o, 1, (int)nh, N, d, block, topk_frac, sc);
+    if (tf == nullptr) {
+      rc = sla_attn(dq + o, dk + o, dv + o, dp, dout + o, 1, (int)nh, N, d, block, topk_frac, sc);
+    } else {   // the chunk's heads h0 .. h0 + nh - 1 of the B*H, head index (h0 + t) % H
+      std::vector<float> ctf((size_t)nh), csf((size_t)nh);
+      for (long long t = 0; t < nh; ++t) {
+        ctf[t] = tf[(h0 + t) % H];
+        csf[t] = sf != nullptr ? sf[(h0 + t) % H] : 0.f;
+      }
+      rc = sla_attn_classes(dq + o, dk + o, dv + o, dp, dout + o, SLA_OUT_BF16, nullptr, nullptr, 1, (int)nh, N, d,
+                            block, ctf.data(), csf.data(), sc);
+    }
     if (rc == SLA_OK &&
         cudaMemcpyAsync(static_cast<char*>(out) + o, dout + o, nb, cudaMemcpyDeviceToHost, sc) != cudaSuccess)
       rc = SLA_ERR_CUDA;
@@ -685,6 +821,21 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
   const cudaError_t se = cudaStreamSynchronize(st[0]);
   if (rc == SLA_OK && se != cudaSuccess) rc = SLA_ERR_CUDA;
   return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N,
+                  int d, int block, float topk_frac) {
+  return attn_host(q, k, v, proj, out, B, H, N, d, block, topk_frac, nullptr, nullptr);
+}
+
+int sla_attn_classes_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
+                          int N, int d, int block, const float* topk_frac, const float* skip_frac) {
+  if (topk_frac == nullptr) return SLA_ERR_INVALID_ARG;
+  return attn_host(q, k, v, proj, out, B, H, N, d, block, 0.f, topk_frac, skip_frac);
 }
 
 int sla_profile_enable(int on) {

@@ -58,6 +58,17 @@ class Workload:
     seed: int
     grid: tuple | None = None   # (T, Hh, W) for "field"
     outliers: bool = False
+    head_fracs: tuple | None = None   # one topk_frac per head (three-class mask), else topk_frac for all
+    skip_frac: float | None = None    # fraction of blocks left out of the linear branch (three-class mask)
+
+    @property
+    def classes(self) -> bool:
+        return self.head_fracs is not None or self.skip_frac is not None
+
+    @property
+    def fracs(self):
+        """topk_frac as the operator takes it: per head for the three-class mask."""
+        return list(self.head_fracs) if self.head_fracs is not None else self.topk_frac
 
     @property
     def nblk(self) -> int:
@@ -65,8 +76,10 @@ class Workload:
 
     def describe(self) -> str:
         g = "x".join(map(str, self.grid)) if self.grid else "-"
+        tf = ",".join(f"{f:g}" for f in self.head_fracs) if self.head_fracs else f"{self.topk_frac}"
+        cls = f" skip_frac={self.skip_frac}" if self.skip_frac is not None else ""
         return (f"{self.name}: B={self.B} H={self.H} N={self.N} d={self.d} block={self.block} "
-                f"topk_frac={self.topk_frac} dist={self.dist} grid={g} outliers={self.outliers} "
+                f"topk_frac={tf}{cls} dist={self.dist} grid={g} outliers={self.outliers} "
                 f"seed={self.seed}")
 
 
@@ -83,6 +96,10 @@ CONFIGS = {
 for _i, _f in enumerate(SWEEP_FRACS):
     CONFIGS[f"sweep{_f:.2f}"] = Workload(f"sweep{_f:.2f}", 2, 12, 32768, 128, 128, _f, "field",
                                           4 + _i, (21, 30, 52), outliers=True)
+# the 480P shape with per-head fractions (5-20%, mean 12.5%) and the lower
+# half of every ranking left out of the linear branch (three-class mask)
+CONFIGS["480p_classes"] = Workload("480p_classes", 1, 12, 32768, 128, 128, 0.125, "field", 8, (21, 30, 52),
+                                   head_fracs=(0.05, 0.10, 0.15, 0.20) * 3, skip_frac=0.5)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:

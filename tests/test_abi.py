@@ -68,3 +68,82 @@ def test_invalid_arguments_are_refused_without_a_gpu():
     assert L.sla_topk_count(10, 128, f(0.0)) == -1
     # the allocation-free mask refuses problems beyond its fixed buffer
     assert L.sla_mask_noalloc(dummy, dummy, dummy, None, 1, 40, 75600, 128, 128, f(0.1), None) == 7
+
+
+def test_head_counts_match_the_oracle_rules():
+    import oracle as O
+
+    fr, sk = [0.1, 0.05, 0.4, 1.0], [0.5, 0.9, 0.0, 0.3]
+    kc, kn, kcp = S.head_counts(32768, 128, 4, fr, sk)
+    okc, okn = O.head_counts(256, 4, fr, sk)
+    assert kc == okc.tolist() and kn == okn.tolist() and kcp == max(kc)
+    kc, kn, kcp = S.head_counts(1000, 64, 3, 0.25)           # scalar, no skip
+    assert kc == [4, 4, 4] and kn == [0, 0, 0] and kcp == 4
+
+
+def test_class_entry_points_refuse_invalid_arguments_without_a_gpu():
+    L = S.lib()
+    dummy = 4096
+    arr = lambda *v: ctypes.cast((ctypes.c_float * len(v))(*v), ctypes.c_void_p)
+    good = arr(0.1, 0.2)
+    for bad in (arr(0.1, 0.0), arr(1.5, 0.1), arr(float("nan"), 0.1)):
+        assert L.sla_attn_classes(dummy, dummy, dummy, dummy, dummy, 0, None, None, 1, 2, 128, 128, 128, bad,
+                                  None, None) == 1
+        assert L.sla_mask_classes(dummy, dummy, dummy, None, 1, 2, 128, 128, 128, bad, None, None) == 1
+    for bad in (arr(0.0, 1.0), arr(-0.1, 0.0)):
+        assert L.sla_attn_classes(dummy, dummy, dummy, dummy, dummy, 0, None, None, 1, 2, 128, 128, 128, good,
+                                  bad, None) == 1
+    assert L.sla_attn_classes(dummy, dummy, dummy, dummy, dummy, 0, None, None, 1, 2, 128, 128, 128, None,
+                              None, None) == 1
+    many = (ctypes.c_float * 600)(*([0.1] * 600))
+    assert L.sla_attn_classes(dummy, dummy, dummy, dummy, dummy, 0, None, None, 1, 600, 128, 128, 128,
+                              ctypes.cast(many, ctypes.c_void_p), None, None) == 2
+    assert L.sla_head_counts(128, 128, 2, None, None, None, None) == -1
+
+
+def test_binding_marshals_the_class_entry_points(monkeypatch):
+    """The binding's argument marshalling for the class entry points, against a
+    stand-in for the library that records each call (no GPU: CPU tensors and
+    a stream object with a null handle)."""
+    import torch
+
+    calls = []
+
+    class FakeFn:
+        def __init__(self, name):
+            self.name = name
+
+        def __call__(self, *a):
+            calls.append((self.name, a))
+            if self.name == "sla_head_counts":
+                kc = ctypes.cast(a[5], ctypes.POINTER(ctypes.c_int))
+                kn = ctypes.cast(a[6], ctypes.POINTER(ctypes.c_int))
+                for h in range(a[2]):
+                    kc[h], kn[h] = 3 + h, 1
+                return 3 + a[2] - 1
+            return 0
+
+    class FakeLib:
+        def __getattr__(self, name):
+            return FakeFn(name)
+
+    class FakeStream:
+        cuda_stream = 0
+
+    monkeypatch.setattr(S, "_lib", FakeLib())
+    q = torch.zeros((1, 2, 256, 64), dtype=torch.bfloat16)
+    idx, cm = S.sla_mask_classes(q, q, 64, [0.1, 0.5], 0.25, classes=True, stream=FakeStream())
+    assert idx.shape == (1, 2, 4, 4) and cm.shape == (1, 2, 4, 4)
+    out = S.sla_attn_classes(q, q, q, torch.zeros((64, 64), dtype=torch.bfloat16), block=64, topk_frac=[0.1, 0.5],
+                             skip_frac=[0.25, 0.0], out_dtype=torch.float32, stream=FakeStream())
+    assert out.dtype == torch.float32 and out.shape == q.shape
+    S.sla_attn_classes_host(q, q, q, q[0, 0, :64], out.bfloat16(), block=64, topk_frac=0.3)
+    names = [c[0] for c in calls]
+    assert names == ["sla_head_counts", "sla_mask_classes", "sla_attn_classes", "sla_attn_classes_host"]
+    fr = ctypes.cast(calls[2][1][13], ctypes.POINTER(ctypes.c_float))
+    sk = ctypes.cast(calls[2][1][14], ctypes.POINTER(ctypes.c_float))
+    assert [fr[0], fr[1]] == [pytest.approx(0.1), 0.5] and [sk[0], sk[1]] == [0.25, 0.0]
+    assert calls[2][1][5] == S.OUT_F32
+    assert calls[3][1][11] is None                  # no skip fractions: NULL
+    with pytest.raises(ValueError):
+        S.sla_attn_classes(q, q, q, q, topk_frac=[0.1, 0.2, 0.3], stream=FakeStream())

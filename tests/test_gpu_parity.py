@@ -229,6 +229,123 @@ def test_repeated_calls_are_deterministic(S):
     assert torch.equal(a, b)
 
 
+# ---------------------------------------------------------------- three classes, per-head fractions
+
+def run_attn_classes(S, x, block, fr, sk):
+    import torch
+
+    q, k, v, w = (to_dev(x[t]) for t in ("q", "k", "v", "proj"))
+    B, H, N, d = x["q"].shape
+
+    def f32():
+        return torch.full((B, H, N, d), float("nan"), dtype=torch.float32, device="cuda")
+
+    out, osp, olin = f32(), f32(), f32()
+    S.sla_attn_classes(q, k, v, w, block=block, topk_frac=fr, skip_frac=sk, out=out, o_sparse=osp, o_lin=olin)
+    ob = S.sla_attn_classes(q, k, v, w, block=block, topk_frac=fr, skip_frac=sk)
+    idx, cls = S.sla_mask_classes(q, k, block, fr, sk, classes=True)
+    assert S.get_error() == 0
+    got = {"out": out, "o_sparse": osp, "o_lin": olin, "out_bf16": ob.float()}
+    return ({key: t.cpu().numpy().astype(np.float64) for key, t in got.items()}, idx.cpu().numpy(),
+            cls.cpu().numpy())
+
+
+def check_attn_classes(x, block, fr, sk, items=None, case="?"):
+    """check_attn for the three-class mask with per-head fractions: the class
+    map and the padded block lists bit-exact off near-tie rows (a differing
+    row is re-run in the oracle with the GPU's classes), the outputs as in
+    check_attn."""
+    import int8_block_sparse_b200 as S
+
+    got, gidx, gcls = run_attn_classes(S, x, block, fr, sk)
+    B, H, N, d = x["q"].shape
+    ref_mask = O.block_mask_classes(x["q"], x["k"], block, fr, sk)
+    diff = np.any(gcls != ref_mask["cls"], axis=-1)
+    bad = diff & ~ref_mask["near_tie"]
+    rec = mask_record(case, ref_mask["near_tie"], diff, bad)
+    print(json.dumps(rec))
+    assert not bad.any(), f"{int(bad.sum())} class rows differ off near ties"
+    assert rec["near_tie_rows"] <= 0.01 * rec["rows"], rec
+    assert np.array_equal(gidx[~diff], ref_mask["idx"][~diff])
+    for b in range(B):                      # the lists are the kept classes, ascending, then -1
+        for h in range(H):
+            kc = int(ref_mask["kc"][h])
+            assert (gidx[b, h, :, kc:] == -1).all()
+            kept = np.argwhere(gcls[b, h] == 2)
+            assert np.array_equal(gidx[b, h, :, :kc].reshape(-1), kept[:, 1])
+    override = {tuple(int(t) for t in ix): gcls[tuple(ix)] for ix in np.argwhere(diff)}
+    res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, fr, skip_frac=sk, items=items,
+                          idx_override=override or None)
+    w64 = O.bf16_to_f64(x["proj"])
+    parts = {"out": [], "o_sparse": [], "o_lin": [], "out_bf16": []}
+    refs = {"out": [], "o_sparse": [], "o_lin": []}
+    for (b, h, i), o in res["out"].items():
+        lo, hi = i * block, min(N, (i + 1) * block)
+        for key in parts:
+            parts[key].append(got[key][b, h, lo:hi])
+        refs["out"].append(o)
+        refs["o_sparse"].append(res["o_sparse"][(b, h, i)])
+        refs["o_lin"].append(res["o_lin"][(b, h, i)] @ w64)
+    cat = {key: np.concatenate(v) for key, v in parts.items()}
+    ref = {key: np.concatenate(v) for key, v in refs.items()}
+    st = compare_out(cat["out"], ref["out"])
+    st_sp = compare_out(cat["o_sparse"], ref["o_sparse"])
+    assert_out_ok(st_sp, "o_sparse")
+    # rows without a linear part must have exactly zero O_lin
+    zero_rows = ~np.any(ref["o_lin"], axis=-1)
+    assert not np.any(cat["o_lin"][zero_rows])
+    st_lin = compare_out(cat["o_lin"], ref["o_lin"]) if np.any(ref["o_lin"]) else None
+    if st_lin is not None:
+        assert_out_ok(st_lin, "o_lin")
+    assert_out_ok(st, "out")
+    st_b = check_bf16(cat["out_bf16"], cat["out"], ref["out"])
+    print(json.dumps({"case": case, "out": st, "o_sparse": st_sp, "o_lin": st_lin, "out_bf16": st_b}))
+    return st, st_sp, rec
+
+
+CLASS_CASES = [
+    # (B, H, N, d, block, topk_frac per head, skip_frac per head or None, dist, seed)
+    (1, 3, 1000, 64, 64, [0.1, 0.3, 0.5], [0.5, 0.2, 0.0], "iid", 31),
+    (2, 3, 777, 128, 128, [0.25, 1.0, 0.05], [0.7, 0.0, 0.9], "iid", 32),   # a dense head; ragged tail
+    (1, 4, 4096, 128, 128, [0.05, 0.1, 0.15, 0.2], [0.5] * 4, "field", 33),
+    (1, 2, 2048, 128, 64, [0.1, 0.2], None, "iid", 34),                    # per-head fractions only
+    (1, 2, 1024, 128, 128, [0.25, 0.5], [0.75, 0.5], "iid", 35),            # no linear block at all
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,block,fr,sk,dist,seed", CLASS_CASES)
+def test_attention_classes_small(S, B, H, N, d, block, fr, sk, dist, seed):
+    grid = (4, 32, 32) if dist == "field" else None
+    x = make_inputs(B, H, N, d, seed, dist, grid)
+    check_attn_classes(x, block, fr, sk, case=f"classes-{seed}")
+
+
+def test_classes_host_buffers_match_device_path(S):
+    import torch
+
+    x = make_inputs(2, 3, 900, 128, 37)
+    fr, sk = [0.1, 0.25, 0.5], [0.5, 0.0, 0.25]
+    dev = [to_dev(x[t]) for t in ("q", "k", "v", "proj")]
+    out_dev = S.sla_attn_classes(*dev, block=128, topk_frac=fr, skip_frac=sk)
+    host = [t.cpu().pin_memory() for t in dev]
+    out_host = torch.empty(host[0].shape, dtype=torch.bfloat16).pin_memory()
+    S.sla_attn_classes_host(*host, out_host, block=128, topk_frac=fr, skip_frac=sk)
+    assert torch.equal(out_host, out_dev.cpu())
+
+
+def test_classes_with_uniform_fractions_equal_the_two_class_operator(S):
+    import torch
+
+    x = make_inputs(1, 3, 1500, 128, 36)
+    dev = [to_dev(x[t]) for t in ("q", "k", "v", "proj")]
+    a = S.sla_attn(*dev, block=128, topk_frac=0.2)
+    b = S.sla_attn_classes(*dev, block=128, topk_frac=[0.2] * 3, skip_frac=[0.0] * 3)
+    assert torch.equal(a, b)
+    ia = S.sla_mask(dev[0], dev[1], 128, 0.2)
+    ib = S.sla_mask_classes(dev[0], dev[1], 128, 0.2)
+    assert torch.equal(ia, ib)
+
+
 # ---------------------------------------------------------------- full-size configurations
 
 def _full_case(S, name, per_head):
@@ -236,7 +353,10 @@ def _full_case(S, name, per_head):
     x = make_workload(w)
     check_quant(run_quant(S, x, w.block), O.quantize(x["q"], x["k"], w.block))
     items = sample_items(w.B, w.H, w.nblk, per_head=per_head, seed=w.seed)
-    st, st_sp, rec = check_attn(x, w.block, w.topk_frac, items=items, case=name)
+    if w.classes:
+        st, st_sp, rec = check_attn_classes(x, w.block, w.fracs, w.skip_frac, items=items, case=name)
+    else:
+        st, st_sp, rec = check_attn(x, w.block, w.topk_frac, items=items, case=name)
     print(json.dumps({"case": name, "out": st, "o_sparse": st_sp}))
 
 
@@ -259,6 +379,10 @@ def test_full_sweep(S, name):
 
 def test_full_720p(S):
     _full_case(S, "720p", per_head=2)
+
+
+def test_full_480p_classes(S):
+    _full_case(S, "480p_classes", per_head=4)
 
 
 def _wide_exponent_inputs(N, d, seed):
