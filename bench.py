@@ -454,6 +454,148 @@ def run_ours(args, dist):
     return line
 
 
+def run_linear(args, dist):
+    """One W8A8 linear layer per step: X quantised in the call (k_quant2d) and
+    the block-scaled INT8 GEMM (k_w8a8_gemm); the weights are quantised once
+    before timing, as a deployed layer holds them."""
+    import numpy as np
+    import torch
+
+    import int8_block_sparse_b200 as S
+    from int8_block_sparse_b200.build import build
+    from synth.linear import LINEAR_CONFIGS, make_linear_workload
+
+    build()
+    S.lib()
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    w = LINEAR_CONFIGS[args.workload]
+    d = make_linear_workload(w)
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x, wt = to_dev(d["x"]), to_dev(d["w"])
+    b = to_dev(d["bias"]) if d["bias"] is not None else None
+    wq, sw = S.w8a8_quant(wt)
+    y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        S.w8a8_linear(x, wq, sw, b, out=y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc = S.get_error()
+    if rc != 0:
+        raise SystemExit(f"device error after warm-up: {S.status_string(rc)}")
+    sampler = ClockSampler(dist.local)
+    sampler.start()
+    S.profile_read()
+    S.profile_enable(True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    S.profile_enable(False)
+    clocks = sampler.stop()
+    prof = S.profile_read()
+    rc = S.get_error()
+    if rc != 0:
+        raise SystemExit(f"device error in the timed region: {S.status_string(rc)}")
+    ms = dist.max(e0.elapsed_time(e1) / args.steps)
+    ops = 2.0 * w.M * w.N * w.K
+    value = weak_scaling_value(ops, dist.world, ms / 1e3)
+    peaks = load_peaks()
+    bf16 = float(peaks["bf16_tflops"]) if peaks else FALLBACK_BF16_TFLOPS
+    hbm = float(peaks["hbm_gbs"]) if peaks else FALLBACK_HBM_GBS
+    i8 = 2.0 * bf16
+    g_ms, g_n = prof["w8a8"]
+    g_avg = g_ms / max(g_n, 1)
+    achieved = ops / (g_avg / 1e3) / 1e12
+    roof = {"bound": "tensor", "kernel": "k_w8a8_gemm (block-scaled INT8 GEMM)", "achieved": round(achieved, 1),
+            "peak": round(i8, 1), "unit": "TOPS", "frac": round(achieved / i8, 4), "traffic": None,
+            "peak_source": ("measured (MEASURED_PEAKS.json bf16_tflops burst; int8 = 2 x bf16, nominal ratio)"
+                            if peaks else "fallback 1.59 PFLOP/s bf16 (int8 = 2 x bf16, nominal ratio)"),
+            "ops_per_launch": ops, "kernel_ms": round(g_avg, 4)}
+    # bytes a call must move: X in (bf16), X codes out and in, W codes in, Y out (bf16), bias
+    bytes_alg = float(w.M * w.K * 2 + 2 * w.M * w.K + w.N * w.K + w.M * w.N * 2 + (w.N * 2 if b is not None else 0))
+    t_tensor, t_hbm = ops / (i8 * 1e12), bytes_alg / (hbm * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    call = {"bound": "tensor" if t_tensor >= t_hbm else "hbm", "t_roof_ms": round(t_roof * 1e3, 4),
+            "t_tensor_ms": round(t_tensor * 1e3, 4), "t_hbm_ms": round(t_hbm * 1e3, 4), "bytes_alg": bytes_alg,
+            "frac": round(t_roof * 1e3 / ms, 4), "peaks": "measured (MEASURED_PEAKS.json)" if peaks else "fallback"}
+    kernels = {k: {"ms_per_call": round(v[0] / max(v[1], 1), 4), "launches": int(v[1])} for k, v in prof.items()
+               if v[1] > 0}
+    line = {
+        "metric": (f"W8A8 linear TOPS & ms/call, M={w.M} N={w.N} K={w.K} (128x128 blocks), 1 B200 "
+                   f"({w.name} workload)"),
+        "value": round(value, 2), "unit": UNIT, "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8 (int32 block sums, f32 promotion; bf16 out)",
+        "data": "synthetic (seeded, see synth/linear.py)",
+        "config": {"workload": w.describe(), "parallelism": f"replicas x{dist.world} (independent problems per rank)",
+                   "l2": f"inputs larger than L2 (X: {w.M * w.K * 2 / 1e6:.0f} MB), no flush"},
+        "roofline": roof, "roofline_call": call, "kernels": kernels,
+        "gpu_launches": int(sum(v["launches"] for v in kernels.values())), "clocks": clocks,
+    }
+    if not args.no_e2e:
+        hx = x.cpu().pin_memory()
+        hy = torch.empty((w.M, w.N), dtype=torch.bfloat16).pin_memory()
+        n = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            dx = hx.to(dev, non_blocking=True)
+            S.w8a8_linear(dx, wq, sw, b, out=y)
+            hy.copy_(y, non_blocking=True)
+            torch.cuda.synchronize(dev)
+
+        e2e_step()
+        dist.barrier()
+        t0 = time.perf_counter()
+        for _ in range(n):
+            e2e_step()
+        dt = dist.max((time.perf_counter() - t0) / n)
+        line["e2e"] = {"value": round(weak_scaling_value(ops, dist.world, dt), 2), "unit": UNIT,
+                       "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": hy.numel() * 2,
+                       "ms_per_step": round(dt * 1e3, 3), "steps": n,
+                       "timer": "host wall clock: pinned X to the device, w8a8_linear, Y back, synchronised"}
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
+        dt, rows = linear_oracle_sample(w, d, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(2.0 * rows * w.N * w.K / dt / 1e12, 6), "unit": UNIT,
+                                "cores": oracle_threads(), "kind": "oracle",
+                                "sample": (f"W8A8 oracle (numpy, float64 BLAS for the exact integer block sums) on "
+                                           f"the first {rows} rows of X of {w.name}: their quantisation and the "
+                                           f"block-scaled product with all N columns; value = 2 * rows * N * K / "
+                                           f"wall time"), "seconds": round(dt, 2)}
+    return line
+
+
+def linear_oracle_sample(w, d, budget_s):
+    """Time the W8A8 oracle on 128-row blocks of X (quantisation + product with
+    the pre-quantised weights), block 0 first, until about budget_s seconds."""
+    from oracle import w8a8_oracle as W
+
+    wq, sw = W.quantize_2d(d["w"])
+    dt, rows = 0.0, 0
+    for rb in range((w.M + 127) // 128):
+        xb = d["x"][rb * 128:(rb + 1) * 128]
+        t0 = time.perf_counter()
+        xq, sx = W.quantize_2d(xb)
+        W.gemm(xq, sx, wq, sw, d["bias"])
+        dt += time.perf_counter() - t0
+        rows += xb.shape[0]
+        if dt >= budget_s:
+            break
+    return dt, rows
+
+
 def run_e2e(S, t, w, args, dist):
     """Same metric through the host-buffer entry point: H2D of q, k, v, proj,
     the operator, D2H of out, every step (host wall clock around the
@@ -476,6 +618,48 @@ def run_e2e(S, t, w, args, dist):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(dt * 1e3, 3),
             "steps": n, "timer": "host wall clock around the synchronous host-buffer call "
                                  f"({'sla_attn_classes_host' if w.classes else 'sla_attn_host'})"}
+
+
+def run_reference_linear(args, dist):
+    """The W8A8 oracle as the reference arm: each step quantises one 128-row
+    block of X and multiplies it with the pre-quantised weights (all N
+    columns), the blocks taken in turn."""
+    from oracle import w8a8_oracle as W
+    from synth.linear import LINEAR_CONFIGS, make_linear_workload
+
+    w = LINEAR_CONFIGS[args.workload]
+    n = args.warmup + args.steps
+    nrb = (w.M + 127) // 128
+    rows = sorted({r for s_ in range(n) for r in range((s_ % nrb) * 128, min(w.M, (s_ % nrb) * 128 + 128))})
+    d = make_linear_workload(w, rows=rows)
+    pos = {r: t for t, r in enumerate(rows)}
+    wq, sw = W.quantize_2d(d["w"])
+
+    def step(s_):
+        rb = s_ % nrb
+        lo, hi = rb * 128, min(w.M, rb * 128 + 128)
+        xq, sx = W.quantize_2d(d["x"][pos[lo]:pos[lo] + (hi - lo)])
+        W.gemm(xq, sx, wq, sw, d["bias"])
+        return hi - lo
+
+    for s_ in range(args.warmup):
+        step(s_)
+    t0 = time.perf_counter()
+    done = sum(step(s_) for s_ in range(args.warmup, n))
+    dt = time.perf_counter() - t0
+    value = 2.0 * done * w.N * w.K / dt / 1e12
+    ms_call = dt / max(done, 1) * w.M * 1e3
+    metric = f"W8A8 linear TOPS & ms/call, M={w.M} N={w.N} K={w.K} (128x128 blocks), 1 B200 ({w.name} workload)"
+    sample = (f"W8A8 oracle (numpy), {args.steps} steps of one 128-row block of X of {w.name} "
+              f"(quantisation + product with all N columns)")
+    return {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": UNIT, "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_call, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (int8 codes)",
+            "data": "synthetic (seeded, see synth/linear.py)",
+            "config": {"workload": w.describe(), "note": "ms_per_step = projected time of one full call"},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def run_reference(args, dist):
@@ -530,7 +714,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["tiny", "480p", "720p", "dense", "sweep0.05", "sweep0.10", "sweep0.20", "sweep0.40",
-                             "480p_classes"])
+                             "480p_classes", "w8a8_14b_ffn", "w8a8_14b_proj", "w8a8_1b3_ffn", "w8a8_small"])
     ap.add_argument("--cpu-heads", type=int, default=6,
                     help="most heads of the workload the CPU oracle baseline runs in full")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
@@ -551,12 +735,12 @@ def main(argv=None):
 
         d = _D()
         d.rank, d.world = 0, world
-        line = run_reference(args, d)
+        line = run_reference_linear(args, d) if args.workload.startswith("w8a8") else run_reference(args, d)
         print(json.dumps(line), flush=True)
         return 0
     dist = Dist(args.gpus)
     try:
-        line = run_ours(args, dist)
+        line = run_linear(args, dist) if args.workload.startswith("w8a8") else run_ours(args, dist)
         if dist.rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -11,7 +11,9 @@
  *        (blog.gitcode.com), section "SageSLA" and the T2V parameter list
  *        (--attention_type sagesla, --sla_topk 0.1 = keep 10%);
  *   [P4] "TurboDiffusion: 即時AI影片生成的重大突破" (bonega.ai), section
- *        "SLA: 稀疏線性注意力".
+ *        "SLA: 稀疏線性注意力";
+ *   [P5] "TuroDiffusion：为高质量视频'系统性提速'" (chooseai.net), the
+ *        linear-layer acceleration paragraph (W8A8 on 128x128 blocks).
  * The pages give no formulas; the exact semantics implemented here are:
  *   1. mu = per-channel mean of K over the N tokens (exact sum, rounded once to
  *      float32, for every finite input); K_s = float32(K) - mu.  ([P1] 三(一) item 1, "outlier smoothing")
@@ -212,6 +214,39 @@ int sla_attn_host(const void* q, const void* k, const void* v, const void* proj,
 int sla_attn_classes_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
                           int N, int d, int block, const float* topk_frac, const float* skip_frac);
 
+/* ---------------------------------------------------------------------------
+ * W8A8 linear layer ([P1] 三(四) item 1: weights and activations in 8 bits,
+ * quantisation parameters per 128x128 block, activations quantised at run
+ * time; [P5] the chooseai.net news page, linear-layer acceleration: both on
+ * 128x128 blocks).  Y = X . W^T + bias, X bf16 [M, K], W [N, K] (out_features
+ * x in_features), bias bf16 [N] or NULL.
+ *   Quantisation of a [R, K] bf16 matrix: blocks of 128 rows x 128 columns
+ *   (the last ones partial); per block s = float32(max|x| / 127) and codes
+ *   clamp(round_half_even(float32(x / s)), -127, 127) (an all-zero block:
+ *   s = 0, codes 0).
+ *   Product: Y[m, n] = sum over column blocks kb of P_kb[m, n] *
+ *   float32(sx[m/128][kb] * sw[n/128][kb]), P_kb the exact int32 sum of the
+ *   int8 products of block kb, accumulated in float32 in kb order, plus
+ *   bias[n]; stored as bf16 (round to nearest even) or float32.
+ * Supported: M, N, K >= 1, K and N multiples of 16.  Row-major, 16-byte
+ * aligned device pointers; `stream` as above. */
+
+/*   x      : in,  bf16 [R, K]
+ *   codes  : out, int8 [R, K]
+ *   scales : out, float [ceil(R/128), ceil(K/128)] */
+int sla_w8a8_quant(const void* x, int R, int K, int8_t* codes, float* scales, void* stream);
+
+/*   xq, sx : in, the codes and scales of X (sla_w8a8_quant)
+ *   wq, sw : in, the codes and scales of W (sla_w8a8_quant of W [N, K])
+ *   y      : out, [M, N] of type out_dtype (SLA_OUT_BF16 or SLA_OUT_F32) */
+int sla_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias, void* y,
+                  int out_dtype, int M, int N, int K, void* stream);
+
+/* The layer with the activations quantised in the call (dynamic): X's codes
+ * and scales go to temporary memory from the library's stream-ordered pool. */
+int sla_w8a8_linear(const void* x, const int8_t* wq, const float* sw, const void* bias, void* y, int out_dtype, int M,
+                    int N, int K, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  The word is shared by every stream of the device: a code
  * recorded by kernels on another stream is reported here as well, and cleared.
@@ -228,7 +263,9 @@ typedef enum {
   SLA_K_MASK = 3,    /* pooled scores + top-k                        */
   SLA_K_ATTN = 4,    /* critical-block attention + linear part       */
   SLA_K_LINGEMM = 5, /* sums of the non-selected states              */
-  SLA_K_COUNT = 6
+  SLA_K_QUANT2D = 6, /* W8A8: 128x128 block quantisation             */
+  SLA_K_W8A8 = 7,    /* W8A8: block-scaled INT8 GEMM                 */
+  SLA_K_COUNT = 8
 } sla_kernel_kind;
 
 /* Measurement support (no counterpart on the pages).  While enabled, every

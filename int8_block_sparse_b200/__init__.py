@@ -23,9 +23,9 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
 EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
            "sla_get_error", "sla_status_string", "sla_profile_enable", "sla_profile_read",
            "sla_mask_noalloc", "sla_selftest_wait_timeout", "sla_head_counts", "sla_mask_classes",
-           "sla_attn_classes", "sla_attn_classes_host")
+           "sla_attn_classes", "sla_attn_classes_host", "sla_w8a8_quant", "sla_w8a8_gemm", "sla_w8a8_linear")
 
-KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm")
+KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm", "quant2d", "w8a8")
 
 OUT_BF16, OUT_F32 = 0, 1
 
@@ -59,6 +59,9 @@ def lib() -> ctypes.CDLL:
         L.sla_mask_classes.argtypes = [vp] * 4 + [i] * 5 + [vp, vp, vp]
         L.sla_attn_classes.argtypes = [vp] * 5 + [i] + [vp] * 2 + [i] * 5 + [vp, vp, vp]
         L.sla_attn_classes_host.argtypes = [vp] * 5 + [i] * 5 + [vp, vp]
+        L.sla_w8a8_quant.argtypes = [vp, i, i, vp, vp, vp]
+        L.sla_w8a8_gemm.argtypes = [vp] * 6 + [i] * 4 + [vp]
+        L.sla_w8a8_linear.argtypes = [vp] * 5 + [i] * 4 + [vp]
         L.sla_get_error.argtypes = [vp]
         L.sla_status_string.argtypes = [i]
         L.sla_status_string.restype = ctypes.c_char_p
@@ -259,6 +262,53 @@ def sla_attn_classes_host(q, k, v, proj, out, block: int = 128, topk_frac=0.1, s
     tf, sf = _head_fracs(H, topk_frac, skip_frac)
     _check(lib().sla_attn_classes_host(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
                                        _cptr(tf), _cptr(sf)), "sla_attn_classes_host")
+
+
+def w8a8_quant(x, stream=None, check: bool = False):
+    """128x128 block quantisation of a bf16 [R, K] matrix: (codes int8 [R, K], scales [ceil(R/128), ceil(K/128)])."""
+    import torch
+
+    if x.dim() != 2:
+        raise ValueError("x must be [R, K]")
+    R, K = (int(t) for t in x.shape)
+    codes = torch.empty((R, K), dtype=torch.int8, device=x.device)
+    scales = torch.empty(((R + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=x.device)
+    _check(lib().sla_w8a8_quant(_ptr(x), R, K, _ptr(codes), _ptr(scales), _stream(stream)), "sla_w8a8_quant")
+    _after(check, stream, "sla_w8a8_quant")
+    return codes, scales
+
+
+def _y_for(M, N, out, out_dtype, device):
+    import torch
+
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=device)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out must be bf16 or float32")
+    return out, (OUT_F32 if out.dtype == torch.float32 else OUT_BF16)
+
+
+def w8a8_gemm(xq, sx, wq, sw, bias=None, out=None, out_dtype=None, stream=None, check: bool = False):
+    """Y = X . W^T + bias from the codes and scales of X [M, K] and W [N, K]."""
+    M, K = (int(t) for t in xq.shape)
+    N = int(wq.shape[0])
+    y, kind = _y_for(M, N, out, out_dtype, xq.device)
+    _check(lib().sla_w8a8_gemm(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), kind, M, N, K,
+                               _stream(stream)), "sla_w8a8_gemm")
+    _after(check, stream, "sla_w8a8_gemm")
+    return y
+
+
+def w8a8_linear(x, wq, sw, bias=None, out=None, out_dtype=None, stream=None, check: bool = False):
+    """The W8A8 layer on bf16 activations x [M, K] (quantised in the call) and
+    pre-quantised weights (wq [N, K], sw from w8a8_quant)."""
+    M, K = (int(t) for t in x.shape)
+    N = int(wq.shape[0])
+    y, kind = _y_for(M, N, out, out_dtype, x.device)
+    _check(lib().sla_w8a8_linear(_ptr(x), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(y), kind, M, N, K, _stream(stream)),
+           "sla_w8a8_linear")
+    _after(check, stream, "sla_w8a8_linear")
+    return y
 
 
 def profile_enable(on: bool = True) -> None:

@@ -6,6 +6,9 @@
 //   K3 k_mask          pooled scores + top-k                 (k_mask.cuh)
 //   K5 k_lingemm       sums of the non-selected states       (k_linear.cuh)
 //   K4 k_attn          critical-block attention + linear part (k_attn.cuh)
+// and of the W8A8 linear layer
+//      k_quant2d       128x128 block quantisation               (k_w8a8.cuh)
+//      k_w8a8_gemm     block-scaled INT8 GEMM                   (k_w8a8.cuh)
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -21,6 +24,7 @@
 #include "k_mask.cuh"
 #include "k_quant.cuh"
 #include "k_stats.cuh"
+#include "k_w8a8.cuh"
 
 using namespace sla;
 
@@ -527,6 +531,61 @@ void* noalloc_scratch() {
   return addr[dev];
 }
 
+// ------------------------------------------------------------------ W8A8 linear layer
+int w8a8_check(int M, int N, int K) {
+  if (M < 1 || N < 1 || K < 1) return SLA_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % 16 != 0) return SLA_ERR_UNSUPPORTED;
+  if ((long long)M * K >= (1LL << 40) || (long long)N * K >= (1LL << 40)) return SLA_ERR_UNSUPPORTED;
+  return SLA_OK;
+}
+
+// codes and scales of a bf16 [R, K] matrix, 128x128 blocks
+int launch_quant2d(const void* x, int R, int K, int8_t* codes, float* scales, cudaStream_t st) {
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)R};
+  cuuint64_t str[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {128u, 128u};
+  if (!make_map(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SLA_ERR_CUDA;
+  cudaFuncSetAttribute(k_quant2d, cudaFuncAttributeMaxDynamicSharedMemorySize, kQ2Smem);
+  dim3 g((unsigned)((K + 127) / 128), (unsigned)((R + 127) / 128));
+  ProfScope ps(SLA_K_QUANT2D, st);
+  k_quant2d<<<g, 256, kQ2Smem, st>>>(m, R, K, codes, scales);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias, void* y,
+                     bool out_f32, int M, int N, int K, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t str[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {128u, 128u};
+    if (!make_map(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, xq, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
+    cuuint64_t str[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {128u, 256u};
+    if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, wq, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SLA_ERR_CUDA;
+  }
+  W8A8Params p;
+  p.sx = sx; p.sw = sw; p.bias = static_cast<const __nv_bfloat16*>(bias); p.y = y;
+  p.M = M; p.N = N; p.K = K; p.KB = (K + 127) / 128;
+  p.tiles_n = (N + 255) / 256;
+  const long long tiles = (long long)((M + 127) / 128) * p.tiles_n;
+  if (tiles >= (1LL << 31)) return SLA_ERR_UNSUPPORTED;
+  p.tiles = (int)tiles;
+  p.out_f32 = out_f32 ? 1 : 0;
+  cudaFuncSetAttribute(k_w8a8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+  const int ctas = (int)std::min<long long>(num_sms(), tiles);
+  ProfScope ps(SLA_K_W8A8, st);
+  k_w8a8_gemm<<<ctas, WG_THREADS, WG_SMEM, st>>>(ma, mb, p);
+  return cuda_status(cudaGetLastError());
+}
+
 // ------------------------------------------------------------------ host-buffer entry point
 // Streams and events of sla_attn_host, created once per device and kept (a
 // call holds the device's set for its duration).
@@ -836,6 +895,43 @@ int sla_attn_classes_host(const void* q, const void* k, const void* v, const voi
                           int N, int d, int block, const float* topk_frac, const float* skip_frac) {
   if (topk_frac == nullptr) return SLA_ERR_INVALID_ARG;
   return attn_host(q, k, v, proj, out, B, H, N, d, block, 0.f, topk_frac, skip_frac);
+}
+
+int sla_w8a8_quant(const void* x, int R, int K, int8_t* codes, float* scales, void* stream) {
+  if (!x || !codes || !scales) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes)) return SLA_ERR_INVALID_ARG;
+  const int rc = w8a8_check(R, 16, K);
+  if (rc) return rc;
+  return launch_quant2d(x, R, K, codes, scales, static_cast<cudaStream_t>(stream));
+}
+
+int sla_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias, void* y,
+                  int out_dtype, int M, int N, int K, void* stream) {
+  if (!xq || !sx || !wq || !sw || !y) return SLA_ERR_INVALID_ARG;
+  if (out_dtype != SLA_OUT_BF16 && out_dtype != SLA_OUT_F32) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y) || !aligned16(bias)) return SLA_ERR_INVALID_ARG;
+  const int rc = w8a8_check(M, N, K);
+  if (rc) return rc;
+  return launch_w8a8_gemm(xq, sx, wq, sw, bias, y, out_dtype == SLA_OUT_F32, M, N, K,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int sla_w8a8_linear(const void* x, const int8_t* wq, const float* sw, const void* bias, void* y, int out_dtype, int M,
+                    int N, int K, void* stream) {
+  if (!x || !wq || !sw || !y) return SLA_ERR_INVALID_ARG;
+  if (out_dtype != SLA_OUT_BF16 && out_dtype != SLA_OUT_F32) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(y) || !aligned16(bias)) return SLA_ERR_INVALID_ARG;
+  int rc = w8a8_check(M, N, K);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t cb = rounded<int8_t>((size_t)M * K);
+  const size_t sb = rounded<float>((size_t)((M + 127) / 128) * ((K + 127) / 128));
+  Scratch sc;
+  if ((rc = sc.get(cb + sb, st))) return rc;
+  int8_t* xq = static_cast<int8_t*>(sc.ptr);
+  float* sx = reinterpret_cast<float*>(static_cast<char*>(sc.ptr) + cb);
+  if ((rc = launch_quant2d(x, M, K, xq, sx, st))) return rc;
+  return launch_w8a8_gemm(xq, sx, wq, sw, bias, y, out_dtype == SLA_OUT_F32, M, N, K, st);
 }
 
 int sla_profile_enable(int on) {

@@ -84,9 +84,11 @@ def gemm(xq: np.ndarray, sx: np.ndarray, wq: np.ndarray, sw: np.ndarray, bias_bi
     nb = np.arange(N) // BLOCK
     for kb in range(nblocks(K)):
         cols = slice(kb * BLOCK, (kb + 1) * BLOCK)
-        P = xq[rows, cols].astype(np.int64) @ wq[:, cols].astype(np.int64).T     # exact integers
+        # exact integers: every product and partial sum is an integer of
+        # magnitude <= 128 * 127^2 < 2^53, so the float64 matmul is exact
+        P = xq[rows, cols].astype(np.float64) @ wq[:, cols].astype(np.float64).T
         s = sx[mb, kb].astype(np.float64)[:, None] * sw[nb, kb].astype(np.float64)[None, :]
-        t = P.astype(np.float64) * s
+        t = P * s
         y += t
         a += np.abs(t)
     if bias_bits is not None:

@@ -51,7 +51,7 @@ LINEAR_CONFIGS = {
     # Wan2.1-1.3B FFN up-projection
     "w8a8_1b3_ffn": LinearWorkload("w8a8_1b3_ffn", 32760, 8960, 1536, 103),
     # small ragged case (no dimension a multiple of 128)
-    "w8a8_small": LinearWorkload("w8a8_small", 1000, 520, 656, 104),
+    "w8a8_small": LinearWorkload("w8a8_small", 1000, 528, 656, 104),
 }
 
 

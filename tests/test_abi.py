@@ -147,3 +147,46 @@ def test_binding_marshals_the_class_entry_points(monkeypatch):
     assert calls[3][1][11] is None                  # no skip fractions: NULL
     with pytest.raises(ValueError):
         S.sla_attn_classes(q, q, q, q, topk_frac=[0.1, 0.2, 0.3], stream=FakeStream())
+
+
+def test_w8a8_entry_points_refuse_invalid_arguments_without_a_gpu():
+    L = S.lib()
+    dummy = 4096
+    # shapes: K and N multiples of 16, every dimension >= 1
+    assert L.sla_w8a8_linear(dummy, dummy, dummy, None, dummy, 0, 128, 128, 100, None) == 2
+    assert L.sla_w8a8_linear(dummy, dummy, dummy, None, dummy, 0, 128, 100, 128, None) == 2
+    assert L.sla_w8a8_linear(dummy, dummy, dummy, None, dummy, 0, 0, 128, 128, None) == 1
+    assert L.sla_w8a8_gemm(dummy, dummy, dummy, dummy, None, dummy, 0, 128, 128, 0, None) == 1
+    assert L.sla_w8a8_quant(dummy, 10, 24, dummy, dummy, None) == 2
+    # null and misaligned pointers, bad output type
+    assert L.sla_w8a8_linear(None, dummy, dummy, None, dummy, 0, 128, 128, 128, None) == 1
+    assert L.sla_w8a8_linear(dummy, dummy, dummy, dummy + 8, dummy, 0, 128, 128, 128, None) == 1
+    assert L.sla_w8a8_gemm(dummy, dummy, dummy + 4, dummy, None, dummy, 0, 128, 128, 128, None) == 1
+    assert L.sla_w8a8_gemm(dummy, dummy, dummy, dummy, None, dummy, 5, 128, 128, 128, None) == 1
+    assert L.sla_w8a8_quant(dummy, 128, 128, None, dummy, None) == 1
+
+
+def test_binding_marshals_the_w8a8_entry_points(monkeypatch):
+    import torch
+
+    calls = []
+
+    class FakeLib:
+        def __getattr__(self, name):
+            return lambda *a: calls.append((name, a)) or 0
+
+    class FakeStream:
+        cuda_stream = 0
+
+    monkeypatch.setattr(S, "_lib", FakeLib())
+    x = torch.zeros((300, 256), dtype=torch.bfloat16)
+    codes, scales = S.w8a8_quant(x, stream=FakeStream())
+    assert codes.shape == (300, 256) and codes.dtype == torch.int8 and scales.shape == (3, 2)
+    wq = torch.zeros((512, 256), dtype=torch.int8)
+    y = S.w8a8_linear(x, wq, scales, None, out_dtype=torch.float32, stream=FakeStream())
+    assert y.shape == (300, 512) and y.dtype == torch.float32
+    y = S.w8a8_gemm(codes, scales, wq, scales, stream=FakeStream())
+    assert y.shape == (300, 512) and y.dtype == torch.bfloat16
+    assert [c[0] for c in calls] == ["sla_w8a8_quant", "sla_w8a8_linear", "sla_w8a8_gemm"]
+    assert calls[1][1][5:9] == (S.OUT_F32, 300, 512, 256)
+    assert calls[2][1][6:10] == (S.OUT_BF16, 300, 512, 256)
