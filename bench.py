@@ -714,7 +714,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["tiny", "480p", "720p", "dense", "sweep0.05", "sweep0.10", "sweep0.20", "sweep0.40",
-                             "480p_classes", "w8a8_14b_ffn", "w8a8_14b_proj", "w8a8_1b3_ffn", "w8a8_small"])
+                             "480p_classes", "w8a8_14b_ffn", "w8a8_14b_proj", "w8a8_1b3_ffn", "w8a8_small",
+                             "w8a8_prof"])
     ap.add_argument("--cpu-heads", type=int, default=6,
                     help="most heads of the workload the CPU oracle baseline runs in full")
     ap.add_argument("--cpu-budget", type=float, default=15.0,

@@ -25,8 +25,9 @@
 // pre-loaded with the bits of 1.5 * 2^23 (0x4B400000) and the products are
 // accumulated onto it, so the int32 result is the bit pattern of the float
 // 1.5 * 2^23 + P, exact because |P| <= 128 * 127^2 < 2^22; one subtraction
-// recovers P and one fused multiply-add adds P * s (two float32 operations
-// per element, in packed pairs).
+// recovers P and one fused multiply-add adds P * s: two float32 operations
+// per element, the subtraction packed in pairs (packed forms run on one half
+// of the FMA pipe only) and the multiply-adds scalar (either half).
 //   warp 0  TMA producer (A: 128 x 128 int8, B: 256 x 128 int8 per stage)
 //   warp 1  TMEM allocation and the MMA issuer (warps 2-3 idle)
 //   warps 4-11 promotion and epilogue: warp w owns TMEM lanes 32 (w % 4) ..
@@ -128,11 +129,23 @@ constexpr int WG_STAGE_BYTES = WG_A_BYTES + WG_B_BYTES;
 constexpr int WG_BAR_BYTES = (2 * WG_STAGES + 4 + 1) * 8 + 16;
 constexpr int WG_SMEM_USED = WG_STAGES * WG_STAGE_BYTES + WG_BAR_BYTES;
 constexpr int WG_SMEM = WG_SMEM_USED + 1024;
-constexpr int WG_THREADS = 384;
-constexpr int kW8RegsLoad = 40;
-constexpr int kW8RegsMath = 232;
-static_assert(128 * kW8RegsLoad + 256 * kW8RegsMath <= WG_THREADS * 168, "register split within the launch's");
 constexpr uint32_t kMagicBits = 0x4B400000u;        // 1.5 * 2^23
+
+constexpr int kW8PromotionWarps = 8;
+
+// PW promotion warps (8 or 16): each owns 32 TMEM lanes and 256 / (PW / 4)
+// columns of the tile; the threads' registers at launch and the split.
+template <int PW>
+struct W8Cfg {
+  static constexpr int THREADS = 128 + 32 * PW;
+  static constexpr int COLS = 256 / (PW / 4);        // columns per promotion warp
+  static constexpr int CW = PW == 8 ? 32 : 16;       // columns per TMEM load
+  static constexpr int LAUNCH_REGS = PW == 8 ? 168 : 96;
+  static constexpr int REGS_LOAD = PW == 8 ? 40 : 32;
+  static constexpr int REGS_MATH = PW == 8 ? 232 : 112;
+  static_assert(128 * REGS_LOAD + 32 * PW * REGS_MATH <= THREADS * LAUNCH_REGS, "register split within the launch's");
+  static_assert(THREADS * LAUNCH_REGS <= 65536, "registers at launch");
+};
 
 // The same 32-bit value into 32 consecutive TMEM columns of the warp's 32 lanes.
 __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t x) {
@@ -143,9 +156,22 @@ __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t x) {
       : "memory");
 }
 
-__global__ void __launch_bounds__(WG_THREADS, 1) k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_a,
-                                                             const __grid_constant__ CUtensorMap tm_b,
-                                                             const W8A8Params p) {
+// CW consecutive TMEM columns of the warp's 32 lanes into registers.
+template <int CW>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
+  if constexpr (CW == 32) {
+    SLA_TMEM_LD32(taddr, r);
+  } else {
+    static_assert(CW == 16, "16 or 32 columns");
+    SLA_TMEM_LD16(taddr, r);
+  }
+}
+
+template <int PW>
+__global__ void __launch_bounds__(W8Cfg<PW>::THREADS, 1) k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_a,
+                                                                     const __grid_constant__ CUtensorMap tm_b,
+                                                                     const W8A8Params p) {
+  using C = W8Cfg<PW>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,7 +196,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1) k_w8a8_gemm(const __grid_consta
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&t_full[q], 1);
-      mbar_init(&t_empty[q], 256);
+      mbar_init(&t_empty[q], 32 * PW);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -187,7 +213,7 @@ __global__ void __launch_bounds__(WG_THREADS, 1) k_w8a8_gemm(const __grid_consta
   // the register split and the roles in one branch each, so that the
   // promotion code is only reachable with the larger register count
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kW8RegsLoad));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_LOAD));
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
@@ -237,33 +263,36 @@ __global__ void __launch_bounds__(WG_THREADS, 1) k_w8a8_gemm(const __grid_consta
       }
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kW8RegsMath));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_MATH));
     // ------------------------------------------------------------ promotion + epilogue
     const int q4 = warp & 3;                       // TMEM lane quarter
-    const int h = (warp - 4) >> 2;                 // column half of the tile
+    const int g = (warp - 4) >> 2;                 // column group of the tile
+    const int cbase = g * C::COLS;                 // first tile column of the group
+    const int h = cbase >> 7;                      // its 128-column block (scale row of W)
     const int r = q4 * 32 + lane;                  // tile row
     const uint32_t lane_off = uint32_t(q4 * 32) << 16;
+    constexpr int NCH = C::COLS / C::CW;           // TMEM loads per k-block
     // arm both buffers
 #pragma unroll
     for (int b = 0; b < 2; ++b)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_fill32(tmem + lane_off + b * 256 + h * 128 + c * 32, kMagicBits);
+      for (int c = 0; c < C::COLS; c += 32) tmem_fill32(tmem + lane_off + b * 256 + cbase + c, kMagicBits);
     tmem_st_wait();
     tc_fence_before();
     mbar_arrive(&t_empty[0]);
     mbar_arrive(&t_empty[1]);
-    const uint64_t negc = f32x2(-12582912.f, -12582912.f);
+    const uint64_t negc2 = f32x2(-12582912.f, -12582912.f);
     uint32_t n = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
       const int m0 = (t / p.tiles_n) * 128, n0 = (t % p.tiles_n) * 256;
       const int mb = m0 >> 7, nb = (n0 >> 7) + h;
-      const bool nb_ok = n0 + h * 128 < p.N;
+      const bool nb_ok = n0 + cbase < p.N;
       const float* sxr = p.sx + (long long)mb * p.KB;
       const float* swr = p.sw + (long long)(nb_ok ? nb : 0) * p.KB;
-      uint64_t acc[64];
+      float acc[C::COLS];
 #pragma unroll
-      for (int e = 0; e < 64; ++e) acc[e] = 0ull;   // (+0.0f, +0.0f)
+      for (int e = 0; e < C::COLS; ++e) acc[e] = 0.f;
       float sxn = __ldg(sxr), swn = __ldg(swr);
       for (int kb = 0; kb < p.KB; ++kb, ++n) {
         const float sc = sxn * swn;                 // one float32 rounding of the scale product
@@ -271,39 +300,49 @@ __global__ void __launch_bounds__(WG_THREADS, 1) k_w8a8_gemm(const __grid_consta
           sxn = __ldg(sxr + kb + 1);
           swn = __ldg(swr + kb + 1);
         }
-        const uint64_t s2 = f32x2(sc, sc);
         const uint32_t b = n & 1;
         if (!(ok = mbar_wait(&t_full[b], (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint32_t tb = tmem + lane_off + b * 256 + h * 128;
+        const uint32_t tb = tmem + lane_off + b * 256 + cbase;
+        // chunk c + 1 is read from TMEM while chunk c is added up
+        uint32_t v[2][C::CW];
+        tmem_ld_cols<C::CW>(tb, v[0]);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          SLA_TMEM_LD32(tb + c * 32, v);
-          tmem_ld_wait();
-          tmem_fill32(tb + c * 32, kMagicBits);     // re-arm this chunk for the k-block after next
+        for (int c = 0; c < NCH; ++c) {
+          tmem_ld_wait();                            // chunk c has landed
+          if (c + 1 < NCH) tmem_ld_cols<C::CW>(tb + (c + 1) * C::CW, v[(c + 1) & 1]);
+          if ((c * C::CW) % 32 + C::CW == 32)        // re-arm the 32 columns just read (the k-block after next)
+            tmem_fill32(tb + (c * C::CW / 32) * 32, kMagicBits);
+          if (c == NCH - 1) {                        // every column read and re-armed: release the buffer
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&t_empty[b]);
+          }
+          const uint32_t* w = v[c & 1];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const uint64_t f = add_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), negc);  // = P exactly
-            acc[c * 16 + e / 2] = fma_f32x2(f, s2, acc[c * 16 + e / 2]);
+          for (int e = 0; e < C::CW; e += 2) {
+            // P of a pair exactly by one packed subtraction (the packed forms
+            // run on one half of the FMA pipe), then two scalar fused
+            // multiply-adds (either half)
+            float p0, p1;
+            f32x2_split(add_f32x2(f32x2(__uint_as_float(w[e]), __uint_as_float(w[e + 1])), negc2), p0, p1);
+            acc[c * C::CW + e] = fmaf(p0, sc, acc[c * C::CW + e]);
+            acc[c * C::CW + e + 1] = fmaf(p1, sc, acc[c * C::CW + e + 1]);
           }
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&t_empty[b]);
       }
       if (!ok) break;
-      // epilogue: + bias, store the row's 128 columns
+      // epilogue: + bias, store the row's columns
       const long long row = (long long)m0 + r;
-      const int c0 = n0 + h * 128;
+      const int c0 = n0 + cbase;
       if (row < p.M && c0 < p.N) {
-        const int ncols = min(128, p.N - c0);      // a multiple of 16
+        const int ncols = min(C::COLS, p.N - c0);   // a multiple of 16
 #pragma unroll
-        for (int c = 0; c < 128; c += 16) {
+        for (int c = 0; c < C::COLS; c += 16) {
           if (c >= ncols) break;
           float o[16];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) f32x2_split(acc[(c + e) / 2], o[e], o[e + 1]);
+          for (int e = 0; e < 16; ++e) o[e] = acc[c + e];
           if (p.bias != nullptr) {
             const uint4* bp = reinterpret_cast<const uint4*>(p.bias + c0 + c);
 #pragma unroll

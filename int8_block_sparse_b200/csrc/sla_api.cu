@@ -579,10 +579,11 @@ int launch_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const 
   if (tiles >= (1LL << 31)) return SLA_ERR_UNSUPPORTED;
   p.tiles = (int)tiles;
   p.out_f32 = out_f32 ? 1 : 0;
-  cudaFuncSetAttribute(k_w8a8_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+  constexpr int PW = kW8PromotionWarps;
+  cudaFuncSetAttribute(k_w8a8_gemm<PW>, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
   const int ctas = (int)std::min<long long>(num_sms(), tiles);
   ProfScope ps(SLA_K_W8A8, st);
-  k_w8a8_gemm<<<ctas, WG_THREADS, WG_SMEM, st>>>(ma, mb, p);
+  k_w8a8_gemm<PW><<<ctas, W8Cfg<PW>::THREADS, WG_SMEM, st>>>(ma, mb, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -50,6 +50,8 @@ LINEAR_CONFIGS = {
     "w8a8_14b_proj": LinearWorkload("w8a8_14b_proj", 32760, 5120, 5120, 102),
     # Wan2.1-1.3B FFN up-projection
     "w8a8_1b3_ffn": LinearWorkload("w8a8_1b3_ffn", 32760, 8960, 1536, 103),
+    # a quarter of the 14B projection's rows: the case the profiler captures
+    "w8a8_prof": LinearWorkload("w8a8_prof", 8192, 5120, 5120, 105),
     # small ragged case (no dimension a multiple of 128)
     "w8a8_small": LinearWorkload("w8a8_small", 1000, 528, 656, 104),
 }
