@@ -423,7 +423,9 @@ def run_ours(args, dist):
             "peak_source": peak_src, "ops_per_launch": qk + pv,
             "kernel_ms": round(attn_avg, 4)}
     launches = int(sum(n for _, n in prof.values()))
-    kernels = {k: {"ms_per_call": round(v[0] / max(v[1], 1), 4), "launches": int(v[1])} for k, v in prof.items()}
+    # per kind: summed event time per call (kernels on the two streams overlap)
+    kernels = {k: {"ms_per_call": round(v[0] / args.steps, 4), "launches": int(v[1])} for k, v in prof.items()
+               if v[1] > 0}
 
     e2e = None
     if not args.no_e2e:

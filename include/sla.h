@@ -143,7 +143,13 @@ int sla_mask_noalloc(const void* q, const void* k, int32_t* blk_idx, uint8_t* bi
  *   q, k, v : in,  bf16 [B,H,N,d]
  *   proj    : in,  bf16 [d,d]
  *   out     : out, bf16 [B,H,N,d], fully overwritten (float32 result rounded
- *             to nearest even) */
+ *             to nearest even)
+ * The kernels run on `stream` and on a second stream the library keeps per
+ * device (created at the first call), ordered by events: work enqueued on
+ * `stream` after the call sees the complete result, and the call can be
+ * captured in a CUDA graph.  The second stream is shared by all calls on the
+ * device, so the part of concurrent calls that runs there is serialised.
+ * (Also sla_attn_ex and sla_attn_classes.) */
 int sla_attn(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N,
              int d, int block, float topk_frac, void* stream);
 

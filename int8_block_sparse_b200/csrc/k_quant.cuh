@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
                                               const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ mu,
                                               int8_t* __restrict__ qi8, int8_t* __restrict__ ki8,
                                               float* __restrict__ sq, float* __restrict__ sk,
-                                              double* __restrict__ qbar, int N, int NB) {
+                                              double* __restrict__ qbar, int N, int NB, int z0) {
   using C = QuantCfg<D, BLK>;
   constexpr int VEC = 8;
   constexpr int GROUPS = D / VEC;
@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
 
   const int j = blockIdx.x;
   const int bh = blockIdx.y;
-  const bool isk = blockIdx.z == 1;
+  const bool isk = blockIdx.z + z0 == 1;   // grid z: {Q, K}, {Q} (z0 0) or {K} (z0 1)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row0 = j * BLK;
   const int rows = min(BLK, N - row0);

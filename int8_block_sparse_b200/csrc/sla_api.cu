@@ -261,10 +261,10 @@ int num_sms() {
   return n;
 }
 
+// K block sums and (states) the linear states (k_kstats), then mu (k_channel_mean).
 template <int D, int BLK>
-int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
-                       const __nv_bfloat16* proj, Workspace& w, bool states, bool kcodes, int8_t* qi8,
-                       int8_t* ki8, float* sq, float* sk, cudaStream_t st) {
+int launch_kstats(const Shape& s, const __nv_bfloat16* k, const __nv_bfloat16* v, const __nv_bfloat16* proj,
+                  Workspace& w, bool states, cudaStream_t st, cudaEvent_t after_stats = nullptr) {
   CUtensorMap mv, mw;
   std::memset(&mv, 0, sizeof(mv));
   std::memset(&mw, 0, sizeof(mw));
@@ -286,8 +286,17 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
   { ProfScope ps(SLA_K_STATS, st);
   k_kstats<D, BLK><<<g1, StatsCfg<D, BLK>::THREADS, sm1, st>>>(mv, mw, k, w.ksum, w.kbar, w.kexp, states ? w.hstate : nullptr, s.N,
                                          (int)s.NB, w.hpitch); }
+  if (after_stats != nullptr && cudaEventRecord(after_stats, st) != cudaSuccess) return SLA_ERR_CUDA;
   { ProfScope ps(SLA_K_MEAN, st);
   k_channel_mean<D><<<dim3((unsigned)s.BH, D / kMeanCG), 1024, 0, st>>>(w.ksum, w.kexp, k, w.mu, (int)s.NB, s.N); }
+  return cuda_status(cudaGetLastError());
+}
+
+// Codes, scales (and for Q the pooled blocks) of Q (which & 1) and of K - mu
+// (which & 2; needs mu) in one launch.
+template <int D, int BLK>
+int launch_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, Workspace& w, int which,
+                 int8_t* qi8, int8_t* ki8, float* sq, float* sk, cudaStream_t st) {
   CUtensorMap mq, mk;
   {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)s.N, (cuuint64_t)s.BH};
@@ -300,10 +309,20 @@ int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat
   }
   const int sm2 = QuantCfg<D, BLK>::SMEM;
   cudaFuncSetAttribute(k_quant<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2);
-  dim3 g2((unsigned)s.NB, (unsigned)s.BH, kcodes ? 2u : 1u);
+  dim3 g2((unsigned)s.NB, (unsigned)s.BH, which == 3 ? 2u : 1u);
   { ProfScope ps(SLA_K_QUANT, st);
-  k_quant<D, BLK><<<g2, 256, sm2, st>>>(mq, mk, w.mu, qi8, ki8, sq, sk, w.qbar, s.N, (int)s.NB); }
+  k_quant<D, BLK><<<g2, 256, sm2, st>>>(mq, mk, w.mu, qi8, ki8, sq, sk, w.qbar, s.N, (int)s.NB, which == 2 ? 1 : 0); }
   return cuda_status(cudaGetLastError());
+}
+
+// Both, in order (the entry points that need no overlap).
+template <int D, int BLK>
+int launch_stats_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                       const __nv_bfloat16* proj, Workspace& w, bool states, bool kcodes, int8_t* qi8,
+                       int8_t* ki8, float* sq, float* sk, cudaStream_t st) {
+  const int rc = launch_kstats<D, BLK>(s, k, v, proj, w, states, st);
+  if (rc) return rc;
+  return launch_quant<D, BLK>(s, q, k, w, kcodes ? 3 : 1, qi8, ki8, sq, sk, st);
 }
 
 template <int D, int R>
@@ -417,19 +436,68 @@ int launch_lingemm(const Shape& s, Workspace& w, cudaStream_t st) {
   return cuda_status(cudaGetLastError());
 }
 
+// ------------------------------------------------------------------ second stream of the operator
+// The operator's kernels run on two streams of the device: the caller's and
+// this one (created at the first call on a device and kept).  Its events
+// order the two; the mutex keeps one call's record/wait sequence from
+// interleaving with another's.
+struct SideStream {
+  std::mutex mu;
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, stats = nullptr, join = nullptr;
+};
+
+SideStream* side_stream() {
+  static std::mutex mu;
+  static SideStream* sets[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (sets[dev] == nullptr) {
+    SideStream* x = new SideStream();
+    if (cudaStreamCreateWithFlags(&x->st, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x->fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x->stats, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&x->join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    sets[dev] = x;
+  }
+  return sets[dev];
+}
+
 // ------------------------------------------------------------------ dispatch
 // s.kc is the pitch of the block lists (the largest count of hc); `linear`:
 // some query block has blocks in the linear branch.
+//
+// Two streams: the caller's runs k_kstats, k_channel_mean, the K half of
+// k_quant and k_attn; the side stream runs the Q half of k_quant (needs no
+// mu: it overlaps k_kstats), then, once k_kstats is done, k_mask and
+// k_lingemm (they need the pooled blocks and the states, not mu or the K
+// codes: they overlap k_channel_mean and the K quantisation).
 template <int D, int BLK>
 int run_attn(const Shape& s, const HeadCounts& hc, bool linear, const __nv_bfloat16* q, const __nv_bfloat16* k,
              const __nv_bfloat16* v, const __nv_bfloat16* proj, void* out, bool out_f32, float* o_sparse,
              float* o_lin, Workspace& w, cudaStream_t st) {
   int* kc_bh = hc.H > 1 || hc.kc[0] != s.kc ? w.kc_bh : nullptr;   // per-head list lengths
-  int rc = launch_stats_quant<D, BLK>(s, q, k, v, proj, w, linear, true, w.qi8, w.ki8, w.sq, w.sk, st);
+  SideStream* ss = side_stream();
+  if (ss == nullptr) return SLA_ERR_CUDA;
+  int rc = SLA_OK;
+  {
+    std::lock_guard<std::mutex> lk(ss->mu);
+    if (cudaEventRecord(ss->fork, st) != cudaSuccess || cudaStreamWaitEvent(ss->st, ss->fork, 0) != cudaSuccess)
+      return SLA_ERR_CUDA;
+    rc = launch_quant<D, BLK>(s, q, k, w, 1, w.qi8, w.ki8, w.sq, w.sk, ss->st);
+    if (rc == SLA_OK) rc = launch_kstats<D, BLK>(s, k, v, proj, w, linear, st, ss->stats);
+    if (rc == SLA_OK && cudaStreamWaitEvent(ss->st, ss->stats, 0) != cudaSuccess) rc = SLA_ERR_CUDA;
+    if (rc == SLA_OK) rc = launch_quant<D, BLK>(s, q, k, w, 2, w.qi8, w.ki8, w.sq, w.sk, st);
+    if (rc == SLA_OK) rc = launch_mask<D>(s, w, hc, kc_bh, w.idx, nullptr, linear ? w.notcrit : nullptr, ss->st);
+    if (rc == SLA_OK && linear) rc = launch_lingemm<D>(s, w, ss->st);
+    // the caller's stream waits for the side stream, on every path (its
+    // temporary memory is released in the caller's stream order)
+    if (cudaEventRecord(ss->join, ss->st) != cudaSuccess || cudaStreamWaitEvent(st, ss->join, 0) != cudaSuccess)
+      if (rc == SLA_OK) rc = SLA_ERR_CUDA;
+  }
   if (rc) return rc;
-  rc = launch_mask<D>(s, w, hc, kc_bh, w.idx, nullptr, linear ? w.notcrit : nullptr, st);
-  if (rc) return rc;
-  if (linear && (rc = launch_lingemm<D>(s, w, st))) return rc;
   if ((rc = launch_attn<D, BLK>(s, w, kc_bh, q, v, out, out_f32, true, linear, st))) return rc;
   // the two parts on their own, in float32 (inspection and tests)
   if (o_sparse != nullptr && (rc = launch_attn<D, BLK>(s, w, kc_bh, q, v, o_sparse, true, true, false, st)))
