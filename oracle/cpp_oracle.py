@@ -36,7 +36,7 @@ def lib() -> ctypes.CDLL:
         vp, i, f, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
         L.ora_round_bf16.argtypes = [vp, ll, vp]
         L.ora_channel_mean.argtypes = [vp, i, i, i, i, vp]
-        L.ora_quantize_blocks.argtypes = [vp, i, i, i, i, i, vp, vp]
+        L.ora_quantize_blocks.argtypes = [vp, i, i, i, i, i, i, vp, vp]
         L.ora_smooth_k.argtypes = [vp, vp, i, i, i, vp]
         L.ora_block_means.argtypes = [vp, i, i, i, i, i, vp]
         L.ora_block_probs.argtypes = [vp, vp, i, i, i, i, vp]
@@ -46,7 +46,7 @@ def lib() -> ctypes.CDLL:
         L.ora_skip_count.argtypes = [i, i, f]
         L.ora_skip_count.restype = i
         L.ora_block_classes.argtypes = [vp, ll, i, ll, i, vp, vp, i, vp, vp]
-        L.ora_sla_rows.argtypes = [vp] * 4 + [i] * 5 + [vp] * 6 + [i] * 3 + [vp, i, i] + [vp] * 3
+        L.ora_sla_rows.argtypes = [vp] * 4 + [i] * 5 + [vp] * 6 + [i] * 4 + [vp, i, i] + [vp] * 3
         L.ora_sla_rows.restype = i
         _lib = L
     return _lib
@@ -103,20 +103,27 @@ def smooth_k(k_bits: np.ndarray, mu: np.ndarray) -> np.ndarray:
     return out
 
 
-def quantize_blocks(x32: np.ndarray, block: int):
+def quantize_groups(x32: np.ndarray, block: int, gran: int):
+    if block % gran:
+        raise ValueError("gran must divide block")
     x = _c(x32, np.float32)
     B, H, N, d = x.shape
     nblk = (N + block - 1) // block
     codes = np.empty((B, H, nblk * block, d), dtype=np.int8)
-    scales = np.empty((B, H, nblk), dtype=np.float32)
-    lib().ora_quantize_blocks(_p(x), B * H, N, d, block, threads(), _p(codes), _p(scales))
+    scales = np.empty((B, H, nblk * block // gran), dtype=np.float32)
+    lib().ora_quantize_blocks(_p(x), B * H, N, d, block, gran, threads(), _p(codes), _p(scales))
     return codes, scales
 
 
-def quantize(q_bits: np.ndarray, k_bits: np.ndarray, block: int) -> dict:
+def quantize_blocks(x32: np.ndarray, block: int):
+    return quantize_groups(x32, block, block)
+
+
+def quantize(q_bits: np.ndarray, k_bits: np.ndarray, block: int, gran=None) -> dict:
     mu = channel_mean(k_bits)
-    qi8, sq = quantize_blocks(bf16_to_f32(q_bits), block)
-    ki8, sk = quantize_blocks(smooth_k(k_bits, mu), block)
+    g = block if gran is None else gran
+    qi8, sq = quantize_groups(bf16_to_f32(q_bits), block, g)
+    ki8, sk = quantize_groups(smooth_k(k_bits, mu), block, g)
     return {"mu": mu, "q_i8": qi8, "q_scale": sq, "k_i8": ki8, "k_scale": sk}
 
 
@@ -217,7 +224,8 @@ def block_mask_classes(q_bits, k_bits, block: int, topk_frac, skip_frac=None) ->
 # ---------------------------------------------------------------- the whole operator
 
 def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
-                  items=None, quant=True, pcast=True, smooth=True, idx_override=None, skip_frac=None):
+                  items=None, quant=True, pcast=True, smooth=True, idx_override=None, skip_frac=None,
+                  gran=None):
     """Same arguments and result as sla_oracle.sla_attention: {"out",
     "o_sparse", "o_lin" (before the projection): {(b, h, i): float64 rows},
     "mask", "quant"}."""
@@ -240,7 +248,7 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
         for (b, h, i), lst in (idx_override or {}).items():
             cls[b, h, i] = CLS_LINEAR
             cls[b, h, i, np.asarray(lst, dtype=np.int64)] = CLS_CRITICAL
-    qz = quantize(q, k, block) if quant else None
+    qz = quantize(q, k, block, gran) if quant else None
     mu = qz["mu"] if quant else channel_mean(k)
     if items is None:
         items = [(b, h, i) for b in range(B) for h in range(H) for i in range(nblk)]
@@ -255,7 +263,8 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
     else:
         ptrs = [None, None, None, None]
     rc = lib().ora_sla_rows(_p(q), _p(k), _p(v), _p(w), B, H, N, d, block, _p(cls),
-                            _p(_c(mu, np.float32)), *ptrs, 1 if quant else 0, 1 if pcast else 0,
+                            _p(_c(mu, np.float32)), *ptrs, block if gran is None else gran, 1 if quant else 0,
+                            1 if pcast else 0,
                             1 if smooth else 0, _p(it), n, threads(), _p(out), _p(osp), _p(olin))
     if rc != 0:
         raise RuntimeError(f"ora_sla_rows failed ({rc})")

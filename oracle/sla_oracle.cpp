@@ -263,25 +263,28 @@ void ora_channel_mean(const uint16_t* k, int BH, int N, int d, int threads, floa
   });
 }
 
-// Symmetric INT8 quantisation with one float32 scale per block of `block`
+// Symmetric INT8 quantisation with one float32 scale per group of `gran`
 // tokens x d channels (section 三(一) item 2, each sub-block has its own
-// parameters).  x: float32 [BH][N][d]; codes: int8 [BH][nblk*block][d] (rows
-// past N are 0); scales: float32 [BH][nblk].  Per block: m = max |x| over its
-// valid rows, s = float32(m / 127), code = clamp(round_half_even(float32(x /
-// s)), -127, 127); a block with m = 0 has s = 0 and zero codes.
-void ora_quantize_blocks(const float* x, int BH, int N, int d, int block, int threads, int8_t* codes,
+// parameters; gran = block: one scale per block of the mask, gran < block:
+// the finer "thread level" groups, gran dividing block).  x: float32
+// [BH][N][d]; codes: int8 [BH][nblk*block][d] (rows past N are 0); scales:
+// float32 [BH][nblk*block/gran].  Per group: m = max |x| over its valid rows,
+// s = float32(m / 127), code = clamp(round_half_even(float32(x / s)), -127,
+// 127); a group with m = 0 (or wholly past N) has s = 0 and zero codes.
+void ora_quantize_blocks(const float* x, int BH, int N, int d, int block, int gran, int threads, int8_t* codes,
                          float* scales) {
   const int nblk = (N + block - 1) / block;
-  parallel_for((long long)BH * nblk, threads, [&](long long t) {
-    const long long bh = t / nblk;
-    const int r = int(t % nblk);
-    const int lo = r * block, hi = std::min(N, lo + block);
+  const int ng = nblk * (block / gran);
+  parallel_for((long long)BH * ng, threads, [&](long long t) {
+    const long long bh = t / ng;
+    const int r = int(t % ng);
+    const int lo = r * gran, hi = std::min(N, lo + gran);
     float m = 0.f;
     for (int n = lo; n < hi; ++n)
       for (int c = 0; c < d; ++c) m = std::max(m, std::fabs(x[(bh * N + n) * d + c]));
     const float s = m / 127.0f;
-    scales[bh * nblk + r] = s;
-    for (int n = lo; n < lo + block; ++n)
+    scales[bh * ng + r] = s;
+    for (int n = lo; n < lo + gran; ++n)
       for (int c = 0; c < d; ++c) {
         int8_t q = 0;
         if (n < hi && s > 0.f) {
@@ -425,12 +428,13 @@ void ora_block_classes(const double* p, long long rows, int nblk, long long rows
 //   cls: uint8 [B][H][nblk][nblk] the class of every (query block, key
 //     block): 2 kept (exact attention), 1 linear branch, 0 left out
 //   mu: float32 [B][H][d] (the K channel mean)
-//   qi8, ki8, sq, sk: the INT8 codes and scales (quant = 1), else unused
+//   qi8, ki8, sq, sk: the INT8 codes and scales (quant = 1), else unused;
+//     one scale per `gran` tokens ([B][H][nblk*block/gran])
 //   items: n_items triples (b, h, i)
 //   out, o_sparse, o_lin: float64 [n_items][block][d] (rows past N are 0);
 //   o_lin is before the projection.
 // Readings (sections 三(一) item 3, 三(二) items 2-3):
-//   S = float32(int32(Qi8 . Ki8^T)) * float32(sq_i * sk_j) * float32(1/sqrt(d))
+//   S = float32(int32(Qi8 . Ki8^T)) * float32(sq_n * sk_m) * float32(1/sqrt(d))
 //   in float32 (quant = 0: S = Q . K_s^T / sqrt(d) in float64, K_s = K - mu
 //   when smooth = 1, else K); keys at or past N are out; softmax with the row
 //   maximum over all kept keys: P = exp(S - max) in float64, l = sum of the
@@ -442,7 +446,7 @@ void ora_block_classes(const double* p, long long rows, int nblk, long long rows
 //   O_lin W.
 int ora_sla_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* w, int B, int H, int N,
                  int d, int block, const uint8_t* cls, const float* mu, const int8_t* qi8,
-                 const int8_t* ki8, const float* sq, const float* sk, int quant, int pcast, int smooth,
+                 const int8_t* ki8, const float* sq, const float* sk, int gran, int quant, int pcast, int smooth,
                  const int32_t* items, int n_items, int threads, double* out, double* o_sparse, double* o_lin) {
   const int nblk = (N + block - 1) / block;
   const long long NP = (long long)nblk * block;
@@ -513,7 +517,8 @@ int ora_sla_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const 
           const int8_t* kb = ki8 + (bh * NP + m) * d;
           int32_t acc = 0;   // exact: |acc| <= d * 127^2
           for (int c = 0; c < d; ++c) acc += int32_t(qa[c]) * int32_t(kb[c]);
-          const float cscale = sq[bh * nblk + i] * sk[bh * nblk + m / block];
+          const long long ng = NP / gran;   // scale groups per head
+          const float cscale = sq[bh * ng + n / gran] * sk[bh * ng + m / gran];
           const float s32 = (float(acc) * cscale) * rsd_f;
           S[u] = double(s32);
         } else {

@@ -212,11 +212,37 @@ def quantize_blocks(x32: np.ndarray, block: int) -> tuple[np.ndarray, np.ndarray
     return codes, scales
 
 
-def quantize(q_bits: np.ndarray, k_bits: np.ndarray, block: int) -> dict:
-    """Everything the quantisation entry point produces: mu, smoothed-K codes, Q codes, scales."""
+def quantize_groups(x32: np.ndarray, block: int, gran: int) -> tuple[np.ndarray, np.ndarray]:
+    """quantize_blocks with one scale per ``gran`` tokens (gran divides block).
+
+    [P1] section 三(一) item 2 names finer, "thread level" quantisation
+    parameters than the attention tiles.  Reading: a scale group is ``gran``
+    consecutive tokens by all d channels, inside the same blocks as the mask
+    (block = gran is quantize_blocks itself).  It is quantize_blocks with
+    block = gran, its codes padded with zero rows to nblk * block and its
+    scales with zeros to nblk * block / gran (groups wholly past N).
+
+    Returns (codes int8 [B, H, nblk*block, d], scales float32 [B, H, nblk*block/gran]).
+    """
+    if block % gran:
+        raise ValueError("gran must divide block")
+    B, H, N, d = np.shape(x32)
+    nblk = (N + block - 1) // block
+    codes_g, scales_g = quantize_blocks(x32, gran)
+    codes = np.zeros((B, H, nblk * block, d), dtype=np.int8)
+    codes[:, :, :codes_g.shape[2]] = codes_g
+    scales = np.zeros((B, H, nblk * block // gran), dtype=np.float32)
+    scales[:, :, :scales_g.shape[2]] = scales_g
+    return codes, scales
+
+
+def quantize(q_bits: np.ndarray, k_bits: np.ndarray, block: int, gran: int | None = None) -> dict:
+    """Everything the quantisation entry point produces: mu, smoothed-K codes, Q codes, scales
+    (one scale per block, or per ``gran`` tokens)."""
     mu = channel_mean(k_bits)
-    qi8, sq = quantize_blocks(bf16_to_f32(q_bits), block)
-    ki8, sk = quantize_blocks(smooth_k(k_bits, mu), block)
+    g = block if gran is None else gran
+    qi8, sq = quantize_groups(bf16_to_f32(q_bits), block, g)
+    ki8, sk = quantize_groups(smooth_k(k_bits, mu), block, g)
     return {"mu": mu, "q_i8": qi8, "q_scale": sq, "k_i8": ki8, "k_scale": sk}
 
 
@@ -381,13 +407,15 @@ def block_mask_classes(q_bits: np.ndarray, k_bits: np.ndarray, block: int, topk_
 # critical blocks: INT8 QK^T, softmax, bf16 P, PV  ([P1] 三(一) item 3, 三(二) item 3)
 # ---------------------------------------------------------------------------
 
-def critical_rows(qi8_blk, sq_i, ki8, sk, v64, crit, N, block, *, pcast=True,
+def critical_rows(qi8_blk, sq_rows, ki8, sk_keys, v64, crit, N, block, *, pcast=True,
                   q64_blk=None, ks64=None):
     """O_sparse for the rows of one query block over its critical key blocks (float64).
 
     Quantised mode (q64_blk is None), readings of [P1] 三(一) item 3 and
-    三(二) item 3: S = float32(int32(Qi8 . Ki8^T)) * float32(sq_i * sk_j) *
-    float32(1/sqrt(d)) in float32; keys at or past N are masked; softmax with
+    三(二) item 3: S = float32(int32(Qi8 . Ki8^T)) * float32(sq_n * sk_m) *
+    float32(1/sqrt(d)) in float32, sq_n the scale of query row n (sq_rows,
+    [block]) and sk_m that of key m (sk_keys, one per padded key); keys at
+    or past N are masked; softmax with
     the row maximum over all critical keys; P = exp(S - max) (float64 here);
     the normaliser l sums the unrounded P; P is rounded to bf16 when
     ``pcast``; O = (P . V) / l.
@@ -402,8 +430,9 @@ def critical_rows(qi8_blk, sq_i, ki8, sk, v64, crit, N, block, *, pcast=True,
     valid = keys < N
     if q64_blk is None:
         acc = np.matmul(qi8_blk.astype(np.float64), ki8[keys].astype(np.float64).T)
-        c = (np.float32(sq_i) * np.repeat(sk[crit], block).astype(np.float32)).astype(np.float32)
-        S = (acc.astype(np.float32) * c[None, :]).astype(np.float32)
+        c = (np.asarray(sq_rows, dtype=np.float32)[:, None] *
+             np.asarray(sk_keys, dtype=np.float32)[keys][None, :]).astype(np.float32)
+        S = (acc.astype(np.float32) * c).astype(np.float32)
         S = (S * np.float32(1.0 / math.sqrt(d))).astype(np.float32).astype(np.float64)
     else:
         kk = np.zeros((len(keys), d))
@@ -479,14 +508,15 @@ def linear_rows(q64_blk: np.ndarray, h: np.ndarray, z: np.ndarray, crit, lin=Non
 # ---------------------------------------------------------------------------
 
 def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
-                  items=None, quant=True, pcast=True, smooth=True, idx_override=None, skip_frac=None):
+                  items=None, quant=True, pcast=True, smooth=True, idx_override=None, skip_frac=None,
+                  gran=None):
     """SageSLA attention: out = O_sparse + O_lin . W_proj.
 
     [P1] 三(二) item 3 (SLA selection, then INT8 computation on the selected
     blocks) and item 2 (the rest through the linear branch and a linear
     projection); [P3] "SageSLA" section.  Readings: W_proj multiplies O_lin on
-    the right (row vectors); no output rounding is named, so the result keeps
-    the accumulation precision (float64 here; the CUDA path returns float32).
+    the right (row vectors); the result is float64 here (the CUDA path forms
+    it in float32 and stores bf16, float32 on request).
 
     items: iterable of (b, h, i) query blocks to evaluate (default: all).
     quant/pcast/smooth: False switches off INT8 quantisation (float64 scores),
@@ -498,6 +528,8 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
     head) leaves the lowest-ranked blocks out of the linear branch; either
     one selects the three-class mask (block_mask_classes), whose "mask"
     entry is then that function's result.
+    gran: tokens per quantisation scale (default: the block; see
+    quantize_groups).
 
     Returns {"out": {(b,h,i): float64 [rows, d]}, "o_sparse", "o_lin",
     "mask": block_mask(...), "quant": quantize(...)}.
@@ -510,7 +542,8 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
         mask = block_mask_classes(q_bits, k_bits, block, topk_frac, skip_frac)
     else:
         mask = block_mask(q_bits, k_bits, block, topk_frac)
-    qz = quantize(q_bits, k_bits, block) if quant else None
+    qz = quantize(q_bits, k_bits, block, gran) if quant else None
+    g = block if gran is None else gran
     mu = qz["mu"] if quant else channel_mean(k_bits)
     w64 = bf16_to_f64(w_bits)
     if items is None:
@@ -540,8 +573,9 @@ def sla_attention(q_bits, k_bits, v_bits, w_bits, block: int, topk_frac, *,
             lo, hi = i * block, min(N, (i + 1) * block)
             if quant:
                 qi8_blk = qz["q_i8"][b, h, i * block:(i + 1) * block]
-                os_ = critical_rows(qi8_blk, qz["q_scale"][b, h, i], qz["k_i8"][b, h],
-                                    qz["k_scale"][b, h], v64, crit, N, block, pcast=pcast)
+                sq_rows = np.repeat(qz["q_scale"][b, h], g)[i * block:(i + 1) * block]
+                os_ = critical_rows(qi8_blk, sq_rows, qz["k_i8"][b, h],
+                                    np.repeat(qz["k_scale"][b, h], g), v64, crit, N, block, pcast=pcast)
             else:
                 qb = np.zeros((block, d))
                 qb[:hi - lo] = q64[lo:hi]

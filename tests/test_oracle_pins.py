@@ -487,3 +487,65 @@ def test_no_linear_class_means_no_linear_part(impl):
     for key in res["out"]:
         assert not res["o_lin"][key].any()
         assert np.array_equal(res["out"][key], res["o_sparse"][key])
+
+
+# ---------------------------------------------------------------- finer quantisation groups
+
+def test_scale_groups_are_the_maximum_over_exactly_their_tokens(impl):
+    """Per 32-token group (brute force), with a ragged N inside the last block
+    and a group wholly past N (scale 0, zero codes)."""
+    rng = np.random.default_rng(51)
+    N, d, block, gran = 200, 16, 128, 32            # nblk 2: groups 0..7, group 7 past N
+    x = (rng.standard_normal((1, 2, N, d)) * np.exp(rng.standard_normal((1, 2, N, d)))).astype(np.float32)
+    codes, scales = impl.quantize_groups(x, block, gran)
+    assert scales.shape == (1, 2, 8) and codes.shape == (1, 2, 256, d)
+    for h in range(2):
+        for g in range(8):
+            rows = [n for n in range(g * gran, (g + 1) * gran) if n < N]
+            m = max((abs(float(x[0, h, n, c])) for n in rows for c in range(d)), default=0.0)
+            assert scales[0, h, g] == np.float32(np.float32(m) / np.float32(127))
+    assert not codes[:, :, N:].any()
+    c2, s2 = O.quantize_blocks(x, gran)                  # the block quantiser with 32-token blocks
+    assert np.array_equal(codes[:, :, :c2.shape[2]], c2) and np.array_equal(scales[:, :, :s2.shape[2]], s2)
+
+
+def test_block_sized_groups_are_the_default_operator(impl):
+    x = make_inputs(1, 2, 300, 16, seed=52)
+    a = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.3)
+    b = impl.sla_attention(x["q"], x["k"], x["v"], x["proj"], 64, 0.3, gran=64)
+    for key in a["out"]:
+        assert np.array_equal(a["out"][key], b["out"][key])
+
+
+def test_32_token_groups_are_lossless_where_each_group_has_its_own_power_of_two(impl):
+    """Integer-valued Q and K rows scaled by a different power of two per 32
+    tokens (K rows in +- pairs inside each group, so mu = 0): with one scale
+    per 32 tokens the codes are the integers and the INT8 path equals the
+    float64 path up to float32 rounding of S; with one scale per 128-token
+    block it is not lossless."""
+    rng = np.random.default_rng(53)
+    N, d, block, gran = 256, 32, 128, 32
+    qi = rng.integers(-127, 128, size=(1, 1, N, d))
+    kh = rng.integers(-127, 128, size=(1, 1, N // 2, d))
+    ki = np.empty_like(qi)
+    for g in range(N // gran):            # +- pairs within each group
+        half = kh[0, 0, g * gran // 2:(g + 1) * gran // 2]
+        ki[0, 0, g * gran:(g + 1) * gran] = np.concatenate([half, -half])
+    for g in range(N // gran):
+        qi[0, 0, g * gran, 0] = 127
+        ki[0, 0, g * gran, 1], ki[0, 0, g * gran + gran // 2, 1] = 127, -127
+    pw = 2.0 ** -np.arange(4, 4 + N // gran)             # one power of two per group
+    qv = (qi * np.repeat(pw, gran)[None, None, :, None]).astype(np.float32)
+    kv = (ki * np.repeat(pw, gran)[None, None, :, None]).astype(np.float32)
+    v = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    qb, kb, vb = bits(qv), bits(kv), f32_to_bf16_bits(v)
+    wb = f32_to_bf16_bits(np.eye(d, dtype=np.float32))
+    qz = impl.quantize(qb, kb, block, gran)
+    assert not qz["mu"].any()
+    assert np.array_equal(qz["q_i8"].astype(np.int64), qi) and np.array_equal(qz["k_i8"].astype(np.int64), ki)
+    a = impl.sla_attention(qb, kb, vb, wb, block, 1.0, pcast=False, gran=gran)
+    b = impl.sla_attention(qb, kb, vb, wb, block, 1.0, pcast=False, quant=False)
+    c = impl.sla_attention(qb, kb, vb, wb, block, 1.0, pcast=False)
+    for key in a["out"]:
+        assert np.max(np.abs(a["o_sparse"][key] - b["o_sparse"][key])) <= 1e-5
+    assert max(np.max(np.abs(c["o_sparse"][k] - b["o_sparse"][k])) for k in c["out"]) > 1e-4
