@@ -58,6 +58,8 @@ def metric_for(w) -> str:
     if w.classes:
         fr = sorted(set(w.head_fracs)) if w.head_fracs else [w.topk_frac]
         pct = f"{fr[0] * 100:g}..{fr[-1] * 100:g}% per head, skip {(w.skip_frac or 0) * 100:g}%"
+    if w.gran is not None:
+        pct += f", scale per {w.gran} tokens"
     return (f"effective sparse-attn TOPS & ms/call, B={w.B} N={w.N} H={w.H} d={w.d} top-{pct}, 1 B200 "
             f"({w.name} workload)")
 
@@ -270,11 +272,19 @@ def op_attn(S, t, w, out):
         S.sla_attn_classes(t["q"], t["k"], t["v"], t["proj"], block=w.block, topk_frac=w.fracs,
                            skip_frac=w.skip_frac, out=out)
     else:
-        S.sla_attn(t["q"], t["k"], t["v"], t["proj"], block=w.block, topk_frac=w.topk_frac, out=out)
+        S.sla_attn(t["q"], t["k"], t["v"], t["proj"], block=w.block, topk_frac=w.topk_frac, out=out, gran=w.gran)
 
 
 def op_host(S, host, hout, w):
-    if w.classes:
+    if w.gran is not None:   # no host-buffer entry: the copies around the device call
+        import torch
+
+        dev = {k: v.to("cuda", non_blocking=True) for k, v in host.items()}
+        out = S.sla_attn(dev["q"], dev["k"], dev["v"], dev["proj"], block=w.block, topk_frac=w.topk_frac,
+                         gran=w.gran)
+        hout.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+    elif w.classes:
         S.sla_attn_classes_host(host["q"], host["k"], host["v"], host["proj"], hout, block=w.block,
                                 topk_frac=w.fracs, skip_frac=w.skip_frac)
     else:
@@ -296,7 +306,7 @@ def oracle_head(O, w, xs, h):
     if w.classes:
         fr = w.fracs[h] if isinstance(w.fracs, list) else w.fracs
         return O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, [fr], skip_frac=w.skip_frac)
-    return O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, w.topk_frac)
+    return O.sla_attention(xs["q"], xs["k"], xs["v"], xs["proj"], w.block, w.topk_frac, gran=w.gran)
 
 
 # ---------------------------------------------------------------- CPU oracle sample
@@ -716,7 +726,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=["tiny", "480p", "720p", "dense", "sweep0.05", "sweep0.10", "sweep0.20", "sweep0.40",
-                             "480p_classes", "w8a8_14b_ffn", "w8a8_14b_proj", "w8a8_1b3_ffn", "w8a8_small",
+                             "480p_classes", "480p_gran32", "w8a8_14b_ffn", "w8a8_14b_proj", "w8a8_1b3_ffn", "w8a8_small",
                              "w8a8_prof"])
     ap.add_argument("--cpu-heads", type=int, default=6,
                     help="most heads of the workload the CPU oracle baseline runs in full")

@@ -168,6 +168,18 @@ int sla_attn_ex(const void* q, const void* k, const void* v, const void* proj, v
                 float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, float topk_frac,
                 void* stream);
 
+/* Finer quantisation granularity ([P1] 三(一) item 2: quantisation parameters
+ * per sub-block, "thread level", finer than the attention tiles): one scale
+ * per group of `gran` tokens x d channels inside each block (gran = 32, 64 or
+ * 128, dividing block; gran = block is the default operator).  Scales are
+ * laid out [B,H,nblk*block/gran]; a group wholly past N has scale 0.  The
+ * block mask and the linear branch do not depend on it.  Q is not smoothed. */
+int sla_quant_gran(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q_scale, float* k_scale,
+                   float* k_mean, int B, int H, int N, int d, int block, int gran, void* stream);
+int sla_attn_gran(const void* q, const void* k, const void* v, const void* proj, void* out, int out_dtype,
+                  float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, float topk_frac, int gran,
+                  void* stream);
+
 /* Three block classes and per-head fractions (an extension: the pages name
  * two classes, the top-K "core" blocks of [P1] 三(二) 1 and the rest through
  * the linear branch of [P1] 三(二) 2; [P4] "SLA: 稀疏線性注意力" replaces dense

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED",
 EXPORTS = ("sla_topk_count", "sla_quant", "sla_mask", "sla_attn", "sla_attn_ex", "sla_attn_host",
            "sla_get_error", "sla_status_string", "sla_profile_enable", "sla_profile_read",
            "sla_mask_noalloc", "sla_selftest_wait_timeout", "sla_head_counts", "sla_mask_classes",
-           "sla_attn_classes", "sla_attn_classes_host", "sla_w8a8_quant", "sla_w8a8_gemm", "sla_w8a8_linear")
+           "sla_attn_classes", "sla_attn_classes_host", "sla_w8a8_quant", "sla_w8a8_gemm", "sla_w8a8_linear",
+           "sla_quant_gran", "sla_attn_gran")
 
 KERNEL_KINDS = ("stats", "mean", "quant", "mask", "attn", "lingemm", "quant2d", "w8a8")
 
@@ -60,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.sla_attn_classes.argtypes = [vp] * 5 + [i] + [vp] * 2 + [i] * 5 + [vp, vp, vp]
         L.sla_attn_classes_host.argtypes = [vp] * 5 + [i] * 5 + [vp, vp]
         L.sla_w8a8_quant.argtypes = [vp, i, i, vp, vp, vp]
+        L.sla_quant_gran.argtypes = [vp] * 7 + [i] * 6 + [vp]
+        L.sla_attn_gran.argtypes = [vp] * 5 + [i] + [vp] * 2 + [i] * 5 + [f, i, vp]
         L.sla_w8a8_gemm.argtypes = [vp] * 6 + [i] * 4 + [vp]
         L.sla_w8a8_linear.argtypes = [vp] * 5 + [i] * 4 + [vp]
         L.sla_get_error.argtypes = [vp]
@@ -119,20 +122,27 @@ def _after(check: bool, stream, where: str) -> None:
         _check(get_error(stream), where)
 
 
-def sla_quant(q, k, block: int, stream=None, check: bool = False):
-    """Smoothing + INT8 quantisation.  Returns (q_i8, k_i8, q_scale, k_scale, k_mean)."""
+def sla_quant(q, k, block: int, stream=None, check: bool = False, gran=None):
+    """Smoothing + INT8 quantisation.  Returns (q_i8, k_i8, q_scale, k_scale, k_mean);
+    one scale per block, or per ``gran`` tokens ([B, H, nblk * block / gran])."""
     import torch
 
     B, H, N, d = _shape(q)
     nb = nblk(N, block)
     dev = q.device
+    g = block if gran is None else int(gran)
     qi8 = torch.empty((B, H, nb * block, d), dtype=torch.int8, device=dev)
     ki8 = torch.empty_like(qi8)
-    sq = torch.empty((B, H, nb), dtype=torch.float32, device=dev)
+    sq = torch.empty((B, H, nb * block // g), dtype=torch.float32, device=dev)
     sk = torch.empty_like(sq)
     mu = torch.empty((B, H, d), dtype=torch.float32, device=dev)
-    _check(lib().sla_quant(_ptr(q), _ptr(k), _ptr(qi8), _ptr(ki8), _ptr(sq), _ptr(sk), _ptr(mu),
-                           B, H, N, d, block, _stream(stream)), "sla_quant")
+    if gran is None:
+        rc = lib().sla_quant(_ptr(q), _ptr(k), _ptr(qi8), _ptr(ki8), _ptr(sq), _ptr(sk), _ptr(mu),
+                             B, H, N, d, block, _stream(stream))
+    else:
+        rc = lib().sla_quant_gran(_ptr(q), _ptr(k), _ptr(qi8), _ptr(ki8), _ptr(sq), _ptr(sk), _ptr(mu),
+                                  B, H, N, d, block, g, _stream(stream))
+    _check(rc, "sla_quant")
     _after(check, stream, "sla_quant")
     return qi8, ki8, sq, sk, mu
 
@@ -153,12 +163,13 @@ def sla_mask(q, k, block: int, topk_frac: float, bitmap: bool = False, stream=No
 
 
 def sla_attn(q, k, v, proj, block: int = 128, topk_frac: float = 0.1, out=None, out_dtype=None,
-             o_sparse=None, o_lin=None, stream=None, check: bool = False):
+             o_sparse=None, o_lin=None, stream=None, check: bool = False, gran=None):
     """SageSLA attention; q, k, v bf16 [B,H,N,d], proj bf16 [d,d] on the GPU.
 
     Returns out [B,H,N,d], bf16 by default (out_dtype=torch.float32, or a
     float32 `out`, for the unrounded result).  o_sparse / o_lin (float32,
-    optional) receive the two parts, O_sparse and O_lin . W_proj."""
+    optional) receive the two parts, O_sparse and O_lin . W_proj.  gran: tokens
+    per quantisation scale (32, 64 or 128; default one scale per block)."""
     import torch
 
     B, H, N, d = _shape(q)
@@ -166,7 +177,11 @@ def sla_attn(q, k, v, proj, block: int = 128, topk_frac: float = 0.1, out=None, 
         out = torch.empty((B, H, N, d), dtype=out_dtype or torch.bfloat16, device=q.device)
     if out.dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out must be bf16 or float32")
-    if out.dtype == torch.bfloat16 and o_sparse is None and o_lin is None:
+    if gran is not None:
+        kind = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+        rc = lib().sla_attn_gran(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), kind, _ptr(o_sparse),
+                                 _ptr(o_lin), B, H, N, d, block, float(topk_frac), int(gran), _stream(stream))
+    elif out.dtype == torch.bfloat16 and o_sparse is None and o_lin is None:
         rc = lib().sla_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(proj), _ptr(out), B, H, N, d, block,
                             float(topk_frac), _stream(stream))
     else:

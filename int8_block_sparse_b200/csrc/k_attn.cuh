@@ -52,12 +52,12 @@ namespace sla {
 struct AttnParams {
   const int32_t* idx;          // [BH][NB][kcp] kept blocks, ascending
   const int* kc_bh;            // [BH] list length per head, or nullptr: kc for every head
-  const float* sq;             // [BH][NB]
-  const float* sk;             // [BH][NB]
+  const float* sq;             // [BH][NB][G] scale per group of 2^gshift query rows (G = BLK >> gshift)
+  const float* sk;             // [BH][NB][G] scale per group of 2^gshift keys
   const __nv_bfloat16* q;      // [BH][N][D] raw queries (phi(q) of the linear part)
   const float* zrest;          // [BH][NB][D] g_i: z sums over the non-selected blocks
   void* out;                   // [BH][N][D], bf16 or float32
-  int N, NB, NP, kc, kcp, items;
+  int N, NB, NP, kc, kcp, items, gshift;
   int sparse;                  // the selected blocks (softmax attention) take part
   int lin;                     // the linear part is added
   int out_f32;                 // float32 output (else bf16)
@@ -151,7 +151,9 @@ __device__ __forceinline__ float linear_den(const __nv_bfloat16* qrow, const flo
   return d0 + d1;
 }
 
-template <int D, int BLK>
+// FINE: one quantisation scale per group of 2^gshift tokens (finer than the
+// block); otherwise one per block (the default operator, its own code path).
+template <int D, int BLK, bool FINE>
 __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant__ CUtensorMap tm_q,
                                                  const __grid_constant__ CUtensorMap tm_k,
                                                  const __grid_constant__ CUtensorMap tm_v,
@@ -211,6 +213,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
   // kept blocks of the items of head bh, and the halves (64 keys) they make
   auto kc_of = [&](int bh) { return p.kc_bh != nullptr ? __ldg(p.kc_bh + bh) : p.kc; };
   auto halves_of = [&](int bh) { return sparse ? kc_of(bh) * NH : 0; };
+  const int G = FINE ? BLK >> p.gshift : 1;   // quantisation scales per block
 
   if (warp < 4)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLoad));
@@ -385,7 +388,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
     for (int item = blockIdx.x * 2 + u; sparse && item < p.items && ok; item += tiles_total) {
       const int bh = item / NB, i = item % NB;
       const int kc = kc_of(bh), H = kc * NH;
-      const float sq_i = __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale;
+      // the scale of this row's group (rows past the block reuse the last one)
+      const float sq_i = FINE ? __ldg(p.sq + ((long long)bh * NB + i) * G + (min(r, BLK - 1) >> p.gshift)) * p.qk_scale
+                              : __ldg(p.sq + (long long)bh * NB + i) * p.qk_scale;
       const int32_t* lst = p.idx + ((long long)bh * NB + i) * p.kcp;
       // running maximum m (log2 domain) and normaliser l of this row
       float m = -INFINITY, l = 0.f;
@@ -394,12 +399,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
       for (int x = 0; x < H; ++x) {
         const int t = x / NH;
         const uint32_t g = hg + x;
-        if ((t & 31) == 0 && x % NH == 0) {   // block list and scales, 32 blocks at a time
+        if ((t & 31) == 0 && x % NH == 0) {   // block list (and block scales), 32 blocks at a time
           jl = (t + lane < kc) ? __ldg(lst + t + lane) : 0;
-          cl = sq_i * __ldg(p.sk + (long long)bh * NB + jl);
+          if (!FINE) cl = sq_i * __ldg(p.sk + (long long)bh * NB + jl);
         }
         const int j = __shfl_sync(0xffffffffu, jl, t & 31);
-        const float c = __shfl_sync(0xffffffffu, cl, t & 31);   // sq_i * sk_j * log2(e) / sqrt(D) >= 0
+        // c0, c1 = sq * sk * log2(e) / sqrt(D) >= 0 for keys 0-31 and 32-63 of the half
+        float c0, c1;
+        if (!FINE) {
+          c0 = c1 = __shfl_sync(0xffffffffu, cl, t & 31);
+        } else {
+          const float* skb = p.sk + ((long long)bh * NB + j) * G;
+          const int ko = (x % NH) * C::HB;
+          c0 = sq_i * __ldg(skb + (ko >> p.gshift));
+          c1 = sq_i * __ldg(skb + ((ko + 32) >> p.gshift));
+        }
         // valid keys of this half (fewer only in a partial last block)
         const int nvalid = (part_rows != 0 && j == NB - 1)
                                ? min(max(part_rows - (x % NH) * C::HB, 0), C::HB)
@@ -421,15 +435,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
           for (int e = 0; e < 64; ++e)
             if (e >= nvalid) v[e] = 0xFF800000u;   // -inf
         }
-        float xm[8];
+        float mx;
+        if constexpr (!FINE) {
+          float xm[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) xm[q] = fmax3(__uint_as_float(v[3 * q]), __uint_as_float(v[3 * q + 1]),
-                                                  __uint_as_float(v[3 * q + 2]));
+          for (int q = 0; q < 8; ++q) xm[q] = fmax3(__uint_as_float(v[3 * q]), __uint_as_float(v[3 * q + 1]),
+                                                    __uint_as_float(v[3 * q + 2]));
 #pragma unroll
-        for (int e = 24; e < 64; e += 2)
-          xm[(e / 2) & 7] = fmax3(xm[(e / 2) & 7], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-        const float xmax = fmaxf(fmax3(xm[0], xm[1], xm[2]), fmax3(fmax3(xm[3], xm[4], xm[5]), xm[6], xm[7]));
-        const float mx = (xmax - 12582912.f) * c;   // exact difference; -inf when no key is valid
+          for (int e = 24; e < 64; e += 2)
+            xm[(e / 2) & 7] = fmax3(xm[(e / 2) & 7], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+          const float xmax = fmaxf(fmax3(xm[0], xm[1], xm[2]), fmax3(fmax3(xm[3], xm[4], xm[5]), xm[6], xm[7]));
+          mx = (xmax - 12582912.f) * c0;   // exact difference; -inf when no key is valid
+        } else {
+          // maxima of keys 0-31 and 32-63 (their scales may differ)
+          float xa[4], xb[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            xa[q] = fmax3(__uint_as_float(v[3 * q]), __uint_as_float(v[3 * q + 1]), __uint_as_float(v[3 * q + 2]));
+            xb[q] = fmax3(__uint_as_float(v[32 + 3 * q]), __uint_as_float(v[33 + 3 * q]),
+                          __uint_as_float(v[34 + 3 * q]));
+          }
+#pragma unroll
+          for (int e = 12; e < 32; e += 2) {
+            xa[(e / 2) & 3] = fmax3(xa[(e / 2) & 3], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+            xb[(e / 2) & 3] = fmax3(xb[(e / 2) & 3], __uint_as_float(v[32 + e]), __uint_as_float(v[33 + e]));
+          }
+          const float xm0 = fmaxf(fmax3(xa[0], xa[1], xa[2]), xa[3]);
+          const float xm1 = fmaxf(fmax3(xb[0], xb[1], xb[2]), xb[3]);
+          // exact differences; -inf for a group without a valid key (NaN, ignored
+          // by the maximum, if that group's scale is 0)
+          mx = fmaxf((xm0 - 12582912.f) * c0, (xm1 - 12582912.f) * c1);
+        }
         if (x == 0) {
           m = mx;
         } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
@@ -458,14 +494,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
         }
         // P = 2^(acc * c - m) = 2^((1.5*2^23 + acc) * c - (1.5*2^23 * c + m)):
         // one FMA per key (two per packed instruction); the one rounding of
-        // the constant shifts all exponents of this row and half by the same
-        // amount (< 2^-24 relative to 1.5*2^23*c), i.e. scales P and l alike.
-        const float kk = -fmaf(12582912.f, c, m);
-        const uint64_t c2 = f32x2(c, c), k2 = f32x2(kk, kk);
+        // the constant shifts all exponents of a scale group by the same
+        // amount (< 2^-24 relative to 1.5*2^23*c), i.e. scales its P and
+        // their share of l alike (with one scale per block, the whole half).
+        const float kk0 = -fmaf(12582912.f, c0, m), kk1 = FINE ? -fmaf(12582912.f, c1, m) : kk0;
+        const uint64_t c20 = f32x2(c0, c0), k20 = f32x2(kk0, kk0);
+        const uint64_t c21 = FINE ? f32x2(c1, c1) : c20, k21 = FINE ? f32x2(kk1, kk1) : k20;
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
           float y0, y1;
-          f32x2_split(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), c2, k2), y0, y1);
+          f32x2_split(fma_f32x2(f32x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), e < 32 ? c20 : c21,
+                                e < 32 ? k20 : k21),
+                      y0, y1);
           v[e] = __float_as_uint(ex2_approx(y0));
           v[e + 1] = __float_as_uint(ex2_approx(y1));
         }

@@ -4,10 +4,11 @@
 // SageAttention2++: item 1 (smooth outliers before quantising -- here K minus
 // its per-channel mean over tokens) and item 2 (every sub-block has its own
 // quantisation parameters -- here one float32 scale per block of BLK tokens x
-// D channels).  Per block: m = max|x|, s = m / 127 (IEEE float32 division),
-// code = clamp(round_half_even(float32(x / s)), -127, 127) (the clamp never
-// acts: see pack_i8x4); a block with m = 0 has s = 0 and zero codes.  Rows
-// past N (up to NB*BLK) get zero codes.  For Q the kernel also writes the
+// D channels, or, finer, one per group of 2^gshift tokens x D channels
+// inside the block: G = BLK >> gshift groups).  Per group: m = max|x|, s = m /
+// 127 (IEEE float32 division), code = clamp(round_half_even(float32(x / s)),
+// -127, 127) (the clamp never acts: see pack_i8x4); a group with m = 0 has
+// s = 0 and zero codes.  Rows past N (up to NB*BLK) get zero codes.  For Q the kernel also writes the
 // float64 mean of each block's valid rows (the pooled query block of the mask).
 //
 // The smoothed K value is recomputed (one float32 subtraction) when it is
@@ -45,19 +46,21 @@ __device__ __forceinline__ uint32_t pack_i8x4(int c0, int c1, int c2, int c3) {
 template <int D, int BLK>
 struct QuantCfg {
   static constexpr int TILE_BYTES = BLK * D * 2;            // the bf16 block, rows past N zero-filled by the TMA
-  static constexpr int RED_BYTES = 8 * D * 8 + 8 * 4;       // per-warp float64 partials, per-warp maxima
+  static constexpr int RED_BYTES = 8 * D * 8 + 8 * 4 * 4;   // per-warp float64 partials, per-warp group maxima
   static constexpr int SMEM = TILE_BYTES + RED_BYTES + 16 + 1024;
 };
 
 // The block arrives in shared memory by one TMA load (several blocks per SM
 // are in flight); pass 1 takes the maximum (and, for Q, the float64 sums),
 // pass 2 quantises from shared memory.
-template <int D, int BLK>
+// FINE: one scale per group of 2^gshift tokens inside the block (G groups);
+// otherwise one per block (the default, its own code path).
+template <int D, int BLK, bool FINE>
 __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorMap tm_q,
                                               const __grid_constant__ CUtensorMap tm_k, const float* __restrict__ mu,
                                               int8_t* __restrict__ qi8, int8_t* __restrict__ ki8,
                                               float* __restrict__ sq, float* __restrict__ sk,
-                                              double* __restrict__ qbar, int N, int NB, int z0) {
+                                              double* __restrict__ qbar, int N, int NB, int z0, int gshift) {
   using C = QuantCfg<D, BLK>;
   constexpr int VEC = 8;
   constexpr int GROUPS = D / VEC;
@@ -69,8 +72,8 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint16_t* tile = reinterpret_cast<const uint16_t*>(base);        // [BLK][D] bf16
   double* red = reinterpret_cast<double*>(base + C::TILE_BYTES);         // [8][D]
-  float* wmax = reinterpret_cast<float*>(red + 8 * D);                   // [8]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(wmax + 8);
+  float* wmax = reinterpret_cast<float*>(red + 8 * D);                   // [8 warps][4 groups]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(wmax + 32);
 
   const int j = blockIdx.x;
   const int bh = blockIdx.y;
@@ -99,8 +102,13 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
     return;
   }
 
-  // pass 1: block maximum of |x| (K: x - mu on valid rows) and, for Q, float64 channel sums
-  float mloc = 0.f;
+  // pass 1: maximum of |x| per group (K: x - mu on valid rows) and, for Q,
+  // float64 channel sums
+  constexpr int MG = FINE ? 4 : 1;              // group maxima a thread keeps
+  const int G = FINE ? BLK >> gshift : 1;       // groups per block
+  float gm[MG];
+#pragma unroll
+  for (int q = 0; q < MG; ++q) gm[q] = 0.f;
   double part[VEC];
 #pragma unroll
   for (int e = 0; e < VEC; ++e) part[e] = 0.0;
@@ -109,13 +117,18 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
     const int r = tid / GROUPS + t * RSTEP;
     const uint4 raw = *reinterpret_cast<const uint4*>(tile + r * D + g * VEC);
     const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
+    float rmax = 0.f;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       float f = __uint_as_float(uint32_t(hv[e]) << 16);
       if (!isk) part[e] += (double)f;                     // rows past N hold 0
       if (isk && r < rows) f = __fsub_rn(f, muc[e]);
-      mloc = fmaxf(mloc, fabsf(f));
+      rmax = fmaxf(rmax, fabsf(f));
     }
+    const int gi = FINE ? r >> gshift : 0;
+#pragma unroll
+    for (int q = 0; q < MG; ++q)
+      if (gi == q) gm[q] = fmaxf(gm[q], rmax);
   }
   if (!isk && qbar != nullptr) {
     // lanes sharing a channel group combine first (fixed order), then warps
@@ -128,15 +141,31 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
       for (int e = 0; e < VEC; ++e) red[warp * D + g * VEC + e] = part[e];
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
-  if ((tid & 31) == 0) wmax[warp] = mloc;
-  __syncthreads();
-  float m = wmax[0];
+  for (int q = 0; q < MG; ++q) {
 #pragma unroll
-  for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
-  const float s = __fdiv_rn(m, 127.0f);
+    for (int o = 16; o > 0; o >>= 1) gm[q] = fmaxf(gm[q], __shfl_xor_sync(0xffffffffu, gm[q], o));
+  }
+  if ((tid & 31) == 0)
+#pragma unroll
+    for (int q = 0; q < MG; ++q) wmax[warp * 4 + q] = gm[q];
+  __syncthreads();
+  float gs[MG], grs[MG];   // scale and its reciprocal per group
+#pragma unroll
+  for (int q = 0; q < MG; ++q) {
+    float m = wmax[q];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w * 4 + q]);
+    gs[q] = __fdiv_rn(m, 127.0f);
+    grs[q] = (gs[q] > 0.f) ? __frcp_rn(gs[q]) : 0.f;
+  }
   float* sdst = isk ? sk : sq;
-  if (tid == 0 && sdst != nullptr) sdst[(long long)bh * NB + j] = s;
+  if (tid < G && sdst != nullptr) {
+    float sv = gs[0];
+#pragma unroll
+    for (int q = 1; q < MG; ++q)
+      if (tid == q) sv = gs[q];
+    sdst[((long long)bh * NB + j) * G + tid] = sv;
+  }
   if (!isk && qbar != nullptr && tid < D) {
     double acc = 0.0;
 #pragma unroll
@@ -147,10 +176,17 @@ __global__ void __launch_bounds__(256) k_quant(const __grid_constant__ CUtensorM
   if (dbase == nullptr) return;
   // pass 2: codes, eight per 8-byte store
   int8_t* dst = dbase + ((long long)bh * NB * BLK + row0) * D;
-  const float rs = (s > 0.f) ? __frcp_rn(s) : 0.f;
 #pragma unroll
   for (int t = 0; t < NV; ++t) {
     const int r = tid / GROUPS + t * RSTEP;
+    const int gi = FINE ? r >> gshift : 0;
+    float s = gs[0], rs = grs[0];
+#pragma unroll
+    for (int q = 1; q < MG; ++q)
+      if (gi == q) {
+        s = gs[q];
+        rs = grs[q];
+      }
     const uint4 raw = *reinterpret_cast<const uint4*>(tile + r * D + g * VEC);
     const uint16_t* hv = reinterpret_cast<const uint16_t*>(&raw);
     uint32_t packed[2] = {0u, 0u};

@@ -34,6 +34,8 @@ namespace {
 struct Shape {
   int B, H, N, d, block;
   long long BH, NB, NP, kc;
+  int gshift;   // log2 of the tokens per quantisation scale (the block by default)
+  long long G() const { return (long long)block >> gshift; }
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -42,6 +44,7 @@ int check_shape(int B, int H, int N, int d, int block, Shape* s) {
   if (B < 1 || H < 1 || N < 1 || d < 1 || block < 1) return SLA_ERR_INVALID_ARG;
   if (!(d == 64 || d == 128) || !(block == 64 || block == 128)) return SLA_ERR_UNSUPPORTED;
   s->B = B; s->H = H; s->N = N; s->d = d; s->block = block;
+  s->gshift = block == 128 ? 7 : 6;
   s->BH = (long long)B * H;
   s->NB = (N + block - 1) / block;
   s->NP = s->NB * block;
@@ -58,6 +61,14 @@ long long topk_count_ll(long long nblk, float frac) {
 }
 
 bool frac_ok(float f) { return f > 0.f && f <= 1.f; }
+
+// Tokens per quantisation scale: 32, 64 or 128, dividing the block.
+int set_gran(Shape* s, int gran) {
+  if (!(gran == 32 || gran == 64 || gran == 128)) return SLA_ERR_UNSUPPORTED;
+  if (gran > s->block) return SLA_ERR_UNSUPPORTED;
+  s->gshift = gran == 32 ? 5 : (gran == 64 ? 6 : 7);
+  return SLA_OK;
+}
 bool skip_ok(float f) { return f >= 0.f && f < 1.f; }
 
 long long skip_count_ll(long long nblk, long long kc, float frac) {
@@ -177,7 +188,7 @@ size_t workspace_bytes(const Shape& s, int what) {
   const size_t ncpitch = (NB + 63) / 64 * 64, hpitch = d * d + d;
   size_t b = rounded<double>(BH * NB * d) * 2 + rounded<double>(BH * d * (size_t)kbar_pitch((int)NB)) +
              rounded<uint8_t>(BH * NB * d * 2) + rounded<float>(BH * d);
-  if (what & 1) b += rounded<int8_t>(BH * NP * d) * 2 + rounded<float>(BH * NB) * 2;
+  if (what & 1) b += rounded<int8_t>(BH * NP * d) * 2 + rounded<float>(BH * NB * (size_t)s.G()) * 2;
   if (what & 2) b += rounded<int32_t>(BH * NB * kc) + rounded<int>(BH);
   if (what & 8)
     b += rounded<__nv_bfloat16>(BH * NB * ncpitch) + rounded<__nv_bfloat16>(BH * NB * hpitch) +
@@ -200,8 +211,8 @@ Workspace carve(const Shape& s, int what, char* base) {
   if (what & 1) {
     w.qi8 = a.take<int8_t>(BH * NP * d);
     w.ki8 = a.take<int8_t>(BH * NP * d);
-    w.sq = a.take<float>(BH * NB);
-    w.sk = a.take<float>(BH * NB);
+    w.sq = a.take<float>(BH * NB * (size_t)s.G());
+    w.sk = a.take<float>(BH * NB * (size_t)s.G());
   }
   if (what & 2) {
     w.idx = a.take<int32_t>(BH * NB * kc);
@@ -308,10 +319,12 @@ int launch_quant(const Shape& s, const __nv_bfloat16* q, const __nv_bfloat16* k,
       return SLA_ERR_CUDA;
   }
   const int sm2 = QuantCfg<D, BLK>::SMEM;
-  cudaFuncSetAttribute(k_quant<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2);
   dim3 g2((unsigned)s.NB, (unsigned)s.BH, which == 3 ? 2u : 1u);
+  const bool fine = s.G() > 1;
+  auto kq = fine ? k_quant<D, BLK, true> : k_quant<D, BLK, false>;
+  cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, sm2);
   { ProfScope ps(SLA_K_QUANT, st);
-  k_quant<D, BLK><<<g2, 256, sm2, st>>>(mq, mk, w.mu, qi8, ki8, sq, sk, w.qbar, s.N, (int)s.NB, which == 2 ? 1 : 0); }
+  kq<<<g2, 256, sm2, st>>>(mq, mk, w.mu, qi8, ki8, sq, sk, w.qbar, s.N, (int)s.NB, which == 2 ? 1 : 0, s.gshift); }
   return cuda_status(cudaGetLastError());
 }
 
@@ -393,14 +406,16 @@ int launch_attn(const Shape& s, Workspace& w, const int* kc_bh, const __nv_bfloa
   p.idx = w.idx; p.sq = w.sq; p.sk = w.sk; p.q = q; p.zrest = w.zrest; p.out = out;
   p.kc_bh = kc_bh;
   p.N = s.N; p.NB = (int)s.NB; p.NP = (int)s.NP; p.kc = (int)s.kc; p.kcp = (int)s.kc; p.items = (int)(s.BH * s.NB);
+  p.gshift = s.gshift;
   p.sparse = sparse ? 1 : 0;
   p.lin = lin ? 1 : 0;
   p.out_f32 = out_f32 ? 1 : 0;
   p.qk_scale = (float)(1.4426950408889634 / std::sqrt((double)D));
-  cudaFuncSetAttribute(k_attn<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  auto ka = s.G() > 1 ? k_attn<D, BLK, true> : k_attn<D, BLK, false>;
+  cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int ctas = (int)std::min<long long>(num_sms(), (p.items + 1) / 2);
   ProfScope ps(SLA_K_ATTN, st);
-  k_attn<D, BLK><<<ctas, kAttnThreads, C::SMEM, st>>>(mq, mk, mv, mg, p);
+  ka<<<ctas, kAttnThreads, C::SMEM, st>>>(mq, mk, mv, mg, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -566,10 +581,10 @@ bool noalloc_load_kernels() {
   load((const void*)k_kstats<128, 128>);
   load((const void*)k_channel_mean<64>);
   load((const void*)k_channel_mean<128>);
-  load((const void*)k_quant<64, 64>);
-  load((const void*)k_quant<64, 128>);
-  load((const void*)k_quant<128, 64>);
-  load((const void*)k_quant<128, 128>);
+  load((const void*)k_quant<64, 64, false>);
+  load((const void*)k_quant<64, 128, false>);
+  load((const void*)k_quant<128, 64, false>);
+  load((const void*)k_quant<128, 128, false>);
   load((const void*)k_mask<64, 1>);
   load((const void*)k_mask<64, 2>);
   load((const void*)k_mask<64, 4>);
@@ -729,6 +744,27 @@ int sla_quant(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q
   });
 }
 
+int sla_quant_gran(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q_scale, float* k_scale,
+                   float* k_mean, int B, int H, int N, int d, int block, int gran, void* stream) {
+  if (!q || !k || !q_i8 || !k_i8 || !q_scale || !k_scale) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  if ((rc = set_gran(&s, gran))) return rc;
+  s.kc = 1;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch sc;
+  if ((rc = sc.get(workspace_bytes(s, 0), st))) return rc;
+  Workspace w = carve(s, 0, static_cast<char*>(sc.ptr));
+  if (k_mean != nullptr) w.mu = k_mean;
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    return launch_stats_quant<D, BLK>(s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                      nullptr, nullptr, w, false, true, q_i8, k_i8, q_scale, k_scale, st);
+  });
+}
+
 int sla_mask(const void* q, const void* k, int32_t* blk_idx, uint8_t* bitmap, int B, int H, int N, int d,
              int block, float topk_frac, void* stream) {
   if (!q || !k || !blk_idx) return SLA_ERR_INVALID_ARG;
@@ -866,6 +902,35 @@ int sla_head_counts(int N, int block, int H, const float* topk_frac, const float
     if (kn) kn[h] = hc.kn[h];
   }
   return hc.kcp;
+}
+
+int sla_attn_gran(const void* q, const void* k, const void* v, const void* proj, void* out, int out_dtype,
+                  float* o_sparse, float* o_lin, int B, int H, int N, int d, int block, float topk_frac, int gran,
+                  void* stream) {
+  if (!q || !k || !v || !proj || !out) return SLA_ERR_INVALID_ARG;
+  if (out_dtype != SLA_OUT_BF16 && out_dtype != SLA_OUT_F32) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(proj) || !aligned16(out) ||
+      !aligned16(o_sparse) || !aligned16(o_lin))
+    return SLA_ERR_INVALID_ARG;
+  if (!frac_ok(topk_frac)) return SLA_ERR_INVALID_ARG;
+  Shape s;
+  int rc = check_shape(B, H, N, d, block, &s);
+  if (rc) return rc;
+  if ((rc = set_gran(&s, gran))) return rc;
+  s.kc = topk_count_ll(s.NB, topk_frac);
+  const bool linear = s.kc < s.NB;
+  const int what = 1 | 2 | 4 | (linear ? 8 : 0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch sc;
+  if ((rc = sc.get(workspace_bytes(s, what), st))) return rc;
+  Workspace w = carve(s, what, static_cast<char*>(sc.ptr));
+  return with_dims(d, block, [&](auto D_, auto B_) {
+    constexpr int D = decltype(D_)::value, BLK = decltype(B_)::value;
+    return run_attn<D, BLK>(s, uniform_counts(s.kc), linear, static_cast<const __nv_bfloat16*>(q),
+                            static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                            static_cast<const __nv_bfloat16*>(proj), out, out_dtype == SLA_OUT_F32, o_sparse, o_lin,
+                            w, st);
+  });
 }
 
 int sla_attn(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H, int N, int d,

@@ -60,6 +60,7 @@ class Workload:
     outliers: bool = False
     head_fracs: tuple | None = None   # one topk_frac per head (three-class mask), else topk_frac for all
     skip_frac: float | None = None    # fraction of blocks left out of the linear branch (three-class mask)
+    gran: int | None = None           # tokens per quantisation scale (None: one scale per block)
 
     @property
     def classes(self) -> bool:
@@ -78,6 +79,7 @@ class Workload:
         g = "x".join(map(str, self.grid)) if self.grid else "-"
         tf = ",".join(f"{f:g}" for f in self.head_fracs) if self.head_fracs else f"{self.topk_frac}"
         cls = f" skip_frac={self.skip_frac}" if self.skip_frac is not None else ""
+        cls += f" gran={self.gran}" if self.gran is not None else ""
         return (f"{self.name}: B={self.B} H={self.H} N={self.N} d={self.d} block={self.block} "
                 f"topk_frac={tf}{cls} dist={self.dist} grid={g} outliers={self.outliers} "
                 f"seed={self.seed}")
@@ -98,6 +100,8 @@ for _i, _f in enumerate(SWEEP_FRACS):
                                           4 + _i, (21, 30, 52), outliers=True)
 # the 480P shape with per-head fractions (5-20%, mean 12.5%) and the lower
 # half of every ranking left out of the linear branch (three-class mask)
+# the 480P workload with one quantisation scale per 32 tokens (finer granularity)
+CONFIGS["480p_gran32"] = Workload("480p_gran32", 1, 12, 32768, 128, 128, 0.10, "field", 1, (21, 30, 52), gran=32)
 CONFIGS["480p_classes"] = Workload("480p_classes", 1, 12, 32768, 128, 128, 0.125, "field", 8, (21, 30, 52),
                                    head_fracs=(0.05, 0.10, 0.15, 0.20) * 3, skip_frac=0.5)
 

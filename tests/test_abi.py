@@ -190,3 +190,18 @@ def test_binding_marshals_the_w8a8_entry_points(monkeypatch):
     assert [c[0] for c in calls] == ["sla_w8a8_quant", "sla_w8a8_linear", "sla_w8a8_gemm"]
     assert calls[1][1][5:9] == (S.OUT_F32, 300, 512, 256)
     assert calls[2][1][6:10] == (S.OUT_BF16, 300, 512, 256)
+
+
+def test_granularity_entry_points_refuse_invalid_arguments_without_a_gpu():
+    L = S.lib()
+    f = ctypes.c_float
+    dummy = 4096
+    for bad in (0, 16, 48, 256):
+        assert L.sla_attn_gran(dummy, dummy, dummy, dummy, dummy, 0, None, None, 1, 1, 128, 128, 128, f(0.1), bad,
+                               None) == 2
+        assert L.sla_quant_gran(dummy, dummy, dummy, dummy, dummy, dummy, None, 1, 1, 128, 128, 128, bad, None) == 2
+    # a group larger than the block
+    assert L.sla_attn_gran(dummy, dummy, dummy, dummy, dummy, 0, None, None, 1, 1, 128, 128, 64, f(0.1), 128,
+                           None) == 2
+    assert L.sla_attn_gran(dummy, dummy, dummy, dummy, dummy, 3, None, None, 1, 1, 128, 128, 64, f(0.1), 32,
+                           None) == 1

@@ -38,9 +38,9 @@ def S():
     return S
 
 
-def run_quant(S, x, block):
+def run_quant(S, x, block, gran=None):
     q, k = to_dev(x["q"]), to_dev(x["k"])
-    qi8, ki8, sq, sk, mu = S.sla_quant(q, k, block)
+    qi8, ki8, sq, sk, mu = S.sla_quant(q, k, block, gran=gran)
     assert S.get_error() == 0
     return {"q_i8": qi8.cpu().numpy(), "k_i8": ki8.cpu().numpy(), "q_scale": sq.cpu().numpy(),
             "k_scale": sk.cpu().numpy(), "mu": mu.cpu().numpy()}
@@ -53,7 +53,7 @@ def check_quant(got, ref):
         assert np.array_equal(got[key], ref[key]), (key, int(np.sum(got[key] != ref[key])))
 
 
-def run_attn(S, x, block, frac):
+def run_attn(S, x, block, frac, gran=None):
     """The operator through the C interface: float32 out with both parts
     (sla_attn_ex), the default bf16 out (sla_attn) and the block lists."""
     import torch
@@ -65,8 +65,8 @@ def run_attn(S, x, block, frac):
         return torch.full((B, H, N, d), float("nan"), dtype=torch.float32, device="cuda")
 
     out, osp, olin = f32(), f32(), f32()
-    S.sla_attn(q, k, v, w, block=block, topk_frac=frac, out=out, o_sparse=osp, o_lin=olin)
-    ob = S.sla_attn(q, k, v, w, block=block, topk_frac=frac)
+    S.sla_attn(q, k, v, w, block=block, topk_frac=frac, out=out, o_sparse=osp, o_lin=olin, gran=gran)
+    ob = S.sla_attn(q, k, v, w, block=block, topk_frac=frac, gran=gran)
     assert ob.dtype == torch.bfloat16
     idx = S.sla_mask(q, k, block, frac)
     assert S.get_error() == 0
@@ -74,7 +74,7 @@ def run_attn(S, x, block, frac):
     return {key: t.cpu().numpy().astype(np.float64) for key, t in got.items()}, idx.cpu().numpy()
 
 
-def check_attn(x, block, frac, items=None, case="?"):
+def check_attn(x, block, frac, items=None, case="?", gran=None):
     """Full comparison (items None) or on sampled query blocks.
 
     Returns (out stats, o_sparse stats, mask record).  The mask record counts
@@ -88,7 +88,7 @@ def check_attn(x, block, frac, items=None, case="?"):
     check_bf16)."""
     import int8_block_sparse_b200 as S
 
-    got, gidx = run_attn(S, x, block, frac)
+    got, gidx = run_attn(S, x, block, frac, gran)
     B, H, N, d = x["q"].shape
     ref_mask = O.block_mask(x["q"], x["k"], block, frac)
     diff, bad = mask_mismatch(gidx, ref_mask["idx"], ref_mask["near_tie"])
@@ -98,7 +98,7 @@ def check_attn(x, block, frac, items=None, case="?"):
     assert rec["near_tie_rows"] <= 0.01 * rec["rows"], rec
     override = {tuple(int(t) for t in ix): gidx[tuple(ix)] for ix in np.argwhere(diff)}
     res = O.sla_attention(x["q"], x["k"], x["v"], x["proj"], block, frac, items=items,
-                          idx_override=override or None)
+                          idx_override=override or None, gran=gran)
     w64 = O.bf16_to_f64(x["proj"])
     parts = {"out": [], "o_sparse": [], "o_lin": [], "out_bf16": []}
     refs = {"out": [], "o_sparse": [], "o_lin": []}
@@ -229,6 +229,43 @@ def test_repeated_calls_are_deterministic(S):
     assert torch.equal(a, b)
 
 
+# ---------------------------------------------------------------- finer quantisation groups
+
+GRAN_CASES = [
+    # (B, H, N, d, block, frac, gran, dist, seed)
+    (1, 2, 1000, 128, 128, 0.25, 32, "iid", 41),    # ragged tail: a partial group and one wholly past N
+    (1, 2, 777, 64, 128, 0.3, 32, "iid", 42),       # d = 64
+    (1, 2, 700, 128, 64, 0.2, 32, "iid", 43),       # 64-token blocks, two groups each
+    (1, 2, 2048, 128, 128, 0.2, 64, "field", 44),   # 64-token groups
+    (2, 2, 640, 128, 128, 1.0, 32, "iid", 45),      # every block kept
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,block,frac,gran,dist,seed", GRAN_CASES)
+def test_quant_and_attention_with_finer_groups(S, B, H, N, d, block, frac, gran, dist, seed):
+    grid = (4, 32, 32) if dist == "field" else None
+    x = make_inputs(B, H, N, d, seed, dist, grid)
+    check_quant(run_quant(S, x, block, gran), O.quantize(x["q"], x["k"], block, gran))
+    check_attn(x, block, frac, case=f"gran{gran}-{seed}", gran=gran)
+
+
+def test_finer_groups_lossless_inputs(S):
+    """Rows scaled by a different power of two per 32 tokens: with 32-token
+    groups the GPU codes are the integers and its output matches the oracle's."""
+    from synth.workloads import f32_to_bf16_bits
+
+    rng = np.random.default_rng(46)
+    N, d, block, gran = 512, 128, 128, 32
+    qi = rng.integers(-127, 128, size=(1, 1, N, d)).astype(np.float32)
+    ki = rng.integers(-127, 128, size=(1, 1, N, d)).astype(np.float32)
+    pw = np.repeat(2.0 ** -(4 + np.arange(N // gran) % 6), gran).astype(np.float32)
+    x = {"q": f32_to_bf16_bits(qi * pw[None, None, :, None]), "k": f32_to_bf16_bits(ki * pw[None, None, :, None]),
+         "v": f32_to_bf16_bits(rng.standard_normal((1, 1, N, d)).astype(np.float32)),
+         "proj": f32_to_bf16_bits((rng.standard_normal((d, d)) / np.sqrt(d)).astype(np.float32))}
+    check_quant(run_quant(S, x, block, gran), O.quantize(x["q"], x["k"], block, gran))
+    check_attn(x, block, 0.5, case="gran32-lossless", gran=gran)
+
+
 # ---------------------------------------------------------------- three classes, per-head fractions
 
 def run_attn_classes(S, x, block, fr, sk):
@@ -351,12 +388,12 @@ def test_classes_with_uniform_fractions_equal_the_two_class_operator(S):
 def _full_case(S, name, per_head):
     w = CONFIGS[name]
     x = make_workload(w)
-    check_quant(run_quant(S, x, w.block), O.quantize(x["q"], x["k"], w.block))
+    check_quant(run_quant(S, x, w.block, w.gran), O.quantize(x["q"], x["k"], w.block, w.gran))
     items = sample_items(w.B, w.H, w.nblk, per_head=per_head, seed=w.seed)
     if w.classes:
         st, st_sp, rec = check_attn_classes(x, w.block, w.fracs, w.skip_frac, items=items, case=name)
     else:
-        st, st_sp, rec = check_attn(x, w.block, w.topk_frac, items=items, case=name)
+        st, st_sp, rec = check_attn(x, w.block, w.topk_frac, items=items, case=name, gran=w.gran)
     print(json.dumps({"case": name, "out": st, "o_sparse": st_sp}))
 
 
@@ -383,6 +420,10 @@ def test_full_720p(S):
 
 def test_full_480p_classes(S):
     _full_case(S, "480p_classes", per_head=4)
+
+
+def test_full_480p_gran32(S):
+    _full_case(S, "480p_gran32", per_head=4)
 
 
 def _wide_exponent_inputs(N, d, seed):
