@@ -17,7 +17,8 @@
 // the maximum, pass 2 the codes.
 //
 // k_w8a8_gemm: persistent, one CTA per SM, output tiles of 128 rows x 256
-// columns.  Per k-block one tcgen05.mma kind::i8 product (M 128, N 256, K
+// columns (the width is a template parameter; 128 and 192 were slower: more
+// operand traffic per product, or register spills).  Per k-block one tcgen05.mma kind::i8 product (M 128, N 256, K
 // 128 as four K=32 instructions) goes into one of two 256-column TMEM buffers;
 // the promotion warps read it, scale it and add it into float32 accumulators
 // in registers while the tensor core fills the other buffer.  The int32 sums
@@ -118,33 +119,32 @@ struct W8A8Params {
   const __nv_bfloat16* bias;       // [N] or nullptr
   void* y;                         // [M][N] bf16 or float32
   int M, N, K, KB;                 // KB = ceil(K / 128) k-blocks
-  int tiles_n, tiles;              // tiles of 128 x 256
+  int tiles_n, tiles;              // tiles of 128 x BN
   int out_f32;
 };
 
-constexpr int WG_STAGES = 4;
-constexpr int WG_A_BYTES = 128 * 128;               // X tile: 128 rows x 128 k (int8)
-constexpr int WG_B_BYTES = 256 * 128;               // W tile: 256 rows x 128 k
-constexpr int WG_STAGE_BYTES = WG_A_BYTES + WG_B_BYTES;
-constexpr int WG_BAR_BYTES = (2 * WG_STAGES + 4 + 1) * 8 + 16;
-constexpr int WG_SMEM_USED = WG_STAGES * WG_STAGE_BYTES + WG_BAR_BYTES;
-constexpr int WG_SMEM = WG_SMEM_USED + 1024;
 constexpr uint32_t kMagicBits = 0x4B400000u;        // 1.5 * 2^23
+constexpr int kW8TileN = 256;                        // output tile width BN
 
-constexpr int kW8PromotionWarps = 8;
-
-// PW promotion warps (8 or 16): each owns 32 TMEM lanes and 256 / (PW / 4)
-// columns of the tile; the threads' registers at launch and the split.
-template <int PW>
+// BN-column tiles: TMEM buffers of BN columns, 8 promotion warps of BN / 2
+// columns each (32 TMEM lanes x BN / 2 columns), threads and register split.
+template <int BN>
 struct W8Cfg {
-  static constexpr int THREADS = 128 + 32 * PW;
-  static constexpr int COLS = 256 / (PW / 4);        // columns per promotion warp
-  static constexpr int CW = PW == 8 ? 32 : 16;       // columns per TMEM load
-  static constexpr int LAUNCH_REGS = PW == 8 ? 168 : 96;
-  static constexpr int REGS_LOAD = PW == 8 ? 40 : 32;
-  static constexpr int REGS_MATH = PW == 8 ? 232 : 112;
-  static_assert(128 * REGS_LOAD + 32 * PW * REGS_MATH <= THREADS * LAUNCH_REGS, "register split within the launch's");
-  static_assert(THREADS * LAUNCH_REGS <= 65536, "registers at launch");
+  static constexpr int STAGES = BN == 256 ? 4 : 5;
+  static constexpr int A_BYTES = 128 * 128;          // X tile: 128 rows x 128 k (int8)
+  static constexpr int B_BYTES = BN * 128;           // W tile: BN rows x 128 k
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_BYTES = (2 * STAGES + 4 + 1) * 8 + 16;
+  static constexpr int SMEM_USED = STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SMEM = SMEM_USED + 1024;
+  static constexpr int THREADS = 384;                // warpgroup 0: producer, MMA; 1-2: promotion
+  static constexpr int COLS = BN / 2;                // columns per promotion warp
+  static constexpr int NCH = COLS / 32;              // 32-column TMEM loads per k-block
+  static constexpr int REGS_LOAD = 40;
+  static constexpr int REGS_MATH = 232;
+  static_assert(128 * REGS_LOAD + 256 * REGS_MATH <= THREADS * 168, "register split within the launch's");
+  static_assert(BN % 64 == 0 && BN <= 256, "two 32-column-aligned halves");
+  static_assert(SMEM <= 232448, "stages fit in shared memory");
 };
 
 // The same 32-bit value into 32 consecutive TMEM columns of the warp's 32 lanes.
@@ -156,47 +156,36 @@ __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t x) {
       : "memory");
 }
 
-// CW consecutive TMEM columns of the warp's 32 lanes into registers.
-template <int CW>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
-  if constexpr (CW == 32) {
-    SLA_TMEM_LD32(taddr, r);
-  } else {
-    static_assert(CW == 16, "16 or 32 columns");
-    SLA_TMEM_LD16(taddr, r);
-  }
-}
-
-template <int PW>
-__global__ void __launch_bounds__(W8Cfg<PW>::THREADS, 1) k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_a,
+template <int BN>
+__global__ void __launch_bounds__(W8Cfg<BN>::THREADS, 1) k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_a,
                                                                      const __grid_constant__ CUtensorMap tm_b,
                                                                      const W8A8Params p) {
-  using C = W8Cfg<PW>;
+  using C = W8Cfg<BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if (uint32_t(base - smem_raw) + WG_SMEM_USED > dynamic_smem_bytes()) {
+  if (uint32_t(base - smem_raw) + C::SMEM_USED > dynamic_smem_bytes()) {
     if (threadIdx.x == 0) raise_error(DEV_ERR_LAYOUT);
     return;   // uniform: every thread sees the same base
   }
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + WG_STAGES * WG_STAGE_BYTES);
-  uint64_t* empty = full + WG_STAGES;
-  uint64_t* t_full = empty + WG_STAGES;     // [2] a k-block's product is in TMEM buffer b
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* t_full = empty + C::STAGES;     // [2] a k-block's product is in TMEM buffer b
   uint64_t* t_empty = t_full + 2;           // [2] buffer b was read and re-armed with the magic bits
   uint64_t* drain = t_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  auto stage = [&](int s) { return base + s * WG_STAGE_BYTES; };
+  auto stage = [&](int s) { return base + s * C::STAGE_BYTES; };
 
   if (tid == 0) {
-    for (int q = 0; q < WG_STAGES; ++q) {
+    for (int q = 0; q < C::STAGES; ++q) {
       mbar_init(&full[q], 1);
       mbar_init(&empty[q], 1);
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&t_full[q], 1);
-      mbar_init(&t_empty[q], 32 * PW);
+      mbar_init(&t_empty[q], 256);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -222,37 +211,37 @@ __global__ void __launch_bounds__(W8Cfg<PW>::THREADS, 1) k_w8a8_gemm(const __gri
         uint32_t n = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-          const int m0 = (t / p.tiles_n) * 128, n0 = (t % p.tiles_n) * 256;
+          const int m0 = (t / p.tiles_n) * 128, n0 = (t % p.tiles_n) * BN;
           for (int kb = 0; kb < p.KB; ++kb, ++n) {
-            const int s = n % WG_STAGES;
-            if (!(ok = mbar_wait(&empty[s], ((n / WG_STAGES) & 1) ^ 1, abort_flag))) break;
-            mbar_expect_tx(&full[s], WG_STAGE_BYTES);
+            const int s = n % C::STAGES;
+            if (!(ok = mbar_wait(&empty[s], ((n / C::STAGES) & 1) ^ 1, abort_flag))) break;
+            mbar_expect_tx(&full[s], C::STAGE_BYTES);
             tma_load_2d(stage(s), &tm_a, &full[s], kb * 128, m0);
-            tma_load_2d(stage(s) + WG_A_BYTES, &tm_b, &full[s], kb * 128, n0);
+            tma_load_2d(stage(s) + C::A_BYTES, &tm_b, &full[s], kb * 128, n0);
           }
         }
         // loads still in flight (only after a failed wait) land before the CTA exits
-        for (uint32_t q = n > WG_STAGES ? n - WG_STAGES : 0; q < n; ++q)
-          (void)mbar_wait(&full[q % WG_STAGES], (q / WG_STAGES) & 1, nullptr);
+        for (uint32_t q = n > C::STAGES ? n - C::STAGES : 0; q < n; ++q)
+          (void)mbar_wait(&full[q % C::STAGES], (q / C::STAGES) & 1, nullptr);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
-        const uint32_t idesc = idesc_i8(256);
+        const uint32_t idesc = idesc_i8(BN);
         uint32_t n = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
           for (int kb = 0; kb < p.KB; ++kb, ++n) {
-            const int s = n % WG_STAGES;
+            const int s = n % C::STAGES;
             const uint32_t b = n & 1;
             if (!(ok = mbar_wait(&t_empty[b], (n >> 1) & 1, abort_flag))) break;
-            if (!(ok = mbar_wait(&full[s], (n / WG_STAGES) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&full[s], (n / C::STAGES) & 1, abort_flag))) break;
             tc_fence_after();
             const uint64_t da = smem_desc(smem_u32(stage(s)), 16, 1024, 2);
-            const uint64_t db = smem_desc(smem_u32(stage(s) + WG_A_BYTES), 16, 1024, 2);
+            const uint64_t db = smem_desc(smem_u32(stage(s) + C::A_BYTES), 16, 1024, 2);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)   // accumulate onto the magic bits
-              mma_i8_ss(tmem + b * 256, da + uint64_t(kk * 2), db + uint64_t(kk * 2), idesc, 1u);
+              mma_i8_ss(tmem + b * BN, da + uint64_t(kk * 2), db + uint64_t(kk * 2), idesc, 1u);
             tc_commit(&empty[s]);
             tc_commit(&t_full[b]);
           }
@@ -266,17 +255,14 @@ __global__ void __launch_bounds__(W8Cfg<PW>::THREADS, 1) k_w8a8_gemm(const __gri
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_MATH));
     // ------------------------------------------------------------ promotion + epilogue
     const int q4 = warp & 3;                       // TMEM lane quarter
-    const int g = (warp - 4) >> 2;                 // column group of the tile
-    const int cbase = g * C::COLS;                 // first tile column of the group
-    const int h = cbase >> 7;                      // its 128-column block (scale row of W)
+    const int cbase = ((warp - 4) >> 2) * C::COLS; // first tile column of the warp
     const int r = q4 * 32 + lane;                  // tile row
     const uint32_t lane_off = uint32_t(q4 * 32) << 16;
-    constexpr int NCH = C::COLS / C::CW;           // TMEM loads per k-block
     // arm both buffers
 #pragma unroll
     for (int b = 0; b < 2; ++b)
 #pragma unroll
-      for (int c = 0; c < C::COLS; c += 32) tmem_fill32(tmem + lane_off + b * 256 + cbase + c, kMagicBits);
+      for (int c = 0; c < C::NCH; ++c) tmem_fill32(tmem + lane_off + b * BN + cbase + c * 32, kMagicBits);
     tmem_st_wait();
     tc_fence_before();
     mbar_arrive(&t_empty[0]);
@@ -285,50 +271,59 @@ __global__ void __launch_bounds__(W8Cfg<PW>::THREADS, 1) k_w8a8_gemm(const __gri
     uint32_t n = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-      const int m0 = (t / p.tiles_n) * 128, n0 = (t % p.tiles_n) * 256;
-      const int mb = m0 >> 7, nb = (n0 >> 7) + h;
-      const bool nb_ok = n0 + cbase < p.N;
-      const float* sxr = p.sx + (long long)mb * p.KB;
-      const float* swr = p.sw + (long long)(nb_ok ? nb : 0) * p.KB;
+      const int m0 = (t / p.tiles_n) * 128, n0 = (t % p.tiles_n) * BN;
+      const float* sxr = p.sx + (long long)(m0 >> 7) * p.KB;
+      // W scale rows of the warp's columns: the first chunk's block and, when
+      // the warp's columns cross into the next 128-column block, that one (a
+      // 32-column chunk never crosses a block boundary)
+      const int col0 = n0 + cbase;
+      const int split = ((col0 >> 7) + 1) * 128 - col0;   // columns in the first block
+      const float* swa = p.sw + (long long)(col0 < p.N ? col0 >> 7 : 0) * p.KB;
+      const float* swb = p.sw + (long long)(col0 + split < p.N ? (col0 >> 7) + 1 : 0) * p.KB;
       float acc[C::COLS];
 #pragma unroll
       for (int e = 0; e < C::COLS; ++e) acc[e] = 0.f;
-      float sxn = __ldg(sxr), swn = __ldg(swr);
+      float sxn = __ldg(sxr), swan = __ldg(swa), swbn = __ldg(swb);
       for (int kb = 0; kb < p.KB; ++kb, ++n) {
-        const float sc = sxn * swn;                 // one float32 rounding of the scale product
+        // one float32 rounding of each scale product
+        const float sca = sxn * swan, scb = sxn * swbn;
         if (kb + 1 < p.KB) {
           sxn = __ldg(sxr + kb + 1);
-          swn = __ldg(swr + kb + 1);
+          swan = __ldg(swa + kb + 1);
+          swbn = __ldg(swb + kb + 1);
         }
         const uint32_t b = n & 1;
         if (!(ok = mbar_wait(&t_full[b], (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint32_t tb = tmem + lane_off + b * 256 + cbase;
-        // chunk c + 1 is read from TMEM while chunk c is added up
-        uint32_t v[2][C::CW];
-        tmem_ld_cols<C::CW>(tb, v[0]);
+        const uint32_t tb = tmem + lane_off + b * BN + cbase;
+        // P of a pair exactly by one packed subtraction (the packed forms run on
+        // one half of the FMA pipe), then two scalar fused multiply-adds (either half)
+        auto add_chunk = [&](const uint32_t* w, int c) {
+          const float scc = c * 32 < split ? sca : scb;
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          tmem_ld_wait();                            // chunk c has landed
-          if (c + 1 < NCH) tmem_ld_cols<C::CW>(tb + (c + 1) * C::CW, v[(c + 1) & 1]);
-          if ((c * C::CW) % 32 + C::CW == 32)        // re-arm the 32 columns just read (the k-block after next)
-            tmem_fill32(tb + (c * C::CW / 32) * 32, kMagicBits);
-          if (c == NCH - 1) {                        // every column read and re-armed: release the buffer
+          for (int e = 0; e < 32; e += 2) {
+            float p0, p1;
+            f32x2_split(add_f32x2(f32x2(__uint_as_float(w[e]), __uint_as_float(w[e + 1])), negc2), p0, p1);
+            acc[c * 32 + e] = fmaf(p0, scc, acc[c * 32 + e]);
+            acc[c * 32 + e + 1] = fmaf(p1, scc, acc[c * 32 + e + 1]);
+          }
+        };
+        // chunk c + 1 is read from TMEM while chunk c is added up; each chunk
+        // is re-armed once read, and the buffer released before the last
+        // chunk's arithmetic
+        uint32_t v[2][32];
+        SLA_TMEM_LD32(tb, v[0]);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          tmem_ld_wait();
+          if (c + 1 < C::NCH) SLA_TMEM_LD32(tb + (c + 1) * 32, v[(c + 1) & 1]);
+          tmem_fill32(tb + c * 32, kMagicBits);
+          if (c == C::NCH - 1) {
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&t_empty[b]);
           }
-          const uint32_t* w = v[c & 1];
-#pragma unroll
-          for (int e = 0; e < C::CW; e += 2) {
-            // P of a pair exactly by one packed subtraction (the packed forms
-            // run on one half of the FMA pipe), then two scalar fused
-            // multiply-adds (either half)
-            float p0, p1;
-            f32x2_split(add_f32x2(f32x2(__uint_as_float(w[e]), __uint_as_float(w[e + 1])), negc2), p0, p1);
-            acc[c * C::CW + e] = fmaf(p0, sc, acc[c * C::CW + e]);
-            acc[c * C::CW + e + 1] = fmaf(p1, sc, acc[c * C::CW + e + 1]);
-          }
+          add_chunk(v[c & 1], c);
         }
       }
       if (!ok) break;

@@ -639,6 +639,8 @@ int launch_quant2d(const void* x, int R, int K, int8_t* codes, float* scales, cu
 
 int launch_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias, void* y,
                      bool out_f32, int M, int N, int K, cudaStream_t st) {
+  constexpr int BN = kW8TileN;
+  using C = W8Cfg<BN>;
   CUtensorMap ma, mb;
   {
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
@@ -650,23 +652,22 @@ int launch_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const 
   {
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)N};
     cuuint64_t str[1] = {(cuuint64_t)K};
-    cuuint32_t box[2] = {128u, 256u};
+    cuuint32_t box[2] = {128u, (cuuint32_t)BN};
     if (!make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, wq, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return SLA_ERR_CUDA;
   }
   W8A8Params p;
   p.sx = sx; p.sw = sw; p.bias = static_cast<const __nv_bfloat16*>(bias); p.y = y;
   p.M = M; p.N = N; p.K = K; p.KB = (K + 127) / 128;
-  p.tiles_n = (N + 255) / 256;
+  p.tiles_n = (N + BN - 1) / BN;
   const long long tiles = (long long)((M + 127) / 128) * p.tiles_n;
   if (tiles >= (1LL << 31)) return SLA_ERR_UNSUPPORTED;
   p.tiles = (int)tiles;
   p.out_f32 = out_f32 ? 1 : 0;
-  constexpr int PW = kW8PromotionWarps;
-  cudaFuncSetAttribute(k_w8a8_gemm<PW>, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+  cudaFuncSetAttribute(k_w8a8_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int ctas = (int)std::min<long long>(num_sms(), tiles);
   ProfScope ps(SLA_K_W8A8, st);
-  k_w8a8_gemm<PW><<<ctas, W8Cfg<PW>::THREADS, WG_SMEM, st>>>(ma, mb, p);
+  k_w8a8_gemm<BN><<<ctas, C::THREADS, C::SMEM, st>>>(ma, mb, p);
   return cuda_status(cudaGetLastError());
 }
 
