@@ -219,6 +219,31 @@ def test_host_buffers_match_device_path(S):
     assert torch.equal(out_host, out_dev.cpu())
 
 
+def test_call_captured_in_a_cuda_graph_matches_eager(S):
+    """The operator's two-stream sequence can be captured in a CUDA graph (the
+    second stream joins the capture through its events) and replayed."""
+    import torch
+
+    x = make_inputs(1, 2, 1500, 128, 7)
+    dev = [to_dev(x[t]) for t in ("q", "k", "v", "proj")]
+    eager = S.sla_attn(*dev, block=128, topk_frac=0.2)
+    out = torch.empty_like(eager)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):            # warm-up outside the capture
+        S.sla_attn(*dev, block=128, topk_frac=0.2, out=out, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        S.sla_attn(*dev, block=128, topk_frac=0.2, out=out)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert S.get_error() == 0
+    assert torch.equal(out, eager)
+
+
 def test_repeated_calls_are_deterministic(S):
     import torch
 
