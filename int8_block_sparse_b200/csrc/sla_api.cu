@@ -443,11 +443,22 @@ int launch_lingemm(const Shape& s, Workspace& w, cudaStream_t st) {
   gp.nkt = (int)((s.NB + 63) / 64);
   gp.mgroups = (int)((s.NB + 255) / 256);
   gp.ntiles = (gp.E + 127) / 128;
-  gp.units = (int)(s.BH * gp.mgroups * gp.ntiles);
-  cudaFuncSetAttribute(k_lingemm, cudaFuncAttributeMaxDynamicSharedMemorySize, LG_SMEM);
+  const bool resident = gp.nkt <= LG_MAX_RESIDENT_KT;
+  const long long groups = s.BH * gp.mgroups;
+  // resident A: the N tiles of a (head, M group) split into runs so that the
+  // units number at most one per SM; otherwise one N tile per unit
+  const long long runs = resident ? std::max<long long>(1, num_sms() / groups) : gp.ntiles;
+  gp.tpu = (int)((gp.ntiles + runs - 1) / runs);
+  gp.units = (int)(groups * ((gp.ntiles + gp.tpu - 1) / gp.tpu));
   const int ctas = std::min(num_sms(), gp.units);
   ProfScope ps(SLA_K_LINGEMM, st);
-  k_lingemm<<<ctas, LG_THREADS, LG_SMEM, st>>>(ma, mb, gp);
+  if (resident) {
+    cudaFuncSetAttribute(k_lingemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinGemmCfg<true>::SMEM);
+    k_lingemm<true><<<ctas, LG_THREADS, LinGemmCfg<true>::SMEM, st>>>(ma, mb, gp);
+  } else {
+    cudaFuncSetAttribute(k_lingemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, LinGemmCfg<false>::SMEM);
+    k_lingemm<false><<<ctas, LG_THREADS, LinGemmCfg<false>::SMEM, st>>>(ma, mb, gp);
+  }
   return cuda_status(cudaGetLastError());
 }
 
