@@ -125,29 +125,32 @@ struct W8A8Params {
 
 constexpr uint32_t kMagicBits = 0x4B400000u;        // 1.5 * 2^23
 constexpr int kW8TileN = 256;                        // output tile width BN
+constexpr int kW8Buffers = 2;                        // TMEM buffers (k-blocks in flight)
 
-// BN-column tiles: TMEM buffers of BN columns, 8 promotion warps of BN / 2
-// columns each (32 TMEM lanes x BN / 2 columns), threads and register split.
-template <int BN>
+// BN-column tiles, NBUF TMEM buffers of BN columns, 8 promotion warps of
+// BN / 2 columns each (32 TMEM lanes x BN / 2 columns) read CW columns at a
+// time; threads and register split.
+template <int BN, int NBUF>
 struct W8Cfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 5;
+  static constexpr int STAGES = BN >= 256 ? 4 : 5;
   static constexpr int A_BYTES = 128 * 128;          // X tile: 128 rows x 128 k (int8)
   static constexpr int B_BYTES = BN * 128;           // W tile: BN rows x 128 k
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BAR_BYTES = (2 * STAGES + 4 + 1) * 8 + 16;
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF + 1) * 8 + 16;
   static constexpr int SMEM_USED = STAGES * STAGE_BYTES + BAR_BYTES;
   static constexpr int SMEM = SMEM_USED + 1024;
   static constexpr int THREADS = 384;                // warpgroup 0: producer, MMA; 1-2: promotion
   static constexpr int COLS = BN / 2;                // columns per promotion warp
-  static constexpr int NCH = COLS / 32;              // 32-column TMEM loads per k-block
+  static constexpr int CW = COLS % 32 == 0 ? 32 : 16; // columns per TMEM load
+  static constexpr int NCH = COLS / CW;              // TMEM loads per k-block
   static constexpr int REGS_LOAD = 40;
   static constexpr int REGS_MATH = 232;
   static_assert(128 * REGS_LOAD + 256 * REGS_MATH <= THREADS * 168, "register split within the launch's");
-  static_assert(BN % 64 == 0 && BN <= 256, "two 32-column-aligned halves");
+  static_assert(BN % 32 == 0 && BN <= 256 && NBUF * BN <= 512, "tile halves of whole chunks; buffers fit TMEM");
   static_assert(SMEM <= 232448, "stages fit in shared memory");
 };
 
-// The same 32-bit value into 32 consecutive TMEM columns of the warp's 32 lanes.
+// The same 32-bit value into 32 (16) consecutive TMEM columns of the warp's 32 lanes.
 __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t x) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
@@ -155,12 +158,32 @@ __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t x) {
       "r"(x)
       : "memory");
 }
+__device__ __forceinline__ void tmem_fill16(uint32_t taddr, uint32_t x) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(
+                   taddr),
+               "r"(x)
+               : "memory");
+}
+template <int CW>
+__device__ __forceinline__ void tmem_fill_cols(uint32_t taddr, uint32_t x) {
+  if constexpr (CW == 32) tmem_fill32(taddr, x);
+  else tmem_fill16(taddr, x);
+}
+template <int CW>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
+  if constexpr (CW == 32) {
+    SLA_TMEM_LD32(taddr, r);
+  } else {
+    SLA_TMEM_LD16(taddr, r);
+  }
+}
 
-template <int BN>
-__global__ void __launch_bounds__(W8Cfg<BN>::THREADS, 1) k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_a,
-                                                                     const __grid_constant__ CUtensorMap tm_b,
-                                                                     const W8A8Params p) {
-  using C = W8Cfg<BN>;
+template <int BN, int NBUF>
+__global__ void __launch_bounds__(W8Cfg<BN, NBUF>::THREADS, 1) k_w8a8_gemm(const __grid_constant__ CUtensorMap tm_a,
+                                                                           const __grid_constant__ CUtensorMap tm_b,
+                                                                           const W8A8Params p) {
+  using C = W8Cfg<BN, NBUF>;
+  constexpr int CW = C::CW;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,9 +193,9 @@ __global__ void __launch_bounds__(W8Cfg<BN>::THREADS, 1) k_w8a8_gemm(const __gri
   }
   uint64_t* full = reinterpret_cast<uint64_t*>(base + C::STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* t_full = empty + C::STAGES;     // [2] a k-block's product is in TMEM buffer b
-  uint64_t* t_empty = t_full + 2;           // [2] buffer b was read and re-armed with the magic bits
-  uint64_t* drain = t_empty + 2;
+  uint64_t* t_full = empty + C::STAGES;     // [NBUF] a k-block's product is in TMEM buffer b
+  uint64_t* t_empty = t_full + NBUF;        // [NBUF] buffer b was read and re-armed with the magic bits
+  uint64_t* drain = t_empty + NBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -183,7 +206,7 @@ __global__ void __launch_bounds__(W8Cfg<BN>::THREADS, 1) k_w8a8_gemm(const __gri
       mbar_init(&full[q], 1);
       mbar_init(&empty[q], 1);
     }
-    for (int q = 0; q < 2; ++q) {
+    for (int q = 0; q < NBUF; ++q) {
       mbar_init(&t_full[q], 1);
       mbar_init(&t_empty[q], 256);
     }
@@ -233,8 +256,8 @@ __global__ void __launch_bounds__(W8Cfg<BN>::THREADS, 1) k_w8a8_gemm(const __gri
         for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
           for (int kb = 0; kb < p.KB; ++kb, ++n) {
             const int s = n % C::STAGES;
-            const uint32_t b = n & 1;
-            if (!(ok = mbar_wait(&t_empty[b], (n >> 1) & 1, abort_flag))) break;
+            const uint32_t b = n % NBUF;
+            if (!(ok = mbar_wait(&t_empty[b], (n / NBUF) & 1, abort_flag))) break;
             if (!(ok = mbar_wait(&full[s], (n / C::STAGES) & 1, abort_flag))) break;
             tc_fence_after();
             const uint64_t da = smem_desc(smem_u32(stage(s)), 16, 1024, 2);
@@ -258,15 +281,15 @@ __global__ void __launch_bounds__(W8Cfg<BN>::THREADS, 1) k_w8a8_gemm(const __gri
     const int cbase = ((warp - 4) >> 2) * C::COLS; // first tile column of the warp
     const int r = q4 * 32 + lane;                  // tile row
     const uint32_t lane_off = uint32_t(q4 * 32) << 16;
-    // arm both buffers
+    // arm every buffer
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < NBUF; ++b)
 #pragma unroll
-      for (int c = 0; c < C::NCH; ++c) tmem_fill32(tmem + lane_off + b * BN + cbase + c * 32, kMagicBits);
+      for (int c = 0; c < C::NCH; ++c) tmem_fill_cols<CW>(tmem + lane_off + b * BN + cbase + c * CW, kMagicBits);
     tmem_st_wait();
     tc_fence_before();
-    mbar_arrive(&t_empty[0]);
-    mbar_arrive(&t_empty[1]);
+#pragma unroll
+    for (int b = 0; b < NBUF; ++b) mbar_arrive(&t_empty[b]);
     const uint64_t negc2 = f32x2(-12582912.f, -12582912.f);
     uint32_t n = 0;
     bool ok = true;
@@ -292,32 +315,32 @@ __global__ void __launch_bounds__(W8Cfg<BN>::THREADS, 1) k_w8a8_gemm(const __gri
           swan = __ldg(swa + kb + 1);
           swbn = __ldg(swb + kb + 1);
         }
-        const uint32_t b = n & 1;
-        if (!(ok = mbar_wait(&t_full[b], (n >> 1) & 1, abort_flag))) break;
+        const uint32_t b = n % NBUF;
+        if (!(ok = mbar_wait(&t_full[b], (n / NBUF) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t tb = tmem + lane_off + b * BN + cbase;
         // P of a pair exactly by one packed subtraction (the packed forms run on
         // one half of the FMA pipe), then two scalar fused multiply-adds (either half)
         auto add_chunk = [&](const uint32_t* w, int c) {
-          const float scc = c * 32 < split ? sca : scb;
+          const float scc = c * CW < split ? sca : scb;
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+          for (int e = 0; e < CW; e += 2) {
             float p0, p1;
             f32x2_split(add_f32x2(f32x2(__uint_as_float(w[e]), __uint_as_float(w[e + 1])), negc2), p0, p1);
-            acc[c * 32 + e] = fmaf(p0, scc, acc[c * 32 + e]);
-            acc[c * 32 + e + 1] = fmaf(p1, scc, acc[c * 32 + e + 1]);
+            acc[c * CW + e] = fmaf(p0, scc, acc[c * CW + e]);
+            acc[c * CW + e + 1] = fmaf(p1, scc, acc[c * CW + e + 1]);
           }
         };
         // chunk c + 1 is read from TMEM while chunk c is added up; each chunk
         // is re-armed once read, and the buffer released before the last
         // chunk's arithmetic
-        uint32_t v[2][32];
-        SLA_TMEM_LD32(tb, v[0]);
+        uint32_t v[2][CW];
+        tmem_ld_cols<CW>(tb, v[0]);
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           tmem_ld_wait();
-          if (c + 1 < C::NCH) SLA_TMEM_LD32(tb + (c + 1) * 32, v[(c + 1) & 1]);
-          tmem_fill32(tb + c * 32, kMagicBits);
+          if (c + 1 < C::NCH) tmem_ld_cols<CW>(tb + (c + 1) * CW, v[(c + 1) & 1]);
+          tmem_fill_cols<CW>(tb + c * CW, kMagicBits);
           if (c == C::NCH - 1) {
             tmem_st_wait();
             tc_fence_before();

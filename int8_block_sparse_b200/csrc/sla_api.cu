@@ -650,8 +650,8 @@ int launch_quant2d(const void* x, int R, int K, int8_t* codes, float* scales, cu
 
 int launch_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, const void* bias, void* y,
                      bool out_f32, int M, int N, int K, cudaStream_t st) {
-  constexpr int BN = kW8TileN;
-  using C = W8Cfg<BN>;
+  constexpr int BN = kW8TileN, NBUF = kW8Buffers;
+  using C = W8Cfg<BN, NBUF>;
   CUtensorMap ma, mb;
   {
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
@@ -675,10 +675,10 @@ int launch_w8a8_gemm(const int8_t* xq, const float* sx, const int8_t* wq, const 
   if (tiles >= (1LL << 31)) return SLA_ERR_UNSUPPORTED;
   p.tiles = (int)tiles;
   p.out_f32 = out_f32 ? 1 : 0;
-  cudaFuncSetAttribute(k_w8a8_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaFuncSetAttribute(k_w8a8_gemm<BN, NBUF>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int ctas = (int)std::min<long long>(num_sms(), tiles);
   ProfScope ps(SLA_K_W8A8, st);
-  k_w8a8_gemm<BN><<<ctas, C::THREADS, C::SMEM, st>>>(ma, mb, p);
+  k_w8a8_gemm<BN, NBUF><<<ctas, C::THREADS, C::SMEM, st>>>(ma, mb, p);
   return cuda_status(cudaGetLastError());
 }
 
