@@ -223,8 +223,9 @@ int sla_attn_classes(const void* q, const void* k, const void* v, const void* pr
  * result is in host memory.  The (batch, head) pairs are processed in up to
  * six chunks spread over three streams of the current device (created at the
  * first call on that device and kept), so that with pinned host buffers one
- * chunk's copies overlap another chunk's operator; the result is the same as
- * sla_attn's.  Calls on the same device are serialised. */
+ * chunk's copies overlap another chunk's operator (each chunk's kernels stay
+ * on that chunk's stream); the result is the same as sla_attn's.  Calls on
+ * the same device are serialised. */
 int sla_attn_host(const void* q, const void* k, const void* v, const void* proj, void* out, int B, int H,
                   int N, int d, int block, float topk_frac);
 

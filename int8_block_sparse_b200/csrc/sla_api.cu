@@ -462,6 +462,10 @@ int launch_lingemm(const Shape& s, Workspace& w, cudaStream_t st) {
   return cuda_status(cudaGetLastError());
 }
 
+// Set by the host-buffer path around its calls: run the operator's kernels
+// on the caller's stream only.
+thread_local bool t_one_stream = false;
+
 // ------------------------------------------------------------------ second stream of the operator
 // The operator's kernels run on two streams of the device: the caller's and
 // this one (created at the first call on a device and kept).  Its events
@@ -505,10 +509,16 @@ int run_attn(const Shape& s, const HeadCounts& hc, bool linear, const __nv_bfloa
              const __nv_bfloat16* v, const __nv_bfloat16* proj, void* out, bool out_f32, float* o_sparse,
              float* o_lin, Workspace& w, cudaStream_t st) {
   int* kc_bh = hc.H > 1 || hc.kc[0] != s.kc ? w.kc_bh : nullptr;   // per-head list lengths
-  SideStream* ss = side_stream();
-  if (ss == nullptr) return SLA_ERR_CUDA;
   int rc = SLA_OK;
-  {
+  if (t_one_stream) {
+    // everything in order on the caller's stream (the host-buffer path
+    // overlaps whole chunks of heads on its own streams instead)
+    rc = launch_stats_quant<D, BLK>(s, q, k, v, proj, w, linear, true, w.qi8, w.ki8, w.sq, w.sk, st);
+    if (rc == SLA_OK) rc = launch_mask<D>(s, w, hc, kc_bh, w.idx, nullptr, linear ? w.notcrit : nullptr, st);
+    if (rc == SLA_OK && linear) rc = launch_lingemm<D>(s, w, st);
+  } else {
+    SideStream* ss = side_stream();
+    if (ss == nullptr) return SLA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(ss->mu);
     if (cudaEventRecord(ss->fork, st) != cudaSuccess || cudaStreamWaitEvent(ss->st, ss->fork, 0) != cudaSuccess)
       return SLA_ERR_CUDA;
@@ -986,7 +996,12 @@ int attn_host(const void* q, const void* k, const void* v, const void* proj, voi
       cudaEventRecord(hs->ev[0], st[0]) != cudaSuccess)
     rc = SLA_ERR_CUDA;
   // heads in chunks over the streams: a chunk's copies in, operator and copy
-  // out are ordered on its stream; chunks on different streams overlap
+  // out are ordered on its stream; chunks on different streams overlap (the
+  // operator of a chunk then keeps to its chunk's stream)
+  struct OneStream {
+    OneStream() { t_one_stream = true; }
+    ~OneStream() { t_one_stream = false; }
+  } one_stream;
   long long chunks = std::min<long long>(s.BH, kHostChunks);
   if (tf != nullptr)   // a chunk's per-head counts must fit the kernels' table
     chunks = std::max<long long>(chunks, (s.BH + kMaxHeadCounts - 1) / kMaxHeadCounts);
