@@ -73,3 +73,20 @@ def test_single_process_helpers():
     assert bench.algorithmic_bytes(1, 12, 32768, 128, 256, 26) == (
         12 * 32768 * 128 * 12 + 2 * 12 * 256 * (128 * 128 + 128) * 4)
     assert bench.algorithmic_bytes(1, 12, 32768, 128, 256, 256) == 12 * 32768 * 128 * 12
+
+
+def test_bench_helpers_for_the_extended_workloads():
+    """Lists shorter than the pitch (-1 entries) count no work; the metric
+    strings name the three-class, finer-granularity and W8A8 workloads."""
+    import numpy as np
+
+    from synth import CONFIGS
+
+    idx = np.array([[[[0, 1, -1], [2, -1, -1], [0, 1, 2]]]], dtype=np.int32)
+    qk, pv = bench.critical_ops(idx, 384, 64, 128)
+    assert qk == pv == 2.0 * 64 * 128 * 128 * (2 + 1 + 3)
+    m = bench.metric_for(CONFIGS["480p_classes"])
+    assert "per head" in m and "skip 50%" in m
+    assert "scale per 32 tokens" in bench.metric_for(CONFIGS["480p_gran32"])
+    assert bench.metric_for(CONFIGS["480p"]) == bench.METRIC
+    assert bench.algorithmic_bytes(1, 12, 32768, 128, 256, 52, linear=False) == 12 * 32768 * 128 * 12
