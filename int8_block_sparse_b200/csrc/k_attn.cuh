@@ -20,7 +20,10 @@
 // the linear part alone l = 1.
 //
 // One persistent CTA per SM runs two independent pipelines ("tiles"), each
-// working on its own sequence of (head, query block) items:
+// working on its own sequence of (head, query block) items: tile u of CTA c
+// takes items c + u * G, then every 2G further (G CTAs).  In the last, partial
+// round the items fall on tile 0 of distinct CTAs, so each runs alone on its
+// SM instead of two sharing one while other SMs idle.
 //   warp 0 / 2   TMA producers of tile 0 / 1: lane 0 loads Q and K, lane 1 V
 //                and G'_i (two-stage rings; G'_i goes through the V ring as
 //                one more block; a K stage is released when its block's QK^T
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
         }
         uint32_t item_it = 0, nq = 0, nl = 0;   // nl: K loads (lane 0) or V-ring loads (lane 1)
         bool ok = true;
-        for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
+        for (int item = blockIdx.x + u * gridDim.x; item < p.items && ok; item += tiles_total, ++item_it) {
           const int bh = item / NB, i = item % NB;
           if (sparse) {
             const int kc = kc_of(bh);
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
         const uint64_t dq = smem_desc(smem_u32(tq), 16, C::KSBO, C::KSW);
         uint32_t kit = 0, vit = 0, item_it = 0, hg = 0;   // hg: halves of the items before this one
         bool ok = true;
-        for (int item = blockIdx.x * 2 + u; item < p.items && ok; item += tiles_total, ++item_it) {
+        for (int item = blockIdx.x + u * gridDim.x; item < p.items && ok; item += tiles_total, ++item_it) {
           const int H = halves_of(item / NB);
           if (sparse) {
             if (!(ok = mbar_wait(&b.q_full, item_it & 1, abort_flag))) break;
@@ -385,7 +388,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
     uint32_t hg = 0;
     bool ok = true;
     const int part_rows = p.N % BLK;                // rows of a partial last block (0: none)
-    for (int item = blockIdx.x * 2 + u; sparse && item < p.items && ok; item += tiles_total) {
+    for (int item = blockIdx.x + u * gridDim.x; sparse && item < p.items && ok; item += tiles_total) {
       const int bh = item / NB, i = item % NB;
       const int kc = kc_of(bh), H = kc * NH;
       // the scale of this row's group (rows past the block reuse the last one)
@@ -559,13 +562,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
     bool ok = true;
     int it = 0;
     auto row_of = [&](int u, int round, int& bh, int& i, long long& n) {
-      const int item = blockIdx.x * 2 + u + round * tiles_total;
+      const int item = blockIdx.x + u * gridDim.x + round * tiles_total;
       bh = item / NB;
       i = item % NB;
       n = (long long)i * BLK + r;
       return r < BLK && n < p.N;                    // a row of the output
     };
-    auto has = [&](int u, int round) { return blockIdx.x * 2 + u + round * tiles_total < p.items; };
+    // tile 1's item of a round lies G items past tile 0's, so it has one only
+    // in rounds where tile 0 has one too
+    auto has = [&](int u, int round) { return blockIdx.x + u * gridDim.x + round * tiles_total < p.items; };
     auto make_dens = [&](int round) {
 #pragma unroll
       for (int u = 0; u < 2; ++u)
@@ -580,7 +585,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) k_attn(const __grid_constant_
     // A of tile u (after its softmax); false if a wait gave up
     auto do_a = [&](int u) -> bool {
       TileBars& b = bars[u];
-      const int H = halves_of((blockIdx.x * 2 + u + it * tiles_total) / NB);
+      const int H = halves_of((blockIdx.x + u * gridDim.x + it * tiles_total) / NB);
       if (sparse) {
         if (!mbar_wait(&b.l_full, it & 1, abort_flag)) return false;
         lrow[u] = l_buf[u * 128 + r];
