@@ -1,7 +1,9 @@
 """CPU oracle for SageSLA attention -- test infrastructure only.
 
 Imported by tests/, by the package entry's smoke check and by the benchmark's
-CPU-baseline leg; never by the library.  See sla_oracle.py.
+CPU-baseline leg; never by the library.  See sla_oracle.py (the operator),
+w8a8_oracle.py (the W8A8 linear layer) and sla_backward_oracle.py (the
+gradient of the fine-tune path).
 """
 
 from . import sla_oracle  # noqa: F401
