@@ -582,17 +582,18 @@ def run_linear(args, dist):
         dt, rows = linear_oracle_sample(w, d, args.cpu_budget)
         line["cpu_baseline"] = {"value": round(2.0 * rows * w.N * w.K / dt / 1e12, 6), "unit": UNIT,
                                 "cores": oracle_threads(), "kind": "oracle",
-                                "sample": (f"W8A8 oracle (numpy, float64 BLAS for the exact integer block sums) on "
-                                           f"the first {rows} rows of X of {w.name}: their quantisation and the "
+                                "sample": (f"W8A8 oracle (plain C++, exact int32 block sums, one thread per core) "
+                                           f"on the first {rows} rows of X of {w.name}: their quantisation and the "
                                            f"block-scaled product with all N columns; value = 2 * rows * N * K / "
                                            f"wall time"), "seconds": round(dt, 2)}
     return line
 
 
 def linear_oracle_sample(w, d, budget_s):
-    """Time the W8A8 oracle on 128-row blocks of X (quantisation + product with
-    the pre-quantised weights), block 0 first, until about budget_s seconds."""
-    from oracle import w8a8_oracle as W
+    """Time the plain C++ W8A8 oracle on 128-row blocks of X (quantisation +
+    product with the pre-quantised weights), block 0 first, until about
+    budget_s seconds."""
+    from oracle import w8a8_cpp as W
 
     wq, sw = W.quantize_2d(d["w"])
     dt, rows = 0.0, 0
@@ -633,10 +634,10 @@ def run_e2e(S, t, w, args, dist):
 
 
 def run_reference_linear(args, dist):
-    """The W8A8 oracle as the reference arm: each step quantises one 128-row
-    block of X and multiplies it with the pre-quantised weights (all N
+    """The plain C++ W8A8 oracle as the reference arm: each step quantises one
+    128-row block of X and multiplies it with the pre-quantised weights (all N
     columns), the blocks taken in turn."""
-    from oracle import w8a8_oracle as W
+    from oracle import w8a8_cpp as W
     from synth.linear import LINEAR_CONFIGS, make_linear_workload
 
     w = LINEAR_CONFIGS[args.workload]
@@ -662,7 +663,7 @@ def run_reference_linear(args, dist):
     value = 2.0 * done * w.N * w.K / dt / 1e12
     ms_call = dt / max(done, 1) * w.M * 1e3
     metric = f"W8A8 linear TOPS & ms/call, M={w.M} N={w.N} K={w.K} (128x128 blocks), 1 B200 ({w.name} workload)"
-    sample = (f"W8A8 oracle (numpy), {args.steps} steps of one 128-row block of X of {w.name} "
+    sample = (f"W8A8 oracle (plain C++), {args.steps} steps of one 128-row block of X of {w.name} "
               f"(quantisation + product with all N columns)")
     return {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": UNIT, "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_call, 1),

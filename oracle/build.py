@@ -1,4 +1,5 @@
-"""Builds the plain C++ CPU oracle (libsla_oracle.so) with g++.
+"""Builds the plain C++ CPU oracles (libsla_oracle.so: the attention operator
+and the W8A8 linear layer) with g++.
 
 Test infrastructure: the library this builds is loaded only by the tests, the
 package's smoke check and the benchmark's CPU-baseline leg (through
@@ -15,18 +16,18 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "sla_oracle.cpp")
+SRCS = [os.path.join(HERE, "sla_oracle.cpp"), os.path.join(HERE, "w8a8_oracle.cpp")]
 LIB = os.path.join(HERE, "libsla_oracle.so")
 
 
 def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= max(os.path.getmtime(SRC),
-                                                                         os.path.getmtime(__file__)):
+    newest = max([os.path.getmtime(s) for s in SRCS] + [os.path.getmtime(__file__)])
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
         return LIB
     cxx = os.environ.get("CXX") or shutil.which("g++") or "g++"
     tmp = LIB + ".tmp"
     subprocess.run([cxx, "-O3", "-std=c++17", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
-                    "-fno-fast-math", "-o", tmp, SRC], check=True)
+                    "-fno-fast-math", "-o", tmp] + SRCS, check=True)
     os.replace(tmp, LIB)
     return LIB
 

@@ -90,3 +90,18 @@ def test_bench_helpers_for_the_extended_workloads():
     assert "scale per 32 tokens" in bench.metric_for(CONFIGS["480p_gran32"])
     assert bench.metric_for(CONFIGS["480p"]) == bench.METRIC
     assert bench.algorithmic_bytes(1, 12, 32768, 128, 256, 52, linear=False) == 12 * 32768 * 128 * 12
+
+
+def test_w8a8_oracle_legs_of_the_bench_run_on_the_cpu():
+    """The W8A8 workloads' CPU baseline and reference arm (plain C++ oracle)."""
+    import argparse
+
+    from synth.linear import LINEAR_CONFIGS, make_linear_workload
+
+    w = LINEAR_CONFIGS["w8a8_small"]
+    dt, rows = bench.linear_oracle_sample(w, make_linear_workload(w), 0.05)
+    assert dt > 0 and 0 < rows <= w.M
+    args = argparse.Namespace(workload="w8a8_small", steps=3, warmup=3)
+    line = bench.run_reference_linear(args, bench.Dist(1))
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert "plain C++" in line["cpu_baseline"]["sample"]
