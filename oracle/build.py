@@ -1,5 +1,5 @@
-"""Builds the plain C++ CPU oracles (libsla_oracle.so: the attention operator
-and the W8A8 linear layer) with g++.
+"""Builds the plain C++ CPU oracles (libsla_oracle.so: the attention operator,
+the W8A8 linear layer and the gradient of the fine-tune path) with g++.
 
 Test infrastructure: the library this builds is loaded only by the tests, the
 package's smoke check and the benchmark's CPU-baseline leg (through
@@ -16,7 +16,7 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRCS = [os.path.join(HERE, "sla_oracle.cpp"), os.path.join(HERE, "w8a8_oracle.cpp")]
+SRCS = [os.path.join(HERE, f) for f in ("sla_oracle.cpp", "w8a8_oracle.cpp", "sla_backward_oracle.cpp")]
 LIB = os.path.join(HERE, "libsla_oracle.so")
 
 
