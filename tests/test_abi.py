@@ -205,3 +205,23 @@ def test_granularity_entry_points_refuse_invalid_arguments_without_a_gpu():
                            None) == 2
     assert L.sla_attn_gran(dummy, dummy, dummy, dummy, dummy, 3, None, None, 1, 1, 128, 128, 64, f(0.1), 32,
                            None) == 1
+
+
+def test_product_path_has_no_cpu_fallback(monkeypatch, tmp_path):
+    """Without libsla.so the binding raises instead of computing anything, and
+    no product source imports, loads or names the CPU oracle."""
+    import pathlib
+
+    import int8_block_sparse_b200 as S
+
+    monkeypatch.setattr(S, "_lib", None)
+    monkeypatch.setattr(S, "LIB_PATH", str(tmp_path / "missing" / "libsla.so"))
+    with pytest.raises(ImportError, match="missing"):
+        S.lib()
+    with pytest.raises(ImportError):
+        S.topk_count(1024, 128, 0.1)
+    root = pathlib.Path(S.__file__).parent
+    for f in list(root.rglob("*.py")) + list(root.rglob("*.cu")) + list(root.rglob("*.cuh")) + \
+            list((root.parent / "include").glob("*.h")):
+        text = f.read_text()
+        assert "oracle" not in text, f
